@@ -1,0 +1,397 @@
+// C ABI entry points: host-side validation, workspace planning and launch
+// orchestration.  Nothing is launched unless every check passes.
+#include <cmath>
+#include <cstring>
+
+#include "kernels.cuh"
+
+namespace lla {
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr int kTargetCtas = 4 * 148;   // split heuristics aim at ~4 CTAs per SM
+constexpr size_t kAlign = 256;
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t elem_size(int dt) { return dt == LLA_BF16 ? 2 : 4; }
+inline bool dtype_ok(int dt) { return dt == LLA_F32 || dt == LLA_BF16; }
+inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Carve {
+  size_t off = 0;
+  size_t take(size_t bytes) { size_t o = off; off = round_up(off + bytes); return o; }
+};
+
+inline int ring_ok(int W, int N, int Wcap) {
+  const long need = (long)std::min<long>(W, (long)N - 1) + 1;
+  return Wcap >= need;
+}
+
+// --------------------------------------------------------------- writer --
+int check_write(const lla_write_params& p) {
+  if (p.B < 0 || p.n < 0 || p.pos0 < 0 || p.Ncap < 0) return LLA_ERR_SHAPE;
+  if (!dtype_ok(p.out_dtype)) return LLA_ERR_DTYPE;
+  if (p.mode != LLA_WRITE_HLA && p.mode != LLA_WRITE_PERHEAD && p.mode != LLA_WRITE_FOLDED)
+    return LLA_ERR_UNSUPPORTED;
+  if (p.T < 1 || p.H < 1 || p.d_h < 2) return LLA_ERR_SHAPE;
+  if ((long)p.pos0 + p.n > p.Ncap) return LLA_ERR_SHAPE;
+  const int mult = p.out_dtype == LLA_BF16 ? 8 : 4;
+  if (p.mode == LLA_WRITE_HLA) {
+    if (p.T < 2 || p.D < 16 || p.D % 16) return LLA_ERR_SHAPE;
+    if (p.r_k < 2 || p.r_v < 1 || p.r_1 < 1) return LLA_ERR_SHAPE;
+    if (p.r_k % 2 || p.r_1 % 2 || p.d_h % 2) return LLA_ERR_SHAPE;
+    if ((p.r_k + p.r_v) % mult || (2 * p.r_1) % mult) return LLA_ERR_ALIGN;
+  } else {
+    if (p.d_h % 16) return LLA_ERR_SHAPE;
+    if (p.r_k < 1 || p.r_v < 1) return LLA_ERR_SHAPE;
+    if (p.mode == LLA_WRITE_PERHEAD && (p.r_k != p.r_v)) return LLA_ERR_SHAPE;
+    if (p.mode == LLA_WRITE_PERHEAD && (p.r_k % mult)) return LLA_ERR_ALIGN;
+    if (p.mode == LLA_WRITE_FOLDED && ((p.r_k + p.r_v) % mult || p.r_k % 2)) return LLA_ERR_ALIGN;
+  }
+  if (p.B == 0 || p.n == 0) return LLA_OK;
+  if (!p.x || !p.out0) return LLA_ERR_NULL;
+  if (p.mode == LLA_WRITE_HLA && (!p.E_main || !p.E_1 || !p.out1)) return LLA_ERR_NULL;
+  if (p.mode != LLA_WRITE_HLA && (!p.xv || !p.E_K || !p.E_V)) return LLA_ERR_NULL;
+  if (p.mode == LLA_WRITE_PERHEAD && !p.out1) return LLA_ERR_NULL;
+  const size_t es = elem_size(p.out_dtype);
+  if (!aligned(p.out0, 16) || (p.out1 && !aligned(p.out1, 16))) return LLA_ERR_ALIGN;
+  if ((p.out_stride_b * es) % 16 || (p.out_stride_n * es) % 16) return LLA_ERR_ALIGN;
+  if (p.mode == LLA_WRITE_PERHEAD && (p.out_stride_h * es) % 16) return LLA_ERR_ALIGN;
+  if (p.mode == LLA_WRITE_HLA && ((p.out1_stride_b * es) % 16 || (p.out1_stride_n * es) % 16))
+    return LLA_ERR_ALIGN;
+  if (!aligned(p.x, 4) || (p.xv && !aligned(p.xv, 4))) return LLA_ERR_ALIGN;
+  if (p.x_stride_b < 0 || p.x_stride_n < 0 || p.x_stride_t < 0) return LLA_ERR_SHAPE;
+  const int64_t row = p.mode == LLA_WRITE_HLA ? (int64_t)p.D : (int64_t)p.H * p.d_h;
+  if (p.x_stride_t < row) return LLA_ERR_SHAPE;
+  if (p.mode == LLA_WRITE_HLA) {
+    if (p.out_stride_n < p.r_k + p.r_v || p.out1_stride_n < 2 * p.r_1) return LLA_ERR_SHAPE;
+  } else if (p.mode == LLA_WRITE_PERHEAD) {
+    if (p.out_stride_n < p.r_k) return LLA_ERR_SHAPE;
+  } else if (p.out_stride_n < p.r_k + p.r_v) {
+    return LLA_ERR_SHAPE;
+  }
+  return LLA_OK;
+}
+
+WriterArgs writer_args(const lla_write_params& p) {
+  WriterArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.mode = p.mode; a.B = p.B; a.n_tok = p.n; a.pos0 = p.pos0; a.T = p.T; a.H = p.H;
+  a.d_h = p.d_h; a.D = p.D; a.r_k = p.r_k; a.r_v = p.r_v; a.r_1 = p.r_1;
+  a.rotate = p.mode == LLA_WRITE_HLA ? (p.rotate_keys != 0) : 0;
+  a.base = p.rope_base;
+  a.x = p.x; a.xv = p.xv; a.xs_b = p.x_stride_b; a.xs_n = p.x_stride_n; a.xs_t = p.x_stride_t;
+  a.E_main = p.E_main; a.E_1 = p.E_1; a.E_K = p.E_K; a.E_V = p.E_V;
+  a.out0 = p.out0; a.out1 = p.out1; a.dtype = p.out_dtype;
+  a.os_b = p.out_stride_b; a.os_h = p.out_stride_h; a.os_n = p.out_stride_n;
+  a.o1s_b = p.out1_stride_b; a.o1s_n = p.out1_stride_n;
+  a.M = p.B * p.n;
+  if (p.mode == LLA_WRITE_HLA) {
+    a.Z = 2; a.Nmax = std::max(p.r_k + p.r_v, 2 * p.r_1);
+  } else if (p.mode == LLA_WRITE_PERHEAD) {
+    a.Z = 2 * p.H; a.Nmax = std::max(p.r_k, p.r_v);
+  } else {
+    a.Z = 2; a.Nmax = std::max(p.r_k, p.r_v);
+  }
+  a.Nmax += a.Nmax % 2;
+  a.S = writer_pick_splits(a, 148);
+  return a;
+}
+
+// ------------------------------------------------------- decode checks --
+int check_hla(const hla_decode_params& p) {
+  if (p.B < 0 || p.nt < 0) return LLA_ERR_SHAPE;
+  if (!dtype_ok(p.lat_dtype) || !dtype_ok(p.win_dtype)) return LLA_ERR_DTYPE;
+  if (p.H < 1 || p.d_h < 2 || p.d_h % 2 || p.T < 1 || p.t0 < 0 || p.t0 + p.nt > p.T) return LLA_ERR_SHAPE;
+  if (p.N < 1 || p.W < 0 || p.r_k < 2 || p.r_k % 2 || p.r_v < 1) return LLA_ERR_SHAPE;
+  if (p.d_h > 128) return LLA_ERR_UNSUPPORTED;
+  if (p.r_v > 1024 || p.r_k + p.r_v > 2048) return LLA_ERR_UNSUPPORTED;
+  if ((long)p.nt * p.H > 65535) return LLA_ERR_UNSUPPORTED;
+  if (!ring_ok(p.W, p.N, p.Wcap)) return LLA_ERR_SHAPE;
+  if (!std::isfinite(p.scale) || p.scale < 0.f) return LLA_ERR_SHAPE;
+  if (p.B == 0 || p.nt == 0) return LLA_OK;
+  const int n_lat = std::max(0, p.N - 1 - p.W);
+  if (!p.A || !p.Bm || !p.q || !p.win_k || !p.win_v || !p.out) return LLA_ERR_NULL;
+  if (n_lat > 0 && !p.lat) return LLA_ERR_NULL;
+  const size_t es = elem_size(p.lat_dtype);
+  if (n_lat > 0) {
+    if (!aligned(p.lat, 16) || (p.lat_stride_b * es) % 16 || (p.lat_stride_n * es) % 16) return LLA_ERR_ALIGN;
+    if (((size_t)(p.r_k + p.r_v) * es) % 16 || ((size_t)p.r_k * es) % 16) return LLA_ERR_ALIGN;
+    if (p.lat_stride_n < p.r_k + p.r_v || p.lat_stride_b < 0) return LLA_ERR_SHAPE;
+  }
+  if (!aligned(p.A, 16) || !aligned(p.Bm, 16) || p.r_k % 4) return LLA_ERR_ALIGN;
+  if (!aligned(p.q, 4) || !aligned(p.out, 4)) return LLA_ERR_ALIGN;
+  if (!aligned(p.win_k, 16) || !aligned(p.win_v, 16)) return LLA_ERR_ALIGN;
+  const int64_t rowlen = (int64_t)p.nt * p.H * p.d_h;
+  if (p.q_stride_b < rowlen || p.out_stride_b < rowlen) return LLA_ERR_SHAPE;
+  if (p.win_stride_b < (int64_t)p.T * p.Wcap * p.H * p.d_h) return LLA_ERR_SHAPE;
+  return LLA_OK;
+}
+
+int check_lla(const lla_decode_params& p) {
+  if (p.B < 0 || p.nt < 0) return LLA_ERR_SHAPE;
+  if (!dtype_ok(p.lat_dtype) || !dtype_ok(p.win_dtype)) return LLA_ERR_DTYPE;
+  if (p.H < 1 || p.d_h < 1 || p.T < 1 || p.t0 < 0 || p.t0 + p.nt > p.T) return LLA_ERR_SHAPE;
+  if (p.N < 1 || p.W < 0 || p.r < 1) return LLA_ERR_SHAPE;
+  if (p.d_h > 128 || p.r > 128) return LLA_ERR_UNSUPPORTED;
+  if ((long)p.nt * p.H > 65535) return LLA_ERR_UNSUPPORTED;
+  if (!ring_ok(p.W, p.N, p.Wcap)) return LLA_ERR_SHAPE;
+  if (!std::isfinite(p.scale) || p.scale < 0.f) return LLA_ERR_SHAPE;
+  if (p.B == 0 || p.nt == 0) return LLA_OK;
+  const int n_lat = std::max(0, p.N - 1 - p.W);
+  if (!p.UK || !p.UV || !p.q || !p.win_k || !p.win_v || !p.out) return LLA_ERR_NULL;
+  if (n_lat > 0 && (!p.cK || !p.cV)) return LLA_ERR_NULL;
+  const size_t es = elem_size(p.lat_dtype);
+  if (n_lat > 0) {
+    if (!aligned(p.cK, 16) || !aligned(p.cV, 16)) return LLA_ERR_ALIGN;
+    if ((p.lat_stride_b * es) % 16 || (p.lat_stride_h * es) % 16 || ((size_t)p.r * es) % 16) return LLA_ERR_ALIGN;
+    if (p.lat_stride_h < (int64_t)n_lat * p.r || p.lat_stride_b < 0) return LLA_ERR_SHAPE;
+  }
+  if (!aligned(p.UK, 16) || !aligned(p.UV, 16)) return LLA_ERR_ALIGN;
+  if (!aligned(p.q, 4) || !aligned(p.out, 4)) return LLA_ERR_ALIGN;
+  if (!aligned(p.win_k, 16) || !aligned(p.win_v, 16)) return LLA_ERR_ALIGN;
+  const int64_t rowlen = (int64_t)p.nt * p.H * p.d_h;
+  if (p.q_stride_b < rowlen || p.out_stride_b < rowlen) return LLA_ERR_SHAPE;
+  if (p.win_stride_b < (int64_t)p.T * p.Wcap * p.H * p.d_h) return LLA_ERR_SHAPE;
+  return LLA_OK;
+}
+
+// Workspace layout of the absorbed read.
+struct HlaPlan {
+  int rows, n_lat, win_start, n_win, S, tps;
+  size_t o_qlat, o_qwin, o_pml, o_py, o_wml, o_wy, bytes;
+};
+
+HlaPlan plan_hla(const hla_decode_params& p) {
+  HlaPlan pl;
+  // SIMT split: one CTA per (split, sequence, 16 rows)
+  pl.rows = p.nt * p.H;
+  const int i = p.N - 1;
+  pl.n_lat = std::max(0, i - p.W);
+  pl.win_start = pl.n_lat;
+  pl.n_win = i - pl.win_start + 1;
+  if (pl.n_lat > 0) {
+    const long ctas = (long)p.B * ((pl.rows + 15) / 16);
+    long S = (kTargetCtas + ctas - 1) / ctas;
+    const long tiles = (pl.n_lat + 15) / 16;
+    S = std::max(1L, std::min(S, tiles));
+    pl.tps = (int)(((pl.n_lat + S - 1) / S + 15) / 16 * 16);
+    pl.S = (pl.n_lat + pl.tps - 1) / pl.tps;
+  } else {
+    pl.S = 0; pl.tps = 0;
+  }
+  const size_t br = (size_t)p.B * pl.rows;
+  Carve c;
+  pl.o_qlat = c.take(br * p.r_k * 4);
+  pl.o_qwin = c.take(br * p.d_h * 4);
+  pl.o_pml = c.take((size_t)pl.S * br * 2 * 4);
+  pl.o_py = c.take((size_t)pl.S * br * p.r_v * 4);
+  pl.o_wml = c.take(br * 2 * 4);
+  pl.o_wy = c.take(br * p.d_h * 4);
+  pl.bytes = c.off;
+  return pl;
+}
+
+HlaPlan plan_lla(const lla_decode_params& p) {
+  HlaPlan pl;
+  pl.rows = p.nt * p.H;
+  const int i = p.N - 1;
+  pl.n_lat = std::max(0, i - p.W);
+  pl.win_start = pl.n_lat;
+  pl.n_win = i - pl.win_start + 1;
+  if (pl.n_lat > 0) {
+    const long ctas = (long)p.B * pl.rows;
+    long S = (kTargetCtas + ctas - 1) / ctas;
+    const long tiles = (pl.n_lat + 31) / 32;
+    S = std::max(1L, std::min(S, tiles));
+    pl.tps = (int)(((pl.n_lat + S - 1) / S + 31) / 32 * 32);
+    pl.S = (pl.n_lat + pl.tps - 1) / pl.tps;
+  } else {
+    pl.S = 0; pl.tps = 0;
+  }
+  const size_t br = (size_t)p.B * pl.rows;
+  Carve c;
+  pl.o_qlat = 0;
+  pl.o_qwin = 0;
+  pl.o_pml = c.take((size_t)pl.S * br * 2 * 4);
+  pl.o_py = c.take((size_t)pl.S * br * p.d_h * 4);
+  pl.o_wml = c.take(br * 2 * 4);
+  pl.o_wy = c.take(br * p.d_h * 4);
+  pl.bytes = c.off;
+  return pl;
+}
+
+int ws_ok(void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return LLA_OK;
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < need) return LLA_ERR_WORKSPACE;
+  return LLA_OK;
+}
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? LLA_OK : LLA_ERR_CUDA; }
+
+// Optional measurement hook: record caller-owned event i (0 = before, 1 = after
+// the latent-read kernel) on the stream; captured as an external event node.
+inline cudaError_t mark(void* events, int i, cudaStream_t s) {
+  if (!events) return cudaSuccess;
+  cudaEvent_t ev = reinterpret_cast<cudaEvent_t*>(events)[i];
+  return cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+}
+
+}  // namespace
+}  // namespace lla
+
+using namespace lla;
+
+extern "C" {
+
+int lla_abi_version(void) { return kAbiVersion; }
+
+const char* lla_status_str(int s) {
+  switch (s) {
+    case LLA_OK: return "ok";
+    case LLA_ERR_NULL: return "a required pointer is NULL";
+    case LLA_ERR_SHAPE: return "sizes are out of range or inconsistent";
+    case LLA_ERR_DTYPE: return "unknown dtype code";
+    case LLA_ERR_ALIGN: return "pointer or stride breaks the 16-byte alignment rule";
+    case LLA_ERR_WORKSPACE: return "workspace is NULL, misaligned or too small";
+    case LLA_ERR_UNSUPPORTED: return "valid arguments outside what this build supports";
+    case LLA_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    default: return "unknown status";
+  }
+}
+
+size_t lla_write_workspace_bytes(const lla_write_params* p) {
+  if (!p || check_write(*p) != LLA_OK) return 0;
+  if (p->B == 0 || p->n == 0) return 0;
+  const WriterArgs a = writer_args(*p);
+  return round_up(writer_workspace_floats(a) * sizeof(float));
+}
+
+int lla_write_latents(const lla_write_params* p, void* ws, size_t ws_bytes, lla_stream stream) {
+  if (!p) return LLA_ERR_NULL;
+  int st = check_write(*p);
+  if (st != LLA_OK) return st;
+  if (p->B == 0 || p->n == 0) return LLA_OK;
+  WriterArgs a = writer_args(*p);
+  const size_t need = round_up(writer_workspace_floats(a) * sizeof(float));
+  st = ws_ok(ws, ws_bytes, need);
+  if (st != LLA_OK) return st;
+  a.part = reinterpret_cast<float*>(ws);
+  return cuda_status(launch_writer(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t hla_decode_workspace_bytes(const hla_decode_params* p) {
+  if (!p || check_hla(*p) != LLA_OK || p->B == 0 || p->nt == 0) return 0;
+  return plan_hla(*p).bytes;
+}
+
+int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_stream stream) {
+  if (!p) return LLA_ERR_NULL;
+  int st = check_hla(*p);
+  if (st != LLA_OK) return st;
+  if (p->B == 0 || p->nt == 0) return LLA_OK;
+  const HlaPlan pl = plan_hla(*p);
+  st = ws_ok(ws, ws_bytes, pl.bytes);
+  if (st != LLA_OK) return st;
+  char* w = reinterpret_cast<char*>(ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  AbsorbArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = p->B; a.H = p->H; a.d_h = p->d_h; a.T = p->T; a.t0 = p->t0; a.nt = p->nt;
+  a.N = p->N; a.W = p->W; a.r_k = p->r_k; a.r_v = p->r_v; a.rows = pl.rows;
+  a.n_lat = pl.n_lat; a.win_start = pl.win_start; a.n_win = pl.n_win;
+  a.lat = p->lat; a.lat_dtype = p->lat_dtype; a.ls_b = p->lat_stride_b; a.ls_n = p->lat_stride_n;
+  a.A = p->A; a.Bm = p->Bm; a.q = p->q; a.qs_b = p->q_stride_b;
+  a.rotate = p->rotate_query != 0; a.base = p->rope_base;
+  a.wk = p->win_k; a.wv = p->win_v; a.win_dtype = p->win_dtype; a.Wcap = p->Wcap; a.wins_b = p->win_stride_b;
+  a.out = p->out; a.outs_b = p->out_stride_b;
+  const float scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt((float)p->d_h);
+  a.qmul = scale * kLog2e;
+  a.qlat = reinterpret_cast<float*>(w + pl.o_qlat);
+  a.qwin = reinterpret_cast<float*>(w + pl.o_qwin);
+  a.part_ml = reinterpret_cast<float*>(w + pl.o_pml);
+  a.part_y = reinterpret_cast<float*>(w + pl.o_py);
+  a.win_ml = reinterpret_cast<float*>(w + pl.o_wml);
+  a.win_y = reinterpret_cast<float*>(w + pl.o_wy);
+  a.S = pl.S; a.tps = pl.tps;
+
+  cudaError_t e = launch_absorb_prologue(a, s);
+  if (e == cudaSuccess) e = mark(p->timing_events, 0, s);
+  if (e == cudaSuccess && a.n_lat > 0) e = launch_absorb_split_simt(a, s);
+  if (e == cudaSuccess) e = mark(p->timing_events, 1, s);
+  if (e == cudaSuccess) {
+    WindowArgs wa;
+    wa.B = a.B; wa.rows = a.rows; wa.H = a.H; wa.d_h = a.d_h; wa.t0 = a.t0; wa.Wcap = a.Wcap;
+    wa.win_start = a.win_start; wa.n_win = a.n_win; wa.wk = a.wk; wa.wv = a.wv;
+    wa.dtype = a.win_dtype; wa.wins_b = a.wins_b;
+    wa.q = a.qwin; wa.q_sb = (int64_t)a.rows * a.d_h; wa.q_srow = a.d_h; wa.qmul = 1.f;
+    wa.win_ml = a.win_ml; wa.win_y = a.win_y;
+    e = launch_window(wa, s);
+  }
+  if (e == cudaSuccess) {
+    MergeArgs g;
+    g.B = a.B; g.rows = a.rows; g.H = a.H; g.d_h = a.d_h; g.S = a.S; g.Y = a.r_v;
+    g.part_ml = a.part_ml; g.part_y = a.part_y; g.win_ml = a.win_ml; g.win_y = a.win_y;
+    g.Bm = a.Bm; g.out = a.out; g.outs_b = a.outs_b;
+    e = launch_merge(g, s);
+  }
+  return cuda_status(e);
+}
+
+size_t lla_decode_workspace_bytes(const lla_decode_params* p) {
+  if (!p || check_lla(*p) != LLA_OK || p->B == 0 || p->nt == 0) return 0;
+  return plan_lla(*p).bytes;
+}
+
+int lla_decode_attn(const lla_decode_params* p, void* ws, size_t ws_bytes, lla_stream stream) {
+  if (!p) return LLA_ERR_NULL;
+  int st = check_lla(*p);
+  if (st != LLA_OK) return st;
+  if (p->B == 0 || p->nt == 0) return LLA_OK;
+  const HlaPlan pl = plan_lla(*p);
+  st = ws_ok(ws, ws_bytes, pl.bytes);
+  if (st != LLA_OK) return st;
+  char* w = reinterpret_cast<char*>(ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const float scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt((float)p->d_h);
+
+  ReconArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = p->B; a.H = p->H; a.d_h = p->d_h; a.r = p->r; a.T = p->T; a.t0 = p->t0; a.nt = p->nt;
+  a.N = p->N; a.W = p->W; a.rows = pl.rows;
+  a.n_lat = pl.n_lat; a.win_start = pl.win_start; a.n_win = pl.n_win;
+  a.cK = p->cK; a.cV = p->cV; a.lat_dtype = p->lat_dtype; a.ls_b = p->lat_stride_b; a.ls_h = p->lat_stride_h;
+  a.UK = p->UK; a.UV = p->UV; a.q = p->q; a.qs_b = p->q_stride_b;
+  a.wk = p->win_k; a.wv = p->win_v; a.win_dtype = p->win_dtype; a.Wcap = p->Wcap; a.wins_b = p->win_stride_b;
+  a.out = p->out; a.outs_b = p->out_stride_b;
+  a.qmul = scale * kLog2e;
+  a.part_ml = reinterpret_cast<float*>(w + pl.o_pml);
+  a.part_y = reinterpret_cast<float*>(w + pl.o_py);
+  a.win_ml = reinterpret_cast<float*>(w + pl.o_wml);
+  a.win_y = reinterpret_cast<float*>(w + pl.o_wy);
+  a.S = pl.S; a.tps = pl.tps;
+
+  cudaError_t e = mark(p->timing_events, 0, s);
+  if (e == cudaSuccess && a.n_lat > 0) e = launch_recon_split_simt(a, s);
+  if (e == cudaSuccess) e = mark(p->timing_events, 1, s);
+  if (e == cudaSuccess) {
+    WindowArgs wa;
+    wa.B = a.B; wa.rows = a.rows; wa.H = a.H; wa.d_h = a.d_h; wa.t0 = a.t0; wa.Wcap = a.Wcap;
+    wa.win_start = a.win_start; wa.n_win = a.n_win; wa.wk = a.wk; wa.wv = a.wv;
+    wa.dtype = a.win_dtype; wa.wins_b = a.wins_b;
+    wa.q = a.q; wa.q_sb = a.qs_b; wa.q_srow = a.d_h; wa.qmul = a.qmul;
+    wa.win_ml = a.win_ml; wa.win_y = a.win_y;
+    e = launch_window(wa, s);
+  }
+  if (e == cudaSuccess) {
+    MergeArgs g;
+    g.B = a.B; g.rows = a.rows; g.H = a.H; g.d_h = a.d_h; g.S = a.S; g.Y = a.d_h;
+    g.part_ml = a.part_ml; g.part_y = a.part_y; g.win_ml = a.win_ml; g.win_y = a.win_y;
+    g.Bm = nullptr; g.out = a.out; g.outs_b = a.outs_b;
+    e = launch_merge(g, s);
+  }
+  return cuda_status(e);
+}
+
+}  // extern "C"

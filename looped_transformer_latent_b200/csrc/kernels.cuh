@@ -1,0 +1,100 @@
+// Internal launch interface between the C ABI layer (abi.cu) and the kernels.
+// Argument structs are passed by value as kernel parameters.
+#pragma once
+
+#include "common.cuh"
+
+namespace lla {
+
+// ---------------------------------------------------------------- writer --
+struct WriterArgs {
+  int mode, B, n_tok, pos0, T, H, d_h, D, r_k, r_v, r_1, rotate;
+  double base;
+  const float *x, *xv;
+  int64_t xs_b, xs_n, xs_t;
+  const float *E_main, *E_1, *E_K, *E_V;
+  void *out0, *out1;
+  int dtype;
+  int64_t os_b, os_h, os_n, o1s_b, o1s_n;
+  int M;       // B * n_tok
+  int Z;       // independent GEMMs (HLA: 2; PERHEAD: 2H; FOLDED: 2)
+  int Nmax;    // largest output width over the Z GEMMs
+  int S;       // split-K factor
+  float* part; // [Z][S][M][Nmax] fp32 partial sums
+};
+size_t writer_workspace_floats(const WriterArgs& a);
+int writer_pick_splits(const WriterArgs& a, int num_sms);
+cudaError_t launch_writer(const WriterArgs& a, cudaStream_t st);
+
+// ------------------------------------------------------ absorbed decode --
+struct AbsorbArgs {
+  int B, H, d_h, T, t0, nt, N, W, r_k, r_v, rows;
+  int n_lat, win_start, n_win;
+  const void* lat;
+  int lat_dtype;
+  int64_t ls_b, ls_n;
+  const float *A, *Bm, *q;
+  int64_t qs_b;
+  int rotate;
+  double base;
+  const void *wk, *wv;
+  int win_dtype, Wcap;
+  int64_t wins_b;
+  float* out;
+  int64_t outs_b;
+  float qmul;          // scale * log2(e): scores are kept in base-2 units
+  // workspace views
+  float *qlat;         // [B][rows][r_k]  (scaled, rotated)
+  float *qwin;         // [B][rows][d_h]  (scaled, rotated)
+  float *part_ml;      // [S][B][rows][2] (running max, sum) per split
+  float *part_y;       // [S][B][rows][r_v]
+  float *win_ml;       // [B][rows][2]
+  float *win_y;        // [B][rows][d_h]
+  int S, tps;          // splits of the latent range, tokens per split
+};
+
+// ------------------------------------------------- reconstruct decode --
+struct ReconArgs {
+  int B, H, d_h, r, T, t0, nt, N, W, rows;
+  int n_lat, win_start, n_win;
+  const void *cK, *cV;
+  int lat_dtype;
+  int64_t ls_b, ls_h;
+  const float *UK, *UV, *q;
+  int64_t qs_b;
+  const void *wk, *wv;
+  int win_dtype, Wcap;
+  int64_t wins_b;
+  float* out;
+  int64_t outs_b;
+  float qmul;
+  float *part_ml, *part_y, *win_ml, *win_y;
+  int S, tps;
+};
+
+// Shared pieces.
+struct WindowArgs {
+  int B, rows, H, d_h, t0, Wcap, win_start, n_win;
+  const void *wk, *wv;
+  int dtype;
+  int64_t wins_b;
+  const float* q;
+  int64_t q_sb, q_srow;
+  float qmul;
+  float *win_ml, *win_y;
+};
+struct MergeArgs {
+  int B, rows, H, d_h, S, Y;
+  const float *part_ml, *part_y, *win_ml, *win_y;
+  const float* Bm;   // [rows][Y][d_h] when mapping latent space back; else null
+  float* out;
+  int64_t outs_b;
+};
+
+cudaError_t launch_absorb_prologue(const AbsorbArgs& a, cudaStream_t st);
+cudaError_t launch_absorb_split_simt(const AbsorbArgs& a, cudaStream_t st);
+cudaError_t launch_window(const WindowArgs& w, cudaStream_t st);
+cudaError_t launch_merge(const MergeArgs& m, cudaStream_t st);
+cudaError_t launch_recon_split_simt(const ReconArgs& a, cudaStream_t st);
+
+}  // namespace lla

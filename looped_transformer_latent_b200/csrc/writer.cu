@@ -1,0 +1,199 @@
+// Latent writer: HLA eq. 2 and the LLA per-head / LLA-2D encoders.
+//
+// Every mode is a set of Z independent GEMMs out[m][n] = sum_k X(m,k) E(n,k)
+// with m = (sequence, token) and k = (loop[, head], feature).  Phase 1 is a
+// split-K SIMT fp32 GEMM writing partial sums to the workspace; phase 2 adds
+// the partials in a fixed order (deterministic), rotates key pairs by
+// R~_pos (HLA), rounds once to the storage type and stores the cache rows.
+#include "kernels.cuh"
+
+namespace lla {
+namespace {
+
+constexpr int BM = 64, BN = 64, BK = 16, WT = 256;
+
+struct Slice {
+  const float* X;
+  int64_t x_o_t, x_o_h;
+  int o_h;
+  const float* E;
+  int64_t e_o, e_n;
+  int K_outer, d_in, N;
+  void* out;
+  int64_t os_b, os_n, col0;
+  int rot_dim;
+};
+
+__device__ __forceinline__ Slice slice_of(const WriterArgs& a, int z) {
+  Slice s;
+  if (a.mode == LLA_WRITE_HLA) {
+    if (z == 0) {  // c_j = sum_{t=2..T} E_t h_{j,t}
+      s.X = a.x + a.xs_t; s.x_o_t = a.xs_t; s.x_o_h = 0; s.o_h = 1;
+      s.N = a.r_k + a.r_v;
+      s.E = a.E_main; s.e_o = (int64_t)s.N * a.D; s.e_n = a.D;
+      s.K_outer = a.T - 1; s.d_in = a.D;
+      s.out = a.out0; s.os_b = a.os_b; s.os_n = a.os_n; s.col0 = 0;
+      s.rot_dim = a.rotate ? a.r_k : 0;
+    } else {       // c^(1)_j = E_1 h_{j,1}
+      s.X = a.x; s.x_o_t = 0; s.x_o_h = 0; s.o_h = 1;
+      s.N = 2 * a.r_1;
+      s.E = a.E_1; s.e_o = 0; s.e_n = a.D;
+      s.K_outer = 1; s.d_in = a.D;
+      s.out = a.out1; s.os_b = a.o1s_b; s.os_n = a.o1s_n; s.col0 = 0;
+      s.rot_dim = a.rotate ? a.r_1 : 0;
+    }
+  } else if (a.mode == LLA_WRITE_PERHEAD) {  // c_{j,h} = sum_t E_{t,h} k_{j,t,h}
+    const int part = z / a.H, h = z % a.H;
+    const int r = part ? a.r_v : a.r_k;
+    s.X = (part ? a.xv : a.x) + (int64_t)h * a.d_h; s.x_o_t = a.xs_t; s.x_o_h = 0; s.o_h = 1;
+    s.N = r;
+    s.E = (part ? a.E_V : a.E_K) + (int64_t)h * r * a.d_h;
+    s.e_o = (int64_t)a.H * r * a.d_h; s.e_n = a.d_h;
+    s.K_outer = a.T; s.d_in = a.d_h;
+    s.out = part ? a.out1 : a.out0; s.os_b = a.os_b; s.os_n = a.os_n;
+    s.col0 = (int64_t)h * a.os_h;
+    s.rot_dim = 0;
+  } else {  // FOLDED: c_j = sum_{t,h} E_{t,h} k_{j,t,h}
+    const int part = z;
+    const int r = part ? a.r_v : a.r_k;
+    s.X = part ? a.xv : a.x; s.x_o_t = a.xs_t; s.x_o_h = a.d_h; s.o_h = a.H;
+    s.N = r;
+    s.E = part ? a.E_V : a.E_K; s.e_o = (int64_t)r * a.d_h; s.e_n = a.d_h;
+    s.K_outer = a.T * a.H; s.d_in = a.d_h;
+    s.out = a.out0; s.os_b = a.os_b; s.os_n = a.os_n; s.col0 = part ? a.r_k : 0;
+    s.rot_dim = 0;
+  }
+  return s;
+}
+
+// Phase 1: C_part[z][split][m][n] = sum over this split's k-chunks.
+__global__ void __launch_bounds__(WT) writer_gemm(WriterArgs a) {
+  const int z = blockIdx.z / a.S, split = blockIdx.z % a.S;
+  const Slice s = slice_of(a, z);
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  if (n0 >= s.N) return;
+  const int K = s.K_outer * s.d_in;
+  const int nk = K / BK;
+  const int kc0 = (int)((int64_t)nk * split / a.S), kc1 = (int)((int64_t)nk * (split + 1) / a.S);
+
+  __shared__ float As[BK][BM + 4];
+  __shared__ float Bs[BK][BN + 4];
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  float acc[4][4] = {};
+
+  // loader mapping: 64 rows x 16 k = 1024 values, 4 per thread
+  const int lr = tid / 4, lk = (tid % 4) * 4;
+  const int m = m0 + lr;
+  const bool mval = m < a.M;
+  int64_t xrow = 0;
+  if (mval) {
+    const int b = m / a.n_tok, j = m % a.n_tok;
+    xrow = (int64_t)b * a.xs_b + (int64_t)j * a.xs_n;
+  }
+  const int n = n0 + lr;
+  const bool nval = n < s.N;
+
+  for (int kc = kc0; kc < kc1; ++kc) {
+    const int k = kc * BK;
+    const int o = k / s.d_in, d = k % s.d_in + lk;
+    const int64_t xo = (int64_t)(o / s.o_h) * s.x_o_t + (int64_t)(o % s.o_h) * s.x_o_h;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      As[lk + u][lr] = mval ? __ldg(s.X + xrow + xo + d + u) : 0.f;
+      Bs[lk + u][lr] = nval ? __ldg(s.E + (int64_t)o * s.e_o + (int64_t)n * s.e_n + d + u) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < BK; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bv[i] = Bs[kk][tx * 4 + i];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) acc[i][jj] = fmaf(av[i], bv[jj], acc[i][jj]);
+    }
+    __syncthreads();
+  }
+  float* P = a.part + ((int64_t)(z * a.S + split) * a.M) * a.Nmax;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int mm = m0 + ty * 4 + i;
+    if (mm >= a.M) continue;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int nn = n0 + tx * 4 + jj;
+      if (nn < s.N) P[(int64_t)mm * a.Nmax + nn] = acc[i][jj];
+    }
+  }
+}
+
+// Phase 2: ordered sum of the splits, rotation of key pairs, rounding, store.
+__global__ void writer_epilogue(WriterArgs a) {
+  const int64_t pairs = a.Nmax / 2;
+  const int64_t total = (int64_t)a.Z * a.M * pairs;
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int p = (int)(idx % pairs);
+    const int m = (int)((idx / pairs) % a.M);
+    const int z = (int)(idx / (pairs * a.M));
+    const Slice s = slice_of(a, z);
+    const int n = 2 * p;
+    if (n >= s.N) continue;
+    float x = 0.f, y = 0.f;
+    for (int sp = 0; sp < a.S; ++sp) {
+      const float* P = a.part + ((int64_t)(z * a.S + sp) * a.M + m) * a.Nmax;
+      x += P[n];
+      y += P[n + 1];
+    }
+    const int b = m / a.n_tok, j = m % a.n_tok;
+    const int pos = a.pos0 + j;
+    if (n < s.rot_dim) {
+      float c, sn;
+      rope_cs(p, s.rot_dim, a.d_h, a.base, (double)pos, &c, &sn);
+      const float xr = x * c - y * sn, yr = x * sn + y * c;
+      x = xr; y = yr;
+    }
+    const int64_t o = (int64_t)b * s.os_b + s.col0 + (int64_t)pos * s.os_n + n;
+    store_elem(s.out, o, a.dtype, x);
+    store_elem(s.out, o + 1, a.dtype, y);
+  }
+}
+
+}  // namespace
+
+size_t writer_workspace_floats(const WriterArgs& a) {
+  return (size_t)a.Z * a.S * a.M * a.Nmax;
+}
+
+int writer_pick_splits(const WriterArgs& a, int num_sms) {
+  // enough CTAs for two waves; never more splits than 16-wide k-chunks
+  const int tiles = ceil_div(a.Nmax, BN) * ceil_div(a.M, BM) * a.Z;
+  int K = 0;
+  if (a.mode == LLA_WRITE_HLA) K = a.D;  // smallest GEMM depth (loop-1)
+  else if (a.mode == LLA_WRITE_PERHEAD) K = a.T * a.d_h;
+  else K = a.T * a.H * a.d_h;
+  const int nk = K / BK;
+  int S = ceil_div(2 * num_sms, tiles > 0 ? tiles : 1);
+  if (S > nk) S = nk;
+  if (S > 64) S = 64;
+  if (S < 1) S = 1;
+  return S;
+}
+
+cudaError_t launch_writer(const WriterArgs& a, cudaStream_t st) {
+  if (a.M == 0) return cudaSuccess;
+  dim3 grid(ceil_div(a.Nmax, BN), ceil_div(a.M, BM), a.Z * a.S);
+  writer_gemm<<<grid, WT, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t total = (int64_t)a.Z * a.M * (a.Nmax / 2);
+  int blocks = (int)((total + 255) / 256);
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  writer_epilogue<<<blocks, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace lla

@@ -1,0 +1,330 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+identical seeded inputs.  Tolerances: relative L2 <= 1e-4 for fp32 latents,
+<= 2e-2 for bf16-stored latents (fp32 accumulate); writer layout bit-exact."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import looped_transformer_latent_b200 as L
+import synth
+from oracle import hla, lla, rounding
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_BF16 = 2e-2
+BASE = 10000.0
+
+
+def rel_l2(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def _gen(seed):
+    g = torch.Generator()
+    g.manual_seed(seed)
+    return g
+
+
+# ------------------------------------------------------------- tiny HLA --
+def test_tiny_hla_layer_matches_oracle(cuda_device):
+    """Tiny fp32 HLA layer: writer (eq. 2) then both reads (loop 1 with
+    c^(1), loops 2..4 with c) through the C ABI, against the oracle."""
+    c = synth.CONFIGS["tiny_hla"]
+    x = synth.tiny_hla(0)
+    # oracle
+    lat_o, lat1_o = hla.write(x["h"], x["E_main"], x["E_1"], 0, c.r_k, c.r_v, c.r_1, c.d_h, c.base)
+    lat_o, lat1_o = rounding.to_f32(lat_o), rounding.to_f32(lat1_o)
+    o1 = hla.decode(lat1_o, x["A_1"], x["B_1"], x["q"][:1], x["win_k"], x["win_v"], 0, c.N, c.W,
+                    c.r_1, c.r_1, c.d_h, c.base)
+    om = hla.decode(lat_o, x["A"], x["Bm"], x["q"][1:], x["win_k"], x["win_v"], 1, c.N, c.W,
+                    c.r_k, c.r_v, c.d_h, c.base)
+    # CUDA path
+    dev = cuda_device
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    h = T(x["h"])[None]
+    lat = torch.full((1, c.N, c.r_k + c.r_v), float("nan"), device=dev)
+    lat1 = torch.full((1, c.N, 2 * c.r_1), float("nan"), device=dev)
+    L.lla_write_latents(L.LLA_WRITE_HLA, x=h, E_main=T(x["E_main"]), E_1=T(x["E_1"]), out0=lat,
+                        out1=lat1, r_k=c.r_k, d_h=c.d_h, pos0=0, rope_base=c.base)
+    q = T(x["q"])[None]
+    wk, wv = T(x["win_k"])[None], T(x["win_v"])[None]
+    out1 = torch.empty(1, 1, c.H, c.d_h, device=dev)
+    outm = torch.empty(1, c.T - 1, c.H, c.d_h, device=dev)
+    L.hla_decode_attn(lat=lat1, A=T(x["A_1"]), Bm=T(x["B_1"]), q=q[:, :1].contiguous(), win_k=wk,
+                      win_v=wv, out=out1, N=c.N, W=c.W, t0=0, rope_base=c.base)
+    L.hla_decode_attn(lat=lat, A=T(x["A"]), Bm=T(x["Bm"]), q=q[:, 1:].contiguous(), win_k=wk,
+                      win_v=wv, out=outm, N=c.N, W=c.W, t0=1, rope_base=c.base)
+    torch.cuda.synchronize()
+    assert rel_l2(f64(lat[0]), lat_o) < 1e-6
+    assert rel_l2(f64(lat1[0]), lat1_o) < 1e-6
+    e1, em = rel_l2(f64(out1[0]), o1), rel_l2(f64(outm[0]), om)
+    print(f"tiny HLA rel L2: loop1 {e1:.2e} main {em:.2e}")
+    assert e1 < TOL_F32 and em < TOL_F32
+
+
+# ------------------------------------------------- absorbed read, bf16 --
+def _absorbed_case(seed, B, N, W, H, nt, d_h, r_k, r_v, Wcap, t0=1, lat_dtype=torch.bfloat16,
+                   rotate=True):
+    g = _gen(seed)
+    T = t0 + nt
+    lat = (torch.randn(B, max(N, 1), r_k + r_v, generator=g) * math.sqrt(d_h / r_k)).to(lat_dtype)
+    A = torch.randn(nt, H, d_h, r_k, generator=g) / math.sqrt(d_h)
+    Bm = torch.randn(nt, H, r_v, d_h, generator=g) / math.sqrt(r_v)
+    q = torch.randn(B, nt, H, d_h, generator=g)
+    wk = torch.randn(B, T, Wcap, H, d_h, generator=g).to(torch.bfloat16)
+    wv = torch.randn(B, T, Wcap, H, d_h, generator=g).to(torch.bfloat16)
+    return dict(lat=lat, A=A, Bm=Bm, q=q, wk=wk, wv=wv, t0=t0, T=T)
+
+
+def _absorbed_oracle(cs, N, W, r_k, r_v, d_h, rotate):
+    B = cs["q"].shape[0]
+    out = []
+    for b in range(B):
+        out.append(hla.decode(f64(cs["lat"][b]), f64(cs["A"]), f64(cs["Bm"]), f64(cs["q"][b]),
+                              f64(cs["wk"][b]), f64(cs["wv"][b]), cs["t0"], N, W, r_k, r_v, d_h,
+                              BASE, rotate_query=rotate))
+    return np.stack(out)
+
+
+def _absorbed_gpu(cs, dev, N, W, rotate, **extra):
+    out = torch.full(tuple(cs["q"].shape), float("nan"), device=dev)
+    L.hla_decode_attn(lat=cs["lat"].to(dev), A=cs["A"].to(dev), Bm=cs["Bm"].to(dev),
+                      q=cs["q"].to(dev), win_k=cs["wk"].to(dev), win_v=cs["wv"].to(dev), out=out,
+                      N=N, W=W, t0=cs["t0"], rotate_query=rotate, rope_base=BASE, **extra)
+    torch.cuda.synchronize()
+    return f64(out)
+
+
+ABSORBED_CASES = [
+    # B, N, W, H, nt, d_h, r_k, r_v, Wcap
+    (3, 301, 16, 4, 3, 64, 128, 96, 17),      # several tiles, ragged tail
+    (2, 1, 8, 2, 1, 64, 64, 64, 9),           # N = 1: only the current token
+    (2, 10, 16, 2, 2, 64, 64, 64, 17),        # W >= i: no latent token
+    (2, 18, 16, 2, 1, 64, 64, 64, 17),        # exactly one latent token
+    (2, 700, 128, 16, 3, 128, 512, 512, 129), # Ouro-shaped main latent (48 rows)
+    (2, 650, 128, 16, 1, 128, 256, 256, 129), # Ouro-shaped loop-1 latent (16 rows)
+    (1, 1100, 0, 16, 4, 128, 576, 576, 1),    # LLA-2D-shaped: 64 rows, no window
+    (5, 257, 4, 3, 2, 32, 32, 40, 7),         # small ranks, ring larger than needed
+]
+
+
+@pytest.mark.parametrize("case", ABSORBED_CASES)
+@pytest.mark.parametrize("rotate", [True, False])
+def test_absorbed_read_bf16(cuda_device, case, rotate):
+    B, N, W, H, nt, d_h, r_k, r_v, Wcap = case
+    cs = _absorbed_case(1000 + N + H, B, N, W, H, nt, d_h, r_k, r_v, Wcap)
+    ref = _absorbed_oracle(cs, N, W, r_k, r_v, d_h, rotate)
+    got = _absorbed_gpu(cs, cuda_device, N, W, rotate)
+    err = rel_l2(got, ref)
+    print(f"absorbed {case} rotate={rotate}: rel L2 {err:.2e}")
+    assert np.all(np.isfinite(got))
+    assert err < TOL_BF16
+
+
+def test_absorbed_read_fp32_latents(cuda_device):
+    B, N, W, H, nt, d_h, r_k, r_v, Wcap = 2, 333, 16, 4, 2, 64, 128, 64, 20
+    cs = _absorbed_case(77, B, N, W, H, nt, d_h, r_k, r_v, Wcap, lat_dtype=torch.float32)
+    cs["wk"], cs["wv"] = cs["wk"].float(), cs["wv"].float()
+    err = rel_l2(_absorbed_gpu(cs, cuda_device, N, W, True), _absorbed_oracle(cs, N, W, r_k, r_v, d_h, True))
+    assert err < TOL_F32
+
+
+def test_explicit_scale(cuda_device):
+    B, N, W, H, nt, d_h, r_k, r_v, Wcap = 2, 90, 8, 2, 1, 64, 64, 64, 9
+    cs = _absorbed_case(5, B, N, W, H, nt, d_h, r_k, r_v, Wcap)
+    ref = np.stack([hla.decode(f64(cs["lat"][b]), f64(cs["A"]), f64(cs["Bm"]), f64(cs["q"][b]),
+                               f64(cs["wk"][b]), f64(cs["wv"][b]), cs["t0"], N, W, r_k, r_v, d_h,
+                               BASE, scale=0.3) for b in range(B)])
+    got = _absorbed_gpu(cs, cuda_device, N, W, True, scale=0.3)
+    assert rel_l2(got, ref) < TOL_BF16
+
+
+def test_strided_latent_view(cuda_device):
+    """A latent view with padded rows and a batch stride larger than dense."""
+    B, N, W, H, nt, d_h, r_k, r_v, Wcap = 2, 200, 8, 2, 2, 64, 64, 64, 9
+    cs = _absorbed_case(9, B, N, W, H, nt, d_h, r_k, r_v, Wcap)
+    big = torch.zeros(B, N + 7, r_k + r_v + 64, dtype=torch.bfloat16)
+    big[:, :N, :r_k + r_v] = cs["lat"]
+    ref = _absorbed_oracle(cs, N, W, r_k, r_v, d_h, True)
+    cs["lat"] = big[:, :, :r_k + r_v]
+    dev = cuda_device
+    out = torch.empty(tuple(cs["q"].shape), device=dev)
+    L.hla_decode_attn(lat=big.to(dev)[:, :, :r_k + r_v], A=cs["A"].to(dev), Bm=cs["Bm"].to(dev),
+                      q=cs["q"].to(dev), win_k=cs["wk"].to(dev), win_v=cs["wv"].to(dev), out=out,
+                      N=N, W=W, t0=cs["t0"], rope_base=BASE)
+    torch.cuda.synchronize()
+    assert rel_l2(f64(out), ref) < TOL_BF16
+
+
+# ------------------------------------------------ writer: exact layout --
+def _int_tensor(g, shape, lo, hi):
+    return torch.randint(lo, hi + 1, shape, generator=g).to(torch.float32)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_writer_hla_layout_bit_exact(cuda_device, dtype):
+    """Small integers in h and E make every latent exactly representable, so
+    the stored rows (and the untouched ones) must equal the oracle's bits."""
+    g = _gen(3)
+    B, n, pos0, Ncap, T, D, r_k, r_v, r_1, d_h = 3, 7, 5, 16, 4, 32, 16, 24, 8, 8
+    h = _int_tensor(g, (B, n, T, D), -2, 2)
+    E = (_int_tensor(g, (T - 1, r_k + r_v, D), -1, 1) * (torch.rand(T - 1, r_k + r_v, D, generator=g) < 0.15))
+    E1 = (_int_tensor(g, (2 * r_1, D), -1, 1) * (torch.rand(2 * r_1, D, generator=g) < 0.15))
+    sentinel = 1234.0
+    dev = cuda_device
+    lat = torch.full((B, Ncap, r_k + r_v), sentinel, dtype=dtype, device=dev)
+    lat1 = torch.full((B, Ncap, 2 * r_1), sentinel, dtype=dtype, device=dev)
+    L.lla_write_latents(L.LLA_WRITE_HLA, x=h.to(dev), E_main=E.to(dev), E_1=E1.to(dev), out0=lat,
+                        out1=lat1, r_k=r_k, d_h=d_h, pos0=pos0, rotate_keys=False)
+    torch.cuda.synchronize()
+    exp = torch.full((B, Ncap, r_k + r_v), sentinel, dtype=torch.float64)
+    exp1 = torch.full((B, Ncap, 2 * r_1), sentinel, dtype=torch.float64)
+    for b in range(B):
+        c, c1 = hla.write(h[b].double().numpy(), E.double().numpy(), E1.double().numpy(), pos0,
+                          r_k, r_v, r_1, d_h, BASE, rotate_keys=False)
+        exp[b, pos0:pos0 + n] = torch.from_numpy(c)
+        exp1[b, pos0:pos0 + n] = torch.from_numpy(c1)
+    assert torch.equal(lat.cpu(), exp.to(dtype))
+    assert torch.equal(lat1.cpu(), exp1.to(dtype))
+
+
+@pytest.mark.parametrize("mode", [L.LLA_WRITE_PERHEAD, L.LLA_WRITE_FOLDED])
+def test_writer_lla_layout_bit_exact(cuda_device, mode):
+    g = _gen(4 + mode)
+    B, n, pos0, Ncap, T, H, d_h = 2, 5, 3, 12, 3, 3, 16
+    r = 16 if mode == L.LLA_WRITE_PERHEAD else 24
+    rV = r if mode == L.LLA_WRITE_PERHEAD else 40
+    k = _int_tensor(g, (B, n, T, H, d_h), -2, 2)
+    v = _int_tensor(g, (B, n, T, H, d_h), -2, 2)
+    EK = _int_tensor(g, (T, H, r, d_h), -1, 1) * (torch.rand(T, H, r, d_h, generator=g) < 0.2)
+    EV = _int_tensor(g, (T, H, rV, d_h), -1, 1) * (torch.rand(T, H, rV, d_h, generator=g) < 0.2)
+    dev = cuda_device
+    sentinel = -77.0
+    if mode == L.LLA_WRITE_PERHEAD:
+        cK = torch.full((B, H, Ncap, r), sentinel, dtype=torch.bfloat16, device=dev)
+        cV = torch.full((B, H, Ncap, r), sentinel, dtype=torch.bfloat16, device=dev)
+        L.lla_write_latents(mode, x=k.to(dev), xv=v.to(dev), E_K=EK.to(dev), E_V=EV.to(dev),
+                            out0=cK, out1=cV, pos0=pos0)
+        torch.cuda.synchronize()
+        eK = torch.full((B, H, Ncap, r), sentinel, dtype=torch.float64)
+        eV = eK.clone()
+        for b in range(B):
+            ck, cv = lla.write_perhead(k[b].double().numpy(), v[b].double().numpy(),
+                                       EK.double().numpy(), EV.double().numpy())
+            eK[b, :, pos0:pos0 + n] = torch.from_numpy(ck)
+            eV[b, :, pos0:pos0 + n] = torch.from_numpy(cv)
+        assert torch.equal(cK.cpu(), eK.to(torch.bfloat16))
+        assert torch.equal(cV.cpu(), eV.to(torch.bfloat16))
+    else:
+        lat = torch.full((B, Ncap, r + rV), sentinel, dtype=torch.bfloat16, device=dev)
+        L.lla_write_latents(mode, x=k.to(dev), xv=v.to(dev), E_K=EK.to(dev), E_V=EV.to(dev),
+                            out0=lat, pos0=pos0)
+        torch.cuda.synchronize()
+        e = torch.full((B, Ncap, r + rV), sentinel, dtype=torch.float64)
+        for b in range(B):
+            e[b, pos0:pos0 + n] = torch.from_numpy(lla.write_folded(
+                k[b].double().numpy(), v[b].double().numpy(), EK.double().numpy(), EV.double().numpy()))
+        assert torch.equal(lat.cpu(), e.to(torch.bfloat16))
+
+
+def test_writer_rotation_and_rounding(cuda_device):
+    """Rotated bf16 writes: each value within one bf16 rounding of the
+    oracle's (fp32 accumulation order may move a value across a tie)."""
+    c = synth.CONFIGS["tiny_hla"]
+    x = synth.tiny_hla(1)
+    dev = cuda_device
+    pos0 = 100
+    n = 64
+    h = torch.from_numpy(x["h"][:n])[None].to(dev)
+    lat = torch.zeros(1, pos0 + n, c.r_k + c.r_v, dtype=torch.bfloat16, device=dev)
+    lat1 = torch.zeros(1, pos0 + n, 2 * c.r_1, dtype=torch.bfloat16, device=dev)
+    L.lla_write_latents(L.LLA_WRITE_HLA, x=h, E_main=torch.from_numpy(x["E_main"]).to(dev),
+                        E_1=torch.from_numpy(x["E_1"]).to(dev), out0=lat, out1=lat1, r_k=c.r_k,
+                        d_h=c.d_h, pos0=pos0, rope_base=c.base)
+    torch.cuda.synchronize()
+    ce, c1e = hla.write(x["h"][:n], x["E_main"], x["E_1"], pos0, c.r_k, c.r_v, c.r_1, c.d_h, c.base)
+    for got, exact in ((f64(lat[0, pos0:]), ce), (f64(lat1[0, pos0:]), c1e)):
+        ulp = np.abs(rounding.to_bf16(exact)) * 2.0 ** -7 + 1e-30
+        assert np.all(np.abs(got - exact) <= ulp)
+        assert np.mean(got == rounding.to_bf16(exact)) > 0.95
+
+
+# --------------------------------------------- LLA reconstruct-on-read --
+LLA_CASES = [
+    # B, H, d_h, r, T, t0, nt, N, W, Wcap
+    (2, 3, 32, 32, 4, 0, 4, 200, 0, 1),
+    (2, 2, 96, 96, 8, 2, 3, 77, 5, 6),
+    (1, 1, 64, 64, 1, 0, 1, 1, 0, 1),        # N = 1
+    (3, 2, 64, 32, 2, 0, 2, 129, 3, 4),      # r < d_h, ragged tile
+]
+
+
+@pytest.mark.parametrize("case", LLA_CASES)
+def test_lla_reconstruct_bf16(cuda_device, case):
+    B, H, d_h, r, T, t0, nt, N, W, Wcap = case
+    g = _gen(50 + N)
+    cK = torch.randn(B, H, N, r, generator=g).to(torch.bfloat16)
+    cV = torch.randn(B, H, N, r, generator=g).to(torch.bfloat16)
+    UK = torch.randn(nt, H, d_h, r, generator=g) / math.sqrt(r)
+    UV = torch.randn(nt, H, d_h, r, generator=g) / math.sqrt(r)
+    q = torch.randn(B, nt, H, d_h, generator=g)
+    wk = torch.randn(B, T, Wcap, H, d_h, generator=g).to(torch.bfloat16)
+    wv = torch.randn(B, T, Wcap, H, d_h, generator=g).to(torch.bfloat16)
+    ref = np.stack([lla.decode_reconstruct(f64(cK[b]), f64(cV[b]), f64(UK), f64(UV), f64(q[b]),
+                                           f64(wk[b]), f64(wv[b]), t0, N, W) for b in range(B)])
+    dev = cuda_device
+    out = torch.full((B, nt, H, d_h), float("nan"), device=dev)
+    L.lla_decode_attn(cK=cK.to(dev), cV=cV.to(dev), UK=UK.to(dev), UV=UV.to(dev), q=q.to(dev),
+                      win_k=wk.to(dev), win_v=wv.to(dev), out=out, N=N, W=W, t0=t0)
+    torch.cuda.synchronize()
+    err = rel_l2(f64(out), ref)
+    print(f"lla reconstruct {case}: rel L2 {err:.2e}")
+    assert err < TOL_BF16
+
+
+# ------------------------------------------ LLA-2D: writer + absorbed --
+def test_lla2d_writer_then_absorbed_read(cuda_device):
+    """End to end on LLA-2D: folded writer on both sides, then LLA-D (absorbed,
+    no rotation) on each side's own latents."""
+    g = _gen(60)
+    B, T, H, d_h, rK, rV, N, W = 2, 2, 4, 32, 64, 64, 50, 0
+    k = torch.randn(B, N, T, H, d_h, generator=g)
+    v = torch.randn(B, N, T, H, d_h, generator=g)
+    EK = torch.randn(T, H, rK, d_h, generator=g) / math.sqrt(T * H * d_h)
+    EV = torch.randn(T, H, rV, d_h, generator=g) / math.sqrt(T * H * d_h)
+    UK = torch.randn(T, H, d_h, rK, generator=g) / math.sqrt(rK)
+    UV = torch.randn(T, H, d_h, rV, generator=g) / math.sqrt(rV)
+    q = torch.randn(B, T, H, d_h, generator=g)
+    Wcap = 1
+    wk = torch.zeros(B, T, Wcap, H, d_h)
+    wv = torch.zeros(B, T, Wcap, H, d_h)
+    wk[:, :, (N - 1) % Wcap] = k[:, N - 1]
+    wv[:, :, (N - 1) % Wcap] = v[:, N - 1]
+    dev = cuda_device
+    lat = torch.zeros(B, N, rK + rV, dtype=torch.bfloat16, device=dev)
+    L.lla_write_latents(L.LLA_WRITE_FOLDED, x=k.to(dev), xv=v.to(dev), E_K=EK.to(dev),
+                        E_V=EV.to(dev), out0=lat, pos0=0)
+    out = torch.empty(B, T, H, d_h, device=dev)
+    L.hla_decode_attn(lat=lat, A=UK.to(dev), Bm=UV.transpose(2, 3).contiguous().to(dev), q=q.to(dev),
+                      win_k=wk.to(torch.bfloat16).to(dev), win_v=wv.to(torch.bfloat16).to(dev),
+                      out=out, N=N, W=W, t0=0, rotate_query=False)
+    torch.cuda.synchronize()
+    ref = []
+    for b in range(B):
+        row = rounding.to_bf16(lla.write_folded(f64(k[b]), f64(v[b]), f64(EK), f64(EV)))
+        ref.append(lla.decode_absorbed(row, f64(UK), f64(UV), f64(q[b]),
+                                       f64(wk[b].to(torch.bfloat16)), f64(wv[b].to(torch.bfloat16)),
+                                       0, N, W, rK, rV))
+    err = rel_l2(f64(out), np.stack(ref))
+    print(f"lla2d end to end rel L2 {err:.2e}")
+    assert err < TOL_BF16
