@@ -235,6 +235,30 @@ size_t hla_decode_workspace_bytes(const hla_decode_params *p);
 int hla_decode_attn(const hla_decode_params *p, void *ws, size_t ws_bytes,
                     lla_stream stream);
 
+/* ------------------------------------------------------------------------ */
+/* Absorbed read without a caller-provided workspace                          */
+/* ------------------------------------------------------------------------ */
+/* The pages have no counterpart to this entry point; it is a convenience of
+ * this library.  It computes exactly what hla_decode_attn computes, for
+ * callers that cannot allocate device memory: code that is handed only input
+ * and output buffers (e.g. a plugin whose host interface has no allocator), or
+ * a serving engine that has reserved all device memory for its cache, where an
+ * extra cudaMalloc fails or synchronises the device mid-decode.
+ *
+ * Scratch comes from one static device array of LLA_NOALLOC_SCRATCH_BYTES
+ * inside the library, held on every device that uses it until the process
+ * exits; the call allocates nothing.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current);
+ * make that first call before any stream capture begins.
+ * Errors: as hla_decode_attn; LLA_ERR_WORKSPACE when the problem needs more
+ * scratch than LLA_NOALLOC_SCRATCH_BYTES (hla_decode_workspace_bytes(p) tells
+ * how much).  All calls share the array: calls whose work may overlap on the
+ * GPU (other streams, unordered host threads) race on it and must not be
+ * issued; order them on one stream.  Nothing in the array needs to start at
+ * zero -- each call writes every scratch word before it reads it. */
+#define LLA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int hla_decode_attn_noalloc(const hla_decode_params *p, lla_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -104,7 +104,11 @@ PROTOTYPES = {
     "lla_decode_attn": (ctypes.c_int, [ctypes.POINTER(LlaDecodeParams), c_vp, ctypes.c_size_t, c_vp]),
     "hla_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(HlaDecodeParams)]),
     "hla_decode_attn": (ctypes.c_int, [ctypes.POINTER(HlaDecodeParams), c_vp, ctypes.c_size_t, c_vp]),
+    "hla_decode_attn_noalloc": (ctypes.c_int, [ctypes.POINTER(HlaDecodeParams), c_vp]),
 }
+
+# Size of the library's static scratch used by hla_decode_attn_noalloc.
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class LibraryMissing(RuntimeError):
