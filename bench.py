@@ -355,10 +355,19 @@ def main():
             e1.record(stream)
         step.run()                      # eager warm-up (sets kernel attributes)
     torch.cuda.synchronize()
+    _, outs = step.io_tensors()
+    eager = [o.clone() for o in outs]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         step.run(events=evs)
     torch.cuda.synchronize()
+    for o in outs:
+        o.fill_(float("nan"))
+    graph.replay()
+    torch.cuda.synchronize()
+    for o, e in zip(outs, eager):       # the replayed step must reproduce the eager one
+        if not torch.equal(o, e):
+            raise SystemExit("graph replay output differs from the eager step")
 
     for _ in range(args.warmup):
         graph.replay()

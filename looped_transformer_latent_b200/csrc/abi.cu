@@ -9,7 +9,8 @@ namespace lla {
 namespace {
 
 constexpr int kAbiVersion = 1;
-constexpr int kTargetCtas = 4 * 148;   // split heuristics aim at ~4 CTAs per SM
+constexpr int kNumSms = 148;            // B200
+constexpr int kTargetCtas = 4 * kNumSms;  // SIMT split heuristics aim at ~4 CTAs per SM
 constexpr size_t kAlign = 256;
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -102,7 +103,7 @@ WriterArgs writer_args(const lla_write_params& p) {
 int check_hla(const hla_decode_params& p) {
   if (p.B < 0 || p.nt < 0) return LLA_ERR_SHAPE;
   if (!dtype_ok(p.lat_dtype) || !dtype_ok(p.win_dtype)) return LLA_ERR_DTYPE;
-  if (p.H < 1 || p.d_h < 2 || p.d_h % 2 || p.T < 1 || p.t0 < 0 || p.t0 + p.nt > p.T) return LLA_ERR_SHAPE;
+  if (p.H < 1 || p.d_h < 4 || p.d_h % 4 || p.T < 1 || p.t0 < 0 || p.t0 + p.nt > p.T) return LLA_ERR_SHAPE;
   if (p.N < 1 || p.W < 0 || p.r_k < 2 || p.r_k % 2 || p.r_v < 1) return LLA_ERR_SHAPE;
   if (p.d_h > 128) return LLA_ERR_UNSUPPORTED;
   if (p.r_v > 1024 || p.r_k + p.r_v > 2048) return LLA_ERR_UNSUPPORTED;
@@ -122,6 +123,7 @@ int check_hla(const hla_decode_params& p) {
   if (!aligned(p.A, 16) || !aligned(p.Bm, 16) || p.r_k % 4) return LLA_ERR_ALIGN;
   if (!aligned(p.q, 4) || !aligned(p.out, 4)) return LLA_ERR_ALIGN;
   if (!aligned(p.win_k, 16) || !aligned(p.win_v, 16)) return LLA_ERR_ALIGN;
+  if ((p.win_stride_b * elem_size(p.win_dtype)) % 16) return LLA_ERR_ALIGN;
   const int64_t rowlen = (int64_t)p.nt * p.H * p.d_h;
   if (p.q_stride_b < rowlen || p.out_stride_b < rowlen) return LLA_ERR_SHAPE;
   if (p.win_stride_b < (int64_t)p.T * p.Wcap * p.H * p.d_h) return LLA_ERR_SHAPE;
@@ -131,7 +133,7 @@ int check_hla(const hla_decode_params& p) {
 int check_lla(const lla_decode_params& p) {
   if (p.B < 0 || p.nt < 0) return LLA_ERR_SHAPE;
   if (!dtype_ok(p.lat_dtype) || !dtype_ok(p.win_dtype)) return LLA_ERR_DTYPE;
-  if (p.H < 1 || p.d_h < 1 || p.T < 1 || p.t0 < 0 || p.t0 + p.nt > p.T) return LLA_ERR_SHAPE;
+  if (p.H < 1 || p.d_h < 4 || p.d_h % 4 || p.T < 1 || p.t0 < 0 || p.t0 + p.nt > p.T) return LLA_ERR_SHAPE;
   if (p.N < 1 || p.W < 0 || p.r < 1) return LLA_ERR_SHAPE;
   if (p.d_h > 128 || p.r > 128) return LLA_ERR_UNSUPPORTED;
   if ((long)p.nt * p.H > 65535) return LLA_ERR_UNSUPPORTED;
@@ -150,6 +152,7 @@ int check_lla(const lla_decode_params& p) {
   if (!aligned(p.UK, 16) || !aligned(p.UV, 16)) return LLA_ERR_ALIGN;
   if (!aligned(p.q, 4) || !aligned(p.out, 4)) return LLA_ERR_ALIGN;
   if (!aligned(p.win_k, 16) || !aligned(p.win_v, 16)) return LLA_ERR_ALIGN;
+  if ((p.win_stride_b * elem_size(p.win_dtype)) % 16) return LLA_ERR_ALIGN;
   const int64_t rowlen = (int64_t)p.nt * p.H * p.d_h;
   if (p.q_stride_b < rowlen || p.out_stride_b < rowlen) return LLA_ERR_SHAPE;
   if (p.win_stride_b < (int64_t)p.T * p.Wcap * p.H * p.d_h) return LLA_ERR_SHAPE;
@@ -158,8 +161,8 @@ int check_lla(const lla_decode_params& p) {
 
 // Workspace layout of the absorbed read.
 struct HlaPlan {
-  int rows, n_lat, win_start, n_win, S, tps;
-  size_t o_qlat, o_qwin, o_pml, o_py, o_wml, o_wy, bytes;
+  int rows, n_lat, win_start, n_win, S, tps, use_tc, rows_pad;
+  size_t o_qlat, o_qwin, o_pml, o_py, o_wml, o_wy, o_qbf, o_err, bytes;
 };
 
 HlaPlan plan_hla(const hla_decode_params& p) {
@@ -170,11 +173,18 @@ HlaPlan plan_hla(const hla_decode_params& p) {
   pl.n_lat = std::max(0, i - p.W);
   pl.win_start = pl.n_lat;
   pl.n_win = i - pl.win_start + 1;
-  if (pl.n_lat > 0) {
+  pl.use_tc = pl.n_lat > 0 && absorb_tc_supported(p.lat_dtype, p.r_k, p.r_v, pl.rows);
+  pl.rows_pad = pl.use_tc ? absorb_tc_rows_pad(pl.rows) : pl.rows;
+  if (pl.use_tc) {
+    // tensor-core read: one CTA per (split, sequence), 64-token tiles
+    const int S = absorb_tc_splits(p.B, pl.n_lat, kNumSms);
+    pl.tps = (int)(((pl.n_lat + S - 1) / S + 63) / 64 * 64);
+    pl.S = (pl.n_lat + pl.tps - 1) / pl.tps;
+  } else if (pl.n_lat > 0) {
     const long ctas = (long)p.B * ((pl.rows + 15) / 16);
     long S = (kTargetCtas + ctas - 1) / ctas;
     const long tiles = (pl.n_lat + 15) / 16;
-    S = std::max(1L, std::min(S, tiles));
+    S = std::max(1L, std::min(std::min(S, tiles), (long)map_max_splits()));
     pl.tps = (int)(((pl.n_lat + S - 1) / S + 15) / 16 * 16);
     pl.S = (pl.n_lat + pl.tps - 1) / pl.tps;
   } else {
@@ -182,12 +192,14 @@ HlaPlan plan_hla(const hla_decode_params& p) {
   }
   const size_t br = (size_t)p.B * pl.rows;
   Carve c;
-  pl.o_qlat = c.take(br * p.r_k * 4);
+  pl.o_qlat = c.take(pl.use_tc ? 0 : br * p.r_k * 4);
   pl.o_qwin = c.take(br * p.d_h * 4);
   pl.o_pml = c.take((size_t)pl.S * br * 2 * 4);
   pl.o_py = c.take((size_t)pl.S * br * p.r_v * 4);
   pl.o_wml = c.take(br * 2 * 4);
   pl.o_wy = c.take(br * p.d_h * 4);
+  pl.o_qbf = c.take(pl.use_tc ? (size_t)p.B * 64 * p.r_k * 2 : 0);
+  pl.o_err = c.take(sizeof(int));
   pl.bytes = c.off;
   return pl;
 }
@@ -234,7 +246,11 @@ inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? LLA_OK : LLA_E
 inline cudaError_t mark(void* events, int i, cudaStream_t s) {
   if (!events) return cudaSuccess;
   cudaEvent_t ev = reinterpret_cast<cudaEvent_t*>(events)[i];
-  return cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
+  return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal)
+                                             : cudaEventRecord(ev, s);
 }
 
 }  // namespace
@@ -315,10 +331,22 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
   a.win_ml = reinterpret_cast<float*>(w + pl.o_wml);
   a.win_y = reinterpret_cast<float*>(w + pl.o_wy);
   a.S = pl.S; a.tps = pl.tps;
+  a.use_tc = pl.use_tc; a.rows_pad = pl.rows_pad;
+  a.qbf = reinterpret_cast<__nv_bfloat16*>(w + pl.o_qbf);
+  a.err = reinterpret_cast<int*>(w + pl.o_err);
 
-  cudaError_t e = launch_absorb_prologue(a, s);
+  MapArgs qm;
+  std::memset(&qm, 0, sizeof(qm));
+  qm.B = a.B; qm.rows = a.rows; qm.K = a.d_h; qm.N = a.r_k; qm.d_h = a.d_h;
+  qm.W = a.A; qm.X = a.q; qm.xs_b = a.qs_b; qm.xs_row = a.d_h;
+  qm.rotate = a.rotate; qm.pos = a.N - 1; qm.use_tc = a.use_tc; qm.base = a.base; qm.qmul = a.qmul;
+  qm.qlat = a.qlat; qm.qwin = a.qwin; qm.qbf = a.qbf;
+  cudaError_t e = cudaSuccess;
+  if (a.use_tc) e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = launch_query_map(qm, s);
   if (e == cudaSuccess) e = mark(p->timing_events, 0, s);
-  if (e == cudaSuccess && a.n_lat > 0) e = launch_absorb_split_simt(a, s);
+  if (e == cudaSuccess && a.n_lat > 0)
+    e = a.use_tc ? launch_absorb_split_tc(a, s) : launch_absorb_split_simt(a, s);
   if (e == cudaSuccess) e = mark(p->timing_events, 1, s);
   if (e == cudaSuccess) {
     WindowArgs wa;
@@ -330,11 +358,12 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
     e = launch_window(wa, s);
   }
   if (e == cudaSuccess) {
-    MergeArgs g;
-    g.B = a.B; g.rows = a.rows; g.H = a.H; g.d_h = a.d_h; g.S = a.S; g.Y = a.r_v;
-    g.part_ml = a.part_ml; g.part_y = a.part_y; g.win_ml = a.win_ml; g.win_y = a.win_y;
-    g.Bm = a.Bm; g.out = a.out; g.outs_b = a.outs_b;
-    e = launch_merge(g, s);
+    MapArgs om;
+    std::memset(&om, 0, sizeof(om));
+    om.B = a.B; om.rows = a.rows; om.K = a.r_v; om.N = a.d_h; om.d_h = a.d_h; om.W = a.Bm;
+    om.part_ml = a.part_ml; om.part_y = a.part_y; om.win_ml = a.win_ml; om.win_y = a.win_y; om.S = a.S;
+    om.out = a.out; om.outs_b = a.outs_b; om.err = a.use_tc ? a.err : nullptr;
+    e = launch_output_map(om, s);
   }
   return cuda_status(e);
 }
@@ -388,7 +417,7 @@ int lla_decode_attn(const lla_decode_params* p, void* ws, size_t ws_bytes, lla_s
     MergeArgs g;
     g.B = a.B; g.rows = a.rows; g.H = a.H; g.d_h = a.d_h; g.S = a.S; g.Y = a.d_h;
     g.part_ml = a.part_ml; g.part_y = a.part_y; g.win_ml = a.win_ml; g.win_y = a.win_y;
-    g.Bm = nullptr; g.out = a.out; g.outs_b = a.outs_b;
+    g.Bm = nullptr; g.out = a.out; g.outs_b = a.outs_b; g.err = nullptr;
     e = launch_merge(g, s);
   }
   return cuda_status(e);

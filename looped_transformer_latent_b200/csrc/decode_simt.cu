@@ -8,64 +8,6 @@
 namespace lla {
 namespace {
 
-// ------------------------------------------------------------ prologue --
-// q~[b][row] = scale*log2e * R~_i A_{t,h}^T q_{t,h}   (latent space, rank r_k)
-// q_w[b][row] = scale*log2e * R_i q_{t,h}             (head space, exact tokens)
-// Grid: x = pair chunks of 64 (+1 block for q_w), y = row, z = 32-sequence chunk.
-constexpr int PRO_B = 32;
-
-__global__ void __launch_bounds__(64) absorb_prologue(AbsorbArgs a) {
-  extern __shared__ float qsm[];  // [PRO_B][d_h]
-  const int row = blockIdx.y, tt = row / a.H, h = row % a.H;
-  const int b0 = blockIdx.z * PRO_B;
-  const int nb = min(PRO_B, a.B - b0);
-  for (int idx = threadIdx.x; idx < PRO_B * a.d_h; idx += blockDim.x) {
-    const int bb = idx / a.d_h, d = idx % a.d_h;
-    qsm[idx] = bb < nb ? a.q[(int64_t)(b0 + bb) * a.qs_b + (int64_t)(tt * a.H + h) * a.d_h + d] : 0.f;
-  }
-  __syncthreads();
-  const int i = a.N - 1;
-  const int nchunks = ceil_div(a.r_k / 2, 64);
-  if ((int)blockIdx.x < nchunks) {
-    const int p = blockIdx.x * 64 + threadIdx.x;
-    if (2 * p >= a.r_k) return;
-    const float* Ar = a.A + ((int64_t)(tt * a.H + h) * a.d_h) * a.r_k + 2 * p;
-    float acc0[PRO_B], acc1[PRO_B];
-#pragma unroll
-    for (int bb = 0; bb < PRO_B; ++bb) acc0[bb] = acc1[bb] = 0.f;
-    for (int d = 0; d < a.d_h; ++d) {
-      const float2 av = *reinterpret_cast<const float2*>(Ar + (int64_t)d * a.r_k);
-#pragma unroll
-      for (int bb = 0; bb < PRO_B; ++bb) {
-        const float qv = qsm[bb * a.d_h + d];
-        acc0[bb] = fmaf(av.x, qv, acc0[bb]);
-        acc1[bb] = fmaf(av.y, qv, acc1[bb]);
-      }
-    }
-    float c = 1.f, s = 0.f;
-    if (a.rotate) rope_cs(p, a.r_k, a.d_h, a.base, (double)i, &c, &s);
-#pragma unroll
-    for (int bb = 0; bb < PRO_B; ++bb) {
-      if (bb >= nb) break;
-      const float x = acc0[bb], y = acc1[bb];
-      float* dst = a.qlat + ((int64_t)(b0 + bb) * a.rows + row) * a.r_k + 2 * p;
-      dst[0] = (x * c - y * s) * a.qmul;
-      dst[1] = (x * s + y * c) * a.qmul;
-    }
-  } else {
-    const int hp = a.d_h / 2;
-    for (int idx = threadIdx.x; idx < nb * hp; idx += blockDim.x) {
-      const int bb = idx / hp, p = idx % hp;
-      float c = 1.f, s = 0.f;
-      if (a.rotate) rope_cs(p, a.d_h, a.d_h, a.base, (double)i, &c, &s);
-      const float x = qsm[bb * a.d_h + 2 * p], y = qsm[bb * a.d_h + 2 * p + 1];
-      float* dst = a.qwin + ((int64_t)(b0 + bb) * a.rows + row) * a.d_h + 2 * p;
-      dst[0] = (x * c - y * s) * a.qmul;
-      dst[1] = (x * s + y * c) * a.qmul;
-    }
-  }
-}
-
 // ------------------------------------------------- absorbed split, SIMT --
 // One CTA per (split, sequence, block of RB query rows).  A tile of TT latent
 // tokens is staged in shared memory (fp32), scores for RB x TT pairs are one
@@ -168,57 +110,89 @@ __global__ void __launch_bounds__(256) absorb_split_simt(AbsorbArgs a) {
 }
 
 // --------------------------------------------------------------- window --
-// Exact attention over the window ring for one (row, sequence): 4 warps split
-// the tokens, lanes split the head dimension, one online softmax per warp,
-// combined at the end.  Emits (max, sum, y_w) in base-2 units.
+// Exact attention over the window ring for one (row, sequence).  Each lane
+// holds 4 consecutive elements of the head dimension (one 8- or 16-byte load
+// per token), each warp takes every 4th group of WU tokens and issues all of a
+// group's K and V loads before using them, keeps its own online softmax, and
+// the four warps are combined at the end.  Emits (max, sum, y_w) in base-2 units.
+constexpr int WU = 8;
+
+template <bool BF16>
+__device__ __forceinline__ void load4(const void* base, int64_t idx, float* v) {
+  if (BF16) {
+    const uint2 u = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(base) + idx);
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    const float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  } else {
+    const float4 f = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+  }
+}
+
+template <bool BF16>
 __global__ void __launch_bounds__(128) window_attn(WindowArgs w) {
   const int row = blockIdx.x, b = blockIdx.y;
   const int tt = row / w.H, h = row % w.H, t = w.t0 + tt;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int KD = 4;  // d_h <= 128
-  float qv[KD], acc[KD];
+  const int d0 = 4 * lane;
+  const bool dv = d0 < w.d_h;
+  float qv[4] = {0.f, 0.f, 0.f, 0.f}, acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (dv) {
+    const float* q = w.q + (int64_t)b * w.q_sb + (int64_t)row * w.q_srow + d0;
 #pragma unroll
-  for (int k = 0; k < KD; ++k) {
-    const int d = lane + 32 * k;
-    qv[k] = d < w.d_h ? w.q[(int64_t)b * w.q_sb + (int64_t)row * w.q_srow + d] * w.qmul : 0.f;
-    acc[k] = 0.f;
+    for (int e = 0; e < 4; ++e) qv[e] = q[e] * w.qmul;
   }
   float m = -INFINITY, l = 0.f;
-  for (int idx = warp; idx < w.n_win; idx += 4) {
-    const int j = w.win_start + idx;
-    const int slot = j % w.Wcap;
-    const int64_t base = (int64_t)b * w.wins_b + (((int64_t)t * w.Wcap + slot) * w.H + h) * w.d_h;
-    float part = 0.f;
-    float vv[KD];
+  const int64_t seq = (int64_t)b * w.wins_b;
+  for (int g0 = warp * WU; g0 < w.n_win; g0 += 4 * WU) {
+    float kk[WU][4], vv[WU][4];
 #pragma unroll
-    for (int k = 0; k < KD; ++k) {
-      const int d = lane + 32 * k;
-      float kk = 0.f;
-      vv[k] = 0.f;
-      if (d < w.d_h) {
-        kk = load_elem(w.wk, base + d, w.dtype);
-        vv[k] = load_elem(w.wv, base + d, w.dtype);
+    for (int u = 0; u < WU; ++u) {
+      const int idx = g0 + u;
+      if (dv && idx < w.n_win) {
+        const int slot = (w.win_start + idx) % w.Wcap;
+        const int64_t base = seq + (((int64_t)t * w.Wcap + slot) * w.H + h) * w.d_h + d0;
+        load4<BF16>(w.wk, base, kk[u]);
+        load4<BF16>(w.wv, base, vv[u]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) kk[u][e] = vv[u][e] = 0.f;
       }
-      part = fmaf(qv[k], kk, part);
     }
-    const float sc = warp_sum(part);
-    const float mn = fmaxf(m, sc);
-    const float al = (m == -INFINITY) ? 0.f : exp2f(m - mn);
-    const float p = exp2f(sc - mn);
-    l = l * al + p;
+    float sc[WU];
 #pragma unroll
-    for (int k = 0; k < KD; ++k) acc[k] = fmaf(p, vv[k], acc[k] * al);
-    m = mn;
+    for (int u = 0; u < WU; ++u) {
+      float part = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) part = fmaf(qv[e], kk[u][e], part);
+      sc[u] = part;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < WU; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
+#pragma unroll
+    for (int u = 0; u < WU; ++u) {
+      if (g0 + u >= w.n_win) break;
+      const float mn = fmaxf(m, sc[u]);
+      const float al = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+      const float p = exp2f(sc[u] - mn);
+      l = l * al + p;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] = fmaf(p, vv[u][e], acc[e] * al);
+      m = mn;
+    }
   }
   __shared__ float sm_m[4], sm_l[4], sm_y[4][128];
   if (lane == 0) { sm_m[warp] = m; sm_l[warp] = l; }
+  if (dv) {
 #pragma unroll
-  for (int k = 0; k < KD; ++k) {
-    const int d = lane + 32 * k;
-    if (d < 128) sm_y[warp][d] = acc[k];
+    for (int e = 0; e < 4; ++e) sm_y[warp][d0 + e] = acc[e];
   }
   __syncthreads();
-  float M = fmaxf(fmaxf(sm_m[0], sm_m[1]), fmaxf(sm_m[2], sm_m[3]));
+  const float M = fmaxf(fmaxf(sm_m[0], sm_m[1]), fmaxf(sm_m[2], sm_m[3]));
   float wgt[4], L = 0.f;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
@@ -236,74 +210,10 @@ __global__ void __launch_bounds__(128) window_attn(WindowArgs w) {
 }
 
 // ---------------------------------------------------------------- merge --
-// Combine split partials and the window partial of each (sequence, row):
+// Combine split partials and the window partial of each (sequence, row) for
+// head-space partials (LLA reconstruct):
 //   M = max_s m_s, w_s = 2^(m_s - M), l = sum_s w_s l_s + w_w l_w,
-//   o = (B_{t,h}^T sum_s w_s y~_s + w_w y_w) / l      (mapped)
-//   o = (sum_s w_s y_s + w_w y_w) / l                 (head-space partials)
-// Mapped variant: one CTA per (row, chunk of MB sequences) so each B_{t,h}
-// is read once per chunk.
-constexpr int MB = 16;
-
-__global__ void __launch_bounds__(256) merge_mapped(MergeArgs g) {
-  extern __shared__ float sm[];
-  float* ybar = sm;                 // [MB][Y]
-  float* wwin = ybar + MB * g.Y;    // [MB]
-  float* linv = wwin + MB;          // [MB]
-  float* red = linv + MB;           // [2][MB][128] partial map results
-  const int row = blockIdx.x, b0 = blockIdx.y * MB;
-  const int nb = min(MB, g.B - b0);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int bb = warp; bb < nb; bb += 8) {
-    const int b = b0 + bb;
-    const int64_t br = (int64_t)b * g.rows + row;
-    float M = g.win_ml[br * 2];
-    for (int s = 0; s < g.S; ++s) M = fmaxf(M, g.part_ml[((int64_t)s * g.B * g.rows + br) * 2]);
-    const float ww = exp2f(g.win_ml[br * 2] - M);
-    float L = ww * g.win_ml[br * 2 + 1];
-    for (int s = 0; s < g.S; ++s) {
-      const float ms = g.part_ml[((int64_t)s * g.B * g.rows + br) * 2];
-      if (ms == -INFINITY) continue;
-      L += exp2f(ms - M) * g.part_ml[((int64_t)s * g.B * g.rows + br) * 2 + 1];
-    }
-    for (int v = lane; v < g.Y; v += 32) {
-      float y = 0.f;
-      for (int s = 0; s < g.S; ++s) {
-        const float ms = g.part_ml[((int64_t)s * g.B * g.rows + br) * 2];
-        if (ms == -INFINITY) continue;
-        y = fmaf(exp2f(ms - M), g.part_y[((int64_t)s * g.B * g.rows + br) * g.Y + v], y);
-      }
-      ybar[bb * g.Y + v] = y;
-    }
-    if (lane == 0) { wwin[bb] = ww; linv[bb] = 1.f / L; }
-  }
-  __syncthreads();
-  // o[b][d] = sum_v Bm[row][v][d] * ybar[b][v]; thread = (d, half of v range)
-  const int d = threadIdx.x % 128, half = threadIdx.x / 128;
-  const float* Bmr = g.Bm + (int64_t)row * g.Y * g.d_h;
-  if (d < g.d_h) {
-    float acc[MB];
-#pragma unroll
-    for (int bb = 0; bb < MB; ++bb) acc[bb] = 0.f;
-    const int vh = (g.Y + 1) / 2;
-    const int v0 = half * vh, v1 = min(g.Y, v0 + vh);
-    for (int v = v0; v < v1; ++v) {
-      const float bm = __ldg(Bmr + (int64_t)v * g.d_h + d);
-#pragma unroll
-      for (int bb = 0; bb < MB; ++bb) acc[bb] = fmaf(bm, ybar[bb * g.Y + v], acc[bb]);
-    }
-#pragma unroll
-    for (int bb = 0; bb < MB; ++bb) red[(half * MB + bb) * 128 + d] = acc[bb];
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < nb * g.d_h; idx += 256) {
-    const int bb = idx / g.d_h, dd = idx % g.d_h;
-    const int b = b0 + bb;
-    const int64_t br = (int64_t)b * g.rows + row;
-    const float v = red[bb * 128 + dd] + red[(MB + bb) * 128 + dd] + wwin[bb] * g.win_y[br * g.d_h + dd];
-    g.out[(int64_t)b * g.outs_b + (int64_t)row * g.d_h + dd] = v * linv[bb];
-  }
-}
-
+//   o = (sum_s w_s y_s + w_w y_w) / l
 __global__ void __launch_bounds__(128) merge_plain(MergeArgs g) {
   const int row = blockIdx.x, b = blockIdx.y;
   const int64_t br = (int64_t)b * g.rows + row;
@@ -324,7 +234,7 @@ __global__ void __launch_bounds__(128) merge_plain(MergeArgs g) {
       if (ms == -INFINITY) continue;
       y = fmaf(exp2f(ms - M), g.part_y[((int64_t)s * g.B * g.rows + br) * g.d_h + d], y);
     }
-    g.out[(int64_t)b * g.outs_b + (int64_t)row * g.d_h + d] = y * li;
+    g.out[(int64_t)b * g.outs_b + (int64_t)row * g.d_h + d] = (g.err && *g.err) ? NAN : y * li;
   }
 }
 
@@ -447,13 +357,6 @@ __global__ void __launch_bounds__(256) recon_split_simt(ReconArgs a) {
 
 }  // namespace
 
-cudaError_t launch_absorb_prologue(const AbsorbArgs& a, cudaStream_t st) {
-  dim3 grid(ceil_div(a.r_k / 2, 64) + 1, a.rows, ceil_div(a.B, PRO_B));
-  const size_t smem = (size_t)PRO_B * a.d_h * sizeof(float);
-  absorb_prologue<<<grid, 64, smem, st>>>(a);
-  return cudaGetLastError();
-}
-
 static size_t absorb_simt_smem(const AbsorbArgs& a) {
   const int R = a.r_k + a.r_v;
   const int LD = R + ((33 - (R % 32)) % 32);
@@ -471,21 +374,16 @@ cudaError_t launch_absorb_split_simt(const AbsorbArgs& a, cudaStream_t st) {
 
 cudaError_t launch_window(const WindowArgs& w, cudaStream_t st) {
   dim3 grid(w.rows, w.B);
-  window_attn<<<grid, 128, 0, st>>>(w);
+  if (w.dtype == LLA_BF16)
+    window_attn<true><<<grid, 128, 0, st>>>(w);
+  else
+    window_attn<false><<<grid, 128, 0, st>>>(w);
   return cudaGetLastError();
 }
 
 cudaError_t launch_merge(const MergeArgs& g, cudaStream_t st) {
-  if (g.Bm) {
-    const size_t smem = sizeof(float) * ((size_t)MB * g.Y + 2 * MB + 2 * MB * 128);
-    cudaError_t e = cudaFuncSetAttribute(merge_mapped, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(g.rows, ceil_div(g.B, MB));
-    merge_mapped<<<grid, 256, smem, st>>>(g);
-  } else {
-    dim3 grid(g.rows, g.B);
-    merge_plain<<<grid, 128, 0, st>>>(g);
-  }
+  dim3 grid(g.rows, g.B);
+  merge_plain<<<grid, 128, 0, st>>>(g);
   return cudaGetLastError();
 }
 

@@ -51,6 +51,11 @@ struct AbsorbArgs {
   float *win_ml;       // [B][rows][2]
   float *win_y;        // [B][rows][d_h]
   int S, tps;          // splits of the latent range, tokens per split
+  // tensor-core path
+  int use_tc;
+  int rows_pad;        // rows rounded up to 16 (N of the accumulate MMA)
+  __nv_bfloat16* qbf;  // [B][r_k/64][64 rows x 64] bf16 Q~, 128-byte swizzled, rows >= rows zero
+  int* err;            // 0, or the code of a timed-out wait in the latent read
 };
 
 // ------------------------------------------------- reconstruct decode --
@@ -89,12 +94,40 @@ struct MergeArgs {
   const float* Bm;   // [rows][Y][d_h] when mapping latent space back; else null
   float* out;
   int64_t outs_b;
+  const int* err;    // optional: when it holds a non-zero code the output is NaN
 };
 
-cudaError_t launch_absorb_prologue(const AbsorbArgs& a, cudaStream_t st);
+// Per-(loop, head) linear maps of the absorbed read (maps.cu).
+struct MapArgs {
+  int B, rows, K, N, d_h;
+  const float* W;          // [rows][K][N]: A_{t,h} (query map) or B_{t,h} (output map)
+  // query map: X = q [B][rows][d_h] (K = d_h, N = r_k)
+  const float* X;
+  int64_t xs_b, xs_row;
+  int rotate, pos, use_tc;
+  double base;
+  float qmul;
+  float *qlat, *qwin;
+  __nv_bfloat16* qbf;
+  // output map: X = sum over splits of the partials (K = r_v, N = d_h)
+  const float *part_ml, *part_y, *win_ml, *win_y;
+  int S;
+  float* out;
+  int64_t outs_b;
+  const int* err;
+};
+int map_max_splits();
+cudaError_t launch_query_map(const MapArgs& g, cudaStream_t st);
+cudaError_t launch_output_map(const MapArgs& g, cudaStream_t st);
+
 cudaError_t launch_absorb_split_simt(const AbsorbArgs& a, cudaStream_t st);
 cudaError_t launch_window(const WindowArgs& w, cudaStream_t st);
 cudaError_t launch_merge(const MergeArgs& m, cudaStream_t st);
 cudaError_t launch_recon_split_simt(const ReconArgs& a, cudaStream_t st);
+
+bool absorb_tc_supported(int lat_dtype, int r_k, int r_v, int rows);
+int absorb_tc_rows_pad(int rows);
+int absorb_tc_splits(int B, int n_lat, int num_sms);
+cudaError_t launch_absorb_split_tc(const AbsorbArgs& a, cudaStream_t st);
 
 }  // namespace lla

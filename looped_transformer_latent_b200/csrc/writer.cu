@@ -10,7 +10,7 @@
 namespace lla {
 namespace {
 
-constexpr int BM = 64, BN = 64, BK = 16, WT = 256;
+constexpr int BK = 16, WT = 256;
 
 struct Slice {
   const float* X;
@@ -66,55 +66,78 @@ __device__ __forceinline__ Slice slice_of(const WriterArgs& a, int z) {
   return s;
 }
 
-// Phase 1: C_part[z][split][m][n] = sum over this split's k-chunks.
+// Phase 1: C_part[z][split][m][n] = sum over this split's k-chunks.  Tile
+// TM x TN (64 x 64, or 32 x 128 for decode-size batches), 16-deep k-chunks
+// staged in shared memory, the next chunk prefetched into registers while the
+// current one is multiplied; each thread owns a 4 x 4 block of outputs.
+template <int TM, int TN>
 __global__ void __launch_bounds__(WT) writer_gemm(WriterArgs a) {
+  constexpr int LA = TM * BK / WT, LB = TN * BK / WT;   // loads per thread
+  constexpr int TX = TN / 4;                              // threads along n
   const int z = blockIdx.z / a.S, split = blockIdx.z % a.S;
   const Slice s = slice_of(a, z);
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  const int n0 = blockIdx.x * TN, m0 = blockIdx.y * TM;
   if (n0 >= s.N) return;
   const int K = s.K_outer * s.d_in;
   const int nk = K / BK;
   const int kc0 = (int)((int64_t)nk * split / a.S), kc1 = (int)((int64_t)nk * (split + 1) / a.S);
 
-  __shared__ float As[BK][BM + 4];
-  __shared__ float Bs[BK][BN + 4];
-  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  __shared__ float As[2][BK][TM + 4];
+  __shared__ float Bs[2][BK][TN + 4];
+  const int tid = threadIdx.x, tx = tid % TX, ty = tid / TX;
   float acc[4][4] = {};
 
-  // loader mapping: 64 rows x 16 k = 1024 values, 4 per thread
-  const int lr = tid / 4, lk = (tid % 4) * 4;
-  const int m = m0 + lr;
+  const int ar = tid / (BK / LA), ak = (tid % (BK / LA)) * LA;
+  const int br = tid / (BK / LB), bk = (tid % (BK / LB)) * LB;
+  const int m = m0 + ar;
   const bool mval = m < a.M;
   int64_t xrow = 0;
   if (mval) {
     const int b = m / a.n_tok, j = m % a.n_tok;
     xrow = (int64_t)b * a.xs_b + (int64_t)j * a.xs_n;
   }
-  const int n = n0 + lr;
+  const int n = n0 + br;
   const bool nval = n < s.N;
-
-  for (int kc = kc0; kc < kc1; ++kc) {
+  float ra[LA], rb[LB];
+  auto load = [&](int kc) {
     const int k = kc * BK;
-    const int o = k / s.d_in, d = k % s.d_in + lk;
+    const int o = k / s.d_in, d = k % s.d_in;
     const int64_t xo = (int64_t)(o / s.o_h) * s.x_o_t + (int64_t)(o % s.o_h) * s.x_o_h;
+    const float* xp = s.X + xrow + xo + d + ak;
+    const float* ep = s.E + (int64_t)o * s.e_o + (int64_t)n * s.e_n + d + bk;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      As[lk + u][lr] = mval ? __ldg(s.X + xrow + xo + d + u) : 0.f;
-      Bs[lk + u][lr] = nval ? __ldg(s.E + (int64_t)o * s.e_o + (int64_t)n * s.e_n + d + u) : 0.f;
-    }
-    __syncthreads();
+    for (int u = 0; u < LA; ++u) ra[u] = mval ? __ldg(xp + u) : 0.f;
+#pragma unroll
+    for (int u = 0; u < LB; ++u) rb[u] = nval ? __ldg(ep + u) : 0.f;
+  };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int u = 0; u < LA; ++u) As[buf][ak + u][ar] = ra[u];
+#pragma unroll
+    for (int u = 0; u < LB; ++u) Bs[buf][bk + u][br] = rb[u];
+  };
+
+  if (kc0 < kc1) {
+    load(kc0);
+    stash(0);
+  }
+  __syncthreads();
+  for (int kc = kc0; kc < kc1; ++kc) {
+    const int buf = (kc - kc0) & 1;
+    if (kc + 1 < kc1) load(kc + 1);
 #pragma unroll
     for (int kk = 0; kk < BK; ++kk) {
       float av[4], bv[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty * 4 + i];
+      for (int i = 0; i < 4; ++i) av[i] = As[buf][kk][ty * 4 + i];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) bv[i] = Bs[kk][tx * 4 + i];
+      for (int i = 0; i < 4; ++i) bv[i] = Bs[buf][kk][tx * 4 + i];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) acc[i][jj] = fmaf(av[i], bv[jj], acc[i][jj]);
     }
+    if (kc + 1 < kc1) stash(buf ^ 1);
     __syncthreads();
   }
   float* P = a.part + ((int64_t)(z * a.S + split) * a.M) * a.Nmax;
@@ -168,9 +191,12 @@ size_t writer_workspace_floats(const WriterArgs& a) {
   return (size_t)a.Z * a.S * a.M * a.Nmax;
 }
 
+static bool small_batch(const WriterArgs& a) { return a.M <= 32; }
+
 int writer_pick_splits(const WriterArgs& a, int num_sms) {
   // enough CTAs for two waves; never more splits than 16-wide k-chunks
-  const int tiles = ceil_div(a.Nmax, BN) * ceil_div(a.M, BM) * a.Z;
+  const int tm = small_batch(a) ? 32 : 64, tn = small_batch(a) ? 128 : 64;
+  const int tiles = ceil_div(a.Nmax, tn) * ceil_div(a.M, tm) * a.Z;
   int K = 0;
   if (a.mode == LLA_WRITE_HLA) K = a.D;  // smallest GEMM depth (loop-1)
   else if (a.mode == LLA_WRITE_PERHEAD) K = a.T * a.d_h;
@@ -185,8 +211,13 @@ int writer_pick_splits(const WriterArgs& a, int num_sms) {
 
 cudaError_t launch_writer(const WriterArgs& a, cudaStream_t st) {
   if (a.M == 0) return cudaSuccess;
-  dim3 grid(ceil_div(a.Nmax, BN), ceil_div(a.M, BM), a.Z * a.S);
-  writer_gemm<<<grid, WT, 0, st>>>(a);
+  if (small_batch(a)) {
+    dim3 grid(ceil_div(a.Nmax, 128), ceil_div(a.M, 32), a.Z * a.S);
+    writer_gemm<32, 128><<<grid, WT, 0, st>>>(a);
+  } else {
+    dim3 grid(ceil_div(a.Nmax, 64), ceil_div(a.M, 64), a.Z * a.S);
+    writer_gemm<64, 64><<<grid, WT, 0, st>>>(a);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t total = (int64_t)a.Z * a.M * (a.Nmax / 2);
