@@ -100,170 +100,312 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------- workloads --
-class HlaStep:
-    """One decode step of an HLA model (absorbed reads + writer), all layers."""
+class Step:
+    """One decode step: every layer's latent reads plus the writer for the new
+    token.  Subclasses fill self.calls with (kind, kwargs, tag) tuples; tag
+    'main' marks the read calls whose latent-read kernel is the roofline's."""
 
-    def __init__(self, cfg, dev, mode, seed=1234):
+    kind_launches = {"hla": 3, "lla": 2, "write": 2}
+
+    def __init__(self, cfg, dev, mode):
         import looped_transformer_latent_b200 as L
         self.L = L
         self.cfg, self.dev, self.mode = cfg, dev, mode
+        self.i = cfg.N - 1
+        self.n_lat = max(0, self.i - cfg.W)
+        self.n_win = self.i - self.n_lat + 1
+        self.calls = []
+
+    def _workspace(self):
+        L = self.L
+        nb = 0
+        for kind, kw, _ in self.calls:
+            if kind == "hla":
+                nb = max(nb, L.hla_decode_workspace_bytes(**kw))
+            elif kind == "lla":
+                nb = max(nb, L.lla_decode_workspace_bytes(**kw))
+            else:
+                mode = kw["mode"]
+                nb = max(nb, L.lla_write_workspace_bytes(mode, **{k: v for k, v in kw.items() if k != "mode"}))
+        self.ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=self.dev)
+
+    def run(self, events=None):
+        L = self.L
+        ei = 0
+        for kind, kw, _ in self.calls:
+            if kind in ("hla", "lla"):
+                ev = None
+                if events is not None:
+                    ev = events[ei]
+                    ei += 1
+                fn = L.hla_decode_attn if kind == "hla" else L.lla_decode_attn
+                fn(workspace=self.ws, timing_events=ev, **kw)
+            else:
+                mode = kw["mode"]
+                L.lla_write_latents(mode, workspace=self.ws, **{k: v for k, v in kw.items() if k != "mode"})
+
+    def read_tags(self):
+        return [tag for kind, _, tag in self.calls if kind in ("hla", "lla")]
+
+    def kernel_launches(self):
+        n = 0
+        for kind, _, _ in self.calls:
+            n += self.kind_launches["write" if kind.startswith("write") else kind]
+            if kind in ("hla", "lla") and self.n_lat > 0:
+                n += 1
+        return n
+
+    def latent_bytes(self, kind, kw):
+        c = self.cfg
+        if kind == "hla":
+            return c.B * self.n_lat * kw["lat"].shape[-1] * 2
+        return c.B * c.H * self.n_lat * kw["cK"].shape[-1] * 2 * 2
+
+    def read_latent_bytes(self):
+        return [self.latent_bytes(kind, kw) for kind, kw, _ in self.calls if kind in ("hla", "lla")]
+
+    def step_bytes(self):
+        """Algorithmic bytes: latents + exact window + codecs read, writer inputs/outputs."""
+        c = self.cfg
+        total = 0
+        for kind, kw, _ in self.calls:
+            if kind in ("hla", "lla"):
+                nt = kw["q"].shape[1]
+                total += self.latent_bytes(kind, kw)
+                total += c.B * nt * self.n_win * c.H * c.d_h * kw["win_k"].element_size() * 2
+                mats = ("A", "Bm") if kind == "hla" else ("UK", "UV")
+                total += sum(kw[m].numel() * 4 for m in mats)
+            else:
+                for k in ("E_main", "E_1", "E_K", "E_V", "x", "xv"):
+                    if kw.get(k) is not None:
+                        total += kw[k].numel() * 4
+                for k in ("out0", "out1"):
+                    o = kw.get(k)
+                    if o is not None:
+                        n_tok = kw["x"].shape[1]
+                        rows = c.B * n_tok * (o.shape[1] if o.dim() == 4 else 1)
+                        total += rows * o.shape[-1] * o.element_size()
+        return total
+
+    def io_tensors(self):
+        return self.ins, self.outs
+
+
+def _clone_layers(bufs, n):
+    """Layer 0's buffer and n-1 independent copies (distinct memory)."""
+    return [bufs] + [bufs.clone() for _ in range(n - 1)]
+
+
+class HlaStep(Step):
+    """HLA (Ouro-shaped): per layer the loop-1 read, the main read (loops 2..T
+    together in M1, one call per loop in M2) and the writer."""
+
+    def __init__(self, cfg, dev, mode, seed=1234):
+        super().__init__(cfg, dev, mode)
+        L = self.L
         c = cfg
         B, N, T, H, d_h, D = c.B, c.N, c.T, c.H, c.d_h, c.D
-        self.i = N - 1
-        Wcap = c.W + 1
-        codec = synth.hla_codec(c, seed)
+        codec = {k: v.to(dev) for k, v in synth.hla_codec(c, seed).items()}
         g = torch.Generator(device=dev)
         g.manual_seed(seed + 7)
-        self.layers = []
-        self.ws_bytes = 0
+        lat0 = torch.empty(B, N, c.r_k + c.r_v, dtype=torch.bfloat16, device=dev)
+        lat10 = torch.empty(B, N, 2 * c.r_1, dtype=torch.bfloat16, device=dev)
+        # prefill: the writer fills layer 0 from synthetic hidden states; the
+        # other layers get copies (the bytes every layer reads are its own)
+        chunk = max(1, (1 << 28) // (N * T * D))
+        for b0 in range(0, B, chunk):
+            nb = min(chunk, B - b0)
+            h = synth.hla_hidden(codec["P"], nb * (N - 1), seed + b0, D, device=dev).reshape(nb, N - 1, T, D)
+            L.lla_write_latents(L.LLA_WRITE_HLA, x=h, E_main=codec["E_main"], E_1=codec["E_1"],
+                                out0=lat0[b0:b0 + nb], out1=lat10[b0:b0 + nb], r_k=c.r_k, d_h=d_h,
+                                pos0=0, rope_base=c.base)
+            del h
+        lats = _clone_layers(lat0, c.L)
+        lat1s = _clone_layers(lat10, c.L)
+        self.ins, self.outs = [], []
         for layer in range(c.L):
-            lay = {}
-            for k in ("E_main", "E_1", "A", "A_1", "Bm", "B_1"):
-                lay[k] = codec[k].to(dev).clone()
-            lay["lat"] = torch.empty(B, N, c.r_k + c.r_v, dtype=torch.bfloat16, device=dev)
-            lay["lat1"] = torch.empty(B, N, 2 * c.r_1, dtype=torch.bfloat16, device=dev)
-            self._prefill(lay, codec["P"], seed + 100 * layer)
+            lay = {k: codec[k].clone() for k in ("E_main", "E_1", "A", "A_1", "Bm", "B_1")}
+            lay["lat"], lay["lat1"] = lats[layer], lat1s[layer]
+            Wcap = c.W + 1
             lay["wk"] = torch.randn(B, T, Wcap, H, d_h, generator=g, device=dev).to(torch.bfloat16)
             lay["wv"] = torch.randn(B, T, Wcap, H, d_h, generator=g, device=dev).to(torch.bfloat16)
             lay["q"] = torch.randn(B, T, H, d_h, generator=g, device=dev)
             lay["h"] = synth.hla_hidden(codec["P"], B, seed + 100 * layer + 1, D, device=dev).reshape(B, 1, T, D)
             lay["out"] = torch.empty(B, T, H, d_h, device=dev)
-            self.layers.append(lay)
-        self.calls = self._calls()
-        for kind, kw in self.calls:
-            nb = (L.hla_decode_workspace_bytes(**kw) if kind == "hla"
-                  else L.lla_write_workspace_bytes(L.LLA_WRITE_HLA, **kw))
-            self.ws_bytes = max(self.ws_bytes, nb)
-        self.ws = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=dev)
-
-    def _prefill(self, lay, P, seed):
-        c = self.cfg
-        L = self.L
-        chunk = max(1, (1 << 28) // (c.N * c.T * c.D))  # ~1 GiB of fp32 hidden states
-        for b0 in range(0, c.B, chunk):
-            nb = min(chunk, c.B - b0)
-            h = synth.hla_hidden(P, nb * (c.N - 1), seed + b0, c.D, device=self.dev).reshape(nb, c.N - 1, c.T, c.D)
-            L.lla_write_latents(L.LLA_WRITE_HLA, x=h, E_main=lay["E_main"], E_1=lay["E_1"],
-                                out0=lay["lat"][b0:b0 + nb], out1=lay["lat1"][b0:b0 + nb], r_k=c.r_k,
-                                d_h=c.d_h, pos0=0, rope_base=c.base)
-            del h
-
-    def _calls(self):
-        c = self.cfg
-        calls = []
-        for lay in self.layers:
-            common = dict(win_k=lay["wk"], win_v=lay["wv"], N=c.N, W=c.W, rope_base=c.base)
-            if self.mode == "m1":
-                groups = [(0, 1), (1, c.T - 1)]
-            else:
-                groups = [(t, 1) for t in range(c.T)]
+            self.ins += [lay["q"], lay["h"]]
+            self.outs.append(lay["out"])
+            common = dict(win_k=lay["wk"], win_v=lay["wv"], N=N, W=c.W, rope_base=c.base)
+            groups = [(0, 1), (1, T - 1)] if mode == "m1" else [(t, 1) for t in range(T)]
             for t0, nt in groups:
                 if t0 == 0:
                     kw = dict(lat=lay["lat1"], A=lay["A_1"], Bm=lay["B_1"], r_k=c.r_1)
+                    tag = "loop1"
                 else:
                     a = t0 - 1
                     kw = dict(lat=lay["lat"], A=lay["A"][a:a + nt], Bm=lay["Bm"][a:a + nt], r_k=c.r_k)
+                    tag = "main"
                 kw.update(common, q=lay["q"][:, t0:t0 + nt], out=lay["out"][:, t0:t0 + nt], t0=t0)
-                calls.append(("hla", kw))
-            calls.append(("write", dict(x=lay["h"], E_main=lay["E_main"], E_1=lay["E_1"],
-                                        out0=lay["lat"], out1=lay["lat1"], r_k=c.r_k, d_h=c.d_h,
-                                        pos0=self.i, rope_base=c.base)))
-        return calls
+                self.calls.append(("hla", kw, tag))
+            self.calls.append(("write", dict(mode=L.LLA_WRITE_HLA, x=lay["h"], E_main=lay["E_main"],
+                                             E_1=lay["E_1"], out0=lay["lat"], out1=lay["lat1"], r_k=c.r_k,
+                                             d_h=d_h, pos0=self.i, rope_base=c.base), None))
+        self._workspace()
 
-    def run(self, events=None):
+
+class Lla2dStep(Step):
+    """LLA-2D capacity regime: per layer one absorbed read of the folded latent
+    (all 4 loops x 16 heads = 64 rows share it; LLA-D, no rotation, W = 0) and
+    the folded writer.  The layers alternate between two latent buffers of
+    B x N x (r_K + r_V) bf16 (7.25 GB each at batch 768): every read streams
+    from HBM (each buffer is far larger than L2), 24 separate buffers would
+    not fit in 180 GB next to everything else."""
+
+    NBUF = 2
+
+    def __init__(self, cfg, dev, mode, seed=4321):
+        super().__init__(cfg, dev, mode)
         L = self.L
-        ei = 0
-        for kind, kw in self.calls:
-            if kind == "hla":
-                ev = None
-                if events is not None:
-                    ev = events[ei]
-                    ei += 1
-                L.hla_decode_attn(workspace=self.ws, timing_events=ev, **kw)
-            else:
-                L.lla_write_latents(L.LLA_WRITE_HLA, workspace=self.ws, **kw)
+        c = cfg
+        B, N, T, H, d_h = c.B, c.N, c.T, c.H, c.d_h
+        codec = {k: v.to(dev) for k, v in synth.lla_folded_codec(c, seed).items()}
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed + 7)
+        lat0 = torch.empty(B, N, c.r_k + c.r_v, dtype=torch.bfloat16, device=dev)
+        chunk = max(1, (1 << 28) // (N * T * H * d_h * 2))
+        for b0 in range(0, B, chunk):
+            nb = min(chunk, B - b0)
+            k, v = synth.lla_kv(codec["P"], nb * (N - 1), d_h, seed + b0, device=dev)
+            k = k.reshape(nb, N - 1, T, H, d_h)
+            v = v.reshape(nb, N - 1, T, H, d_h)
+            L.lla_write_latents(L.LLA_WRITE_FOLDED, x=k, xv=v, E_K=codec["E_K"], E_V=codec["E_V"],
+                                out0=lat0[b0:b0 + nb], pos0=0)
+            del k, v
+        lats = [lat0] + [lat0.clone() for _ in range(self.NBUF - 1)]
+        self.ins, self.outs = [], []
+        for layer in range(c.L):
+            lay = {"UK": codec["U_K"].clone(), "UVt": codec["U_V"].transpose(2, 3).contiguous(),
+                   "EK": codec["E_K"].clone(), "EV": codec["E_V"].clone(), "lat": lats[layer % self.NBUF]}
+            k_new, v_new = synth.lla_kv(codec["P"], B, d_h, seed + 1000 + layer, device=dev)
+            lay["k"] = k_new.reshape(B, 1, T, H, d_h)
+            lay["v"] = v_new.reshape(B, 1, T, H, d_h)
+            ring = 1   # W = 0: the ring holds the current token only
+            lay["wk"] = lay["k"].reshape(B, T, ring, H, d_h).to(torch.bfloat16)
+            lay["wv"] = lay["v"].reshape(B, T, ring, H, d_h).to(torch.bfloat16)
+            lay["q"] = torch.randn(B, T, H, d_h, generator=g, device=dev)
+            lay["out"] = torch.empty(B, T, H, d_h, device=dev)
+            self.ins += [lay["q"], lay["k"], lay["v"]]
+            self.outs.append(lay["out"])
+            self.calls.append(("hla", dict(lat=lay["lat"], A=lay["UK"], Bm=lay["UVt"], q=lay["q"],
+                                           win_k=lay["wk"], win_v=lay["wv"], out=lay["out"], N=N, W=0,
+                                           t0=0, rotate_query=False), "main"))
+            self.calls.append(("write", dict(mode=L.LLA_WRITE_FOLDED, x=lay["k"], xv=lay["v"], E_K=lay["EK"],
+                                             E_V=lay["EV"], out0=lay["lat"], pos0=self.i), None))
+        self._workspace()
 
-    def n_read_calls(self):
-        return sum(1 for k, _ in self.calls if k == "hla")
 
-    def kernel_launches(self):
-        n = 0
-        n_lat = max(0, self.i - self.cfg.W)
-        for kind, _ in self.calls:
-            n += (3 + (n_lat > 0)) if kind == "hla" else 2
-        return n
+class LlaStep(Step):
+    """LLA per-head reconstruct-on-read (Huginn-like): one layer, all T loops
+    of every head read their head's latents in one call, plus the per-head
+    writer for the new token."""
 
-    # algorithmic bytes
-    def split_bytes(self):
-        """Latent bytes each read call streams (its latent-read kernel)."""
-        c = self.cfg
-        n_lat = max(0, self.i - c.W)
-        out = []
-        for kind, kw in self.calls:
-            if kind == "hla":
-                width = kw["lat"].shape[-1]
-                out.append(c.B * n_lat * width * 2)
-        return out
-
-    def step_bytes(self):
-        c = self.cfg
-        n_lat = max(0, self.i - c.W)
-        n_win = self.i - n_lat + 1
-        total = 0
-        for kind, kw in self.calls:
-            if kind == "hla":
-                nt = kw["q"].shape[1]
-                total += c.B * n_lat * kw["lat"].shape[-1] * 2                       # latents
-                total += c.B * nt * n_win * c.H * c.d_h * 2 * 2                       # window K and V
-                total += (kw["A"].numel() + kw["Bm"].numel()) * 4                     # codec A, B
-            else:
-                total += (kw["E_main"].numel() + kw["E_1"].numel()) * 4               # writer codec
-                total += kw["x"].numel() * 4                                          # new token h
-                total += c.B * (kw["out0"].shape[-1] + kw["out1"].shape[-1]) * 2      # new rows
-        return total
-
-    def io_tensors(self):
-        ins = [lay["q"] for lay in self.layers] + [lay["h"] for lay in self.layers]
-        outs = [lay["out"] for lay in self.layers]
-        return ins, outs
+    def __init__(self, cfg, dev, mode, seed=777):
+        super().__init__(cfg, dev, mode)
+        L = self.L
+        c = cfg
+        B, N, T, H, d_h, r = c.B, c.N, c.T, c.H, c.d_h, c.r_k
+        codec = {k: v.to(dev) for k, v in synth.lla_perhead_codec(c, seed).items()}
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed + 7)
+        cK = torch.empty(B, H, N, r, dtype=torch.bfloat16, device=dev)
+        cV = torch.empty(B, H, N, r, dtype=torch.bfloat16, device=dev)
+        chunk = max(1, (1 << 28) // (N * T * H * d_h * 2))
+        for b0 in range(0, B, chunk):
+            nb = min(chunk, B - b0)
+            k, v = synth.lla_kv(codec["P"], nb * (N - 1), d_h, seed + b0, device=dev)
+            L.lla_write_latents(L.LLA_WRITE_PERHEAD, x=k.reshape(nb, N - 1, T, H, d_h),
+                                xv=v.reshape(nb, N - 1, T, H, d_h), E_K=codec["E_K"], E_V=codec["E_V"],
+                                out0=cK[b0:b0 + nb], out1=cV[b0:b0 + nb], pos0=0)
+            del k, v
+        k_new, v_new = synth.lla_kv(codec["P"], B, d_h, seed + 99, device=dev)
+        self.k = k_new.reshape(B, 1, T, H, d_h)
+        self.v = v_new.reshape(B, 1, T, H, d_h)
+        wk = self.k.reshape(B, T, 1, H, d_h).to(torch.bfloat16)
+        wv = self.v.reshape(B, T, 1, H, d_h).to(torch.bfloat16)
+        self.q = torch.randn(B, T, H, d_h, generator=g, device=dev)
+        self.out = torch.empty(B, T, H, d_h, device=dev)
+        self.ins, self.outs = [self.q, self.k, self.v], [self.out]
+        self.calls.append(("lla", dict(cK=cK, cV=cV, UK=codec["U_K"], UV=codec["U_V"], q=self.q, win_k=wk,
+                                       win_v=wv, out=self.out, N=N, W=0, t0=0), "main"))
+        self.calls.append(("write", dict(mode=L.LLA_WRITE_PERHEAD, x=self.k, xv=self.v, E_K=codec["E_K"],
+                                         E_V=codec["E_V"], out0=cK, out1=cV, pos0=self.i), None))
+        self._workspace()
 
 
 def make_step(cfg, dev, mode):
     if cfg.kind == "hla":
         return HlaStep(cfg, dev, mode)
-    raise SystemExit(f"config {cfg.name}: kind {cfg.kind} has no bench step yet")
+    if cfg.kind == "lla2d":
+        return Lla2dStep(cfg, dev, mode)
+    return LlaStep(cfg, dev, mode)
 
 
 # ------------------------------------------------------ oracle timing --
 def oracle_sample(cfg, seed=5):
-    """Time the oracle on one (sequence, layer) slice of a decode step.
+    """Time the oracle on one slice of a decode step, fp64 numpy.
 
-    Returns (seconds, threads): both absorbed reads of one sequence for one
-    layer plus the writer for its new token, in fp64 numpy.
-    """
+    HLA and LLA-2D: one (sequence, layer) slice -- its reads and the writer for
+    its new token.  LLA reconstruct: one (sequence, head) slice of the single
+    layer -- all T loops of that head.  Returns (seconds, threads, slices per
+    decoded token)."""
     import numpy as np
-    from oracle import hla
+    from oracle import hla, lla
     c = cfg
     rng = np.random.default_rng(seed)
     n = c.N
-    lat = rng.standard_normal((n, c.r_k + c.r_v)) * math.sqrt(c.d_h / c.r_k)
-    lat1 = rng.standard_normal((n, 2 * c.r_1)) * math.sqrt(c.d_h / c.r_1)
-    A = rng.standard_normal((c.T - 1, c.H, c.d_h, c.r_k)) / math.sqrt(c.d_h)
-    A1 = rng.standard_normal((1, c.H, c.d_h, c.r_1)) / math.sqrt(c.d_h)
-    Bm = rng.standard_normal((c.T - 1, c.H, c.r_v, c.d_h)) / math.sqrt(c.r_v)
-    B1 = rng.standard_normal((1, c.H, c.r_1, c.d_h)) / math.sqrt(c.r_1)
-    q = rng.standard_normal((c.T, c.H, c.d_h))
-    wk = rng.standard_normal((c.T, c.W + 1, c.H, c.d_h))
-    wv = rng.standard_normal((c.T, c.W + 1, c.H, c.d_h))
-    h = rng.standard_normal((1, c.T, c.D))
-    E = rng.standard_normal((c.T - 1, c.r_k + c.r_v, c.D)) / math.sqrt(c.D)
-    E1 = rng.standard_normal((2 * c.r_1, c.D)) / math.sqrt(c.D)
-    t = time.perf_counter()
-    hla.decode(lat1, A1, B1, q[:1], wk, wv, 0, c.N, c.W, c.r_1, c.r_1, c.d_h, c.base)
-    hla.decode(lat, A, Bm, q[1:], wk, wv, 1, c.N, c.W, c.r_k, c.r_v, c.d_h, c.base)
-    hla.write(h, E, E1, c.N - 1, c.r_k, c.r_v, c.r_1, c.d_h, c.base)
+    if c.kind == "hla":
+        lat = rng.standard_normal((n, c.r_k + c.r_v)) * math.sqrt(c.d_h / c.r_k)
+        lat1 = rng.standard_normal((n, 2 * c.r_1)) * math.sqrt(c.d_h / c.r_1)
+        A = rng.standard_normal((c.T - 1, c.H, c.d_h, c.r_k)) / math.sqrt(c.d_h)
+        A1 = rng.standard_normal((1, c.H, c.d_h, c.r_1)) / math.sqrt(c.d_h)
+        Bm = rng.standard_normal((c.T - 1, c.H, c.r_v, c.d_h)) / math.sqrt(c.r_v)
+        B1 = rng.standard_normal((1, c.H, c.r_1, c.d_h)) / math.sqrt(c.r_1)
+        q = rng.standard_normal((c.T, c.H, c.d_h))
+        wk = rng.standard_normal((c.T, c.W + 1, c.H, c.d_h))
+        wv = rng.standard_normal((c.T, c.W + 1, c.H, c.d_h))
+        h = rng.standard_normal((1, c.T, c.D))
+        E = rng.standard_normal((c.T - 1, c.r_k + c.r_v, c.D)) / math.sqrt(c.D)
+        E1 = rng.standard_normal((2 * c.r_1, c.D)) / math.sqrt(c.D)
+        t = time.perf_counter()
+        hla.decode(lat1, A1, B1, q[:1], wk, wv, 0, c.N, c.W, c.r_1, c.r_1, c.d_h, c.base)
+        hla.decode(lat, A, Bm, q[1:], wk, wv, 1, c.N, c.W, c.r_k, c.r_v, c.d_h, c.base)
+        hla.write(h, E, E1, c.N - 1, c.r_k, c.r_v, c.r_1, c.d_h, c.base)
+        per_token = c.L
+    elif c.kind == "lla2d":
+        lat = rng.standard_normal((n, c.r_k + c.r_v)) * math.sqrt(c.d_h / c.r_k)
+        UK = rng.standard_normal((c.T, c.H, c.d_h, c.r_k)) / math.sqrt(c.r_k)
+        UV = rng.standard_normal((c.T, c.H, c.d_h, c.r_v)) / math.sqrt(c.r_v)
+        EK = rng.standard_normal((c.T, c.H, c.r_k, c.d_h)) / math.sqrt(c.d_h)
+        EV = rng.standard_normal((c.T, c.H, c.r_v, c.d_h)) / math.sqrt(c.d_h)
+        q = rng.standard_normal((c.T, c.H, c.d_h))
+        k = rng.standard_normal((1, c.T, c.H, c.d_h))
+        v = rng.standard_normal((1, c.T, c.H, c.d_h))
+        t = time.perf_counter()
+        lla.decode_absorbed(lat, UK, UV, q, k[0][:, None], v[0][:, None], 0, c.N, 0, c.r_k, c.r_v)
+        lla.write_folded(k, v, EK, EV)
+        per_token = c.L
+    else:
+        cK = rng.standard_normal((1, n, c.r_k))
+        cV = rng.standard_normal((1, n, c.r_k))
+        UK = rng.standard_normal((c.T, 1, c.d_h, c.r_k)) / math.sqrt(c.r_k)
+        UV = rng.standard_normal((c.T, 1, c.d_h, c.r_k)) / math.sqrt(c.r_k)
+        q = rng.standard_normal((c.T, 1, c.d_h))
+        wk = rng.standard_normal((c.T, 1, 1, c.d_h))
+        wv = rng.standard_normal((c.T, 1, 1, c.d_h))
+        t = time.perf_counter()
+        lla.decode_reconstruct(cK, cV, UK, UV, q, wk, wv, 0, c.N, 0)
+        per_token = c.H * c.L
     dt = time.perf_counter() - t
-    return dt, _blas_threads()
+    return dt, _blas_threads(), per_token
 
 
 def _blas_threads():
@@ -275,16 +417,20 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
+def _slice_name(cfg):
+    return "(sequence, head) slices of the single layer" if cfg.kind == "lla" else "(sequence, layer) slices"
+
+
 def cpu_baseline(cfg, budget_s=12.0):
-    total, n, threads = 0.0, 0, 1
+    total, n, threads, per_token = 0.0, 0, 1, 1
     while total < budget_s and n < 512:
-        dt, threads = oracle_sample(cfg, seed=5 + n)
+        dt, threads, per_token = oracle_sample(cfg, seed=5 + n)
         total += dt
         n += 1
-    tok_s = n / (cfg.L * total)   # n (sequence, layer) slices; a token needs L of them
+    tok_s = n / (per_token * total)   # a decoded token needs per_token slices
     return {"value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n} (sequence, layer) slices of the {cfg.name} step "
-                      f"(both reads + writer, fp64 numpy), {total:.1f} s; tokens/s = slices / (L * time)"}
+            "sample": f"{n} {_slice_name(cfg)} of the {cfg.name} step (fp64 numpy), {total:.1f} s; "
+                      f"tokens/s = slices / ({per_token} slices per token x time)"}
 
 
 # ---------------------------------------------------------------- main --
@@ -304,23 +450,40 @@ def run_reference(args, cfg):
         return
     for w in range(args.warmup):
         oracle_sample(cfg, seed=100 + w)
-    times, threads = [], 1
+    times, threads, per_token = [], 1, 1
     for s in range(args.steps):
-        dt, threads = oracle_sample(cfg, seed=200 + s)
+        dt, threads, per_token = oracle_sample(cfg, seed=200 + s)
         times.append(dt)
     total = sum(times)
-    v = args.steps / (cfg.L * total)
+    v = args.steps / (per_token * total)
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.L * total / args.steps,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * per_token * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": cfg.name, "mode": args.mode,
-                                        "sample": "one (sequence, layer) slice per step"},
+                                        "sample": f"one of the {_slice_name(cfg)} per step"},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{args.steps} (sequence, layer) slices of {cfg.name}, {total:.1f} s"},
+                         "sample": f"{args.steps} {_slice_name(cfg)} of {cfg.name}, {total:.1f} s"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
+
+
+# DRAM traffic (read + write) per latent token of the tensor-core latent read,
+# from one ncu capture of the Ouro main latent (profiles/absorb_split_tc_ouro_main_b16.md),
+# keyed by the sha256 prefix of the kernel source it was taken on: a changed
+# kernel reports no traffic until it is captured again.
+TC_TRAFFIC_PER_TOKEN = {"5163ad08b2a9e31d": 2122.7}
+
+
+def tc_traffic_per_token():
+    import hashlib
+    src = os.path.join(ROOT, "looped_transformer_latent_b200", "csrc", "decode_tc.cu")
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return TC_TRAFFIC_PER_TOKEN.get(h)
 
 
 def main():
@@ -346,7 +509,8 @@ def main():
     build.build()
     step = make_step(cfg, dev, args.mode)
     stream = torch.cuda.Stream(dev)
-    nread = step.n_read_calls()
+    tags = step.read_tags()
+    nread = len(tags)
     evs = [(torch.cuda.Event(enable_timing=True, external=True),
             torch.cuda.Event(enable_timing=True, external=True)) for _ in range(nread)]
     with torch.cuda.stream(stream):
@@ -430,11 +594,21 @@ def main():
         ms_e2e = float(tt.item())
 
     hbm, tflops, src = peaks()
-    sb = step.split_bytes()
-    tot_split_ms = sum(split_ms)
-    achieved = (sum(sb) / 1e9) / (tot_split_ms / 1e3) if tot_split_ms > 0 else 0.0
+    lb = step.read_latent_bytes()
+    main_ix = [k for k, t in enumerate(tags) if t == "main"]
+    main_ms = [split_ms[k] for k in main_ix]
+    main_bytes = [lb[k] for k in main_ix]
+    mean_ms = sum(main_ms) / max(1, len(main_ms))
+    achieved = (sum(main_bytes) / 1e9) / (sum(main_ms) / 1e3) if sum(main_ms) > 0 else 0.0
+    all_gbs = (sum(lb) / 1e9) / (sum(split_ms) / 1e3) if sum(split_ms) > 0 else 0.0
+    per_tok = tc_traffic_per_token() if cfg.kind != "lla" else None
+    traffic = None
+    if per_tok is not None and main_ix:
+        c0 = cfg
+        traffic = per_tok * c0.B * step.n_lat
     step_bytes = step.step_bytes()
     tokens = cfg.B * world
+    srt = sorted(main_ms)
     line = {
         "metric": METRIC,
         "value": tokens / (ms / 1e3),
@@ -461,13 +635,32 @@ def main():
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": step.kernel_launches() * args.steps,
         "clocks": clocks,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None,
-                     "kernel": "latent-read split kernel (absorbed read)",
-                     "peak_source": src,
-                     "per_launch_ms": tot_split_ms / max(1, len(split_ms)),
-                     "launches_per_step": len(split_ms)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm,
+                     "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
+                     "kernel": "tensor-core latent read (absorb_split_tc), main-latent launches",
+                     "peak_source": src, "per_launch_ms": mean_ms,
+                     "per_launch_ms_min_med_max": [srt[0], srt[len(srt) // 2], srt[-1]] if srt else None,
+                     "launches_per_step": len(main_ix),
+                     "algorithmic_bytes_per_launch": (sum(main_bytes) / max(1, len(main_bytes))),
+                     "all_latent_reads_gbs": all_gbs,
+                     "timing": "CUDA events around each latent-read kernel in the captured step, "
+                               "read after the last replay of the timed region"},
     }
+    if cfg.kind == "lla":
+        # reconstruct-on-read is bound by the fp32 reconstruction arithmetic:
+        # per latent token, loop and head 2*2*d_h*r flops (k^ and v^) plus
+        # 2*2*d_h for the score and the weighted sum.  Peak: 148 SMs x 128
+        # fp32 lanes x 2 flops x the maximum SM clock.
+        flops = cfg.B * cfg.T * cfg.H * step.n_lat * (4.0 * cfg.d_h * cfg.r_k + 4.0 * cfg.d_h)
+        tf = flops / 1e12 / (mean_ms / 1e3) if mean_ms > 0 else 0.0
+        max_mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
+        alu_peak = 148 * 128 * 2 * max_mhz * 1e6 / 1e12
+        line["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu_peak, "unit": "TFLOP/s",
+                            "frac": tf / alu_peak, "traffic": None,
+                            "kernel": "LLA reconstruct-on-read (recon_split_simt)",
+                            "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x max SM clock",
+                            "per_launch_ms": mean_ms, "flops_per_launch": flops,
+                            "latent_gbs": achieved, "launches_per_step": len(main_ix)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg)
     if rank == 0:

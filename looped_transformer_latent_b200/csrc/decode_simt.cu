@@ -115,24 +115,37 @@ __global__ void __launch_bounds__(256) absorb_split_simt(AbsorbArgs a) {
 // per token), each warp takes every 4th group of WU tokens and issues all of a
 // group's K and V loads before using them, keeps its own online softmax, and
 // the four warps are combined at the end.  Emits (max, sum, y_w) in base-2 units.
-constexpr int WU = 8;
-
 template <bool BF16>
-__device__ __forceinline__ void load4(const void* base, int64_t idx, float* v) {
-  if (BF16) {
-    const uint2 u = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(base) + idx);
-    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
-    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
-    const float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
-    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
-  } else {
-    const float4 f = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx);
-    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+struct WinTraits;
+template <>
+struct WinTraits<true> {   // 4 bf16 per lane, packed in a uint2
+  typedef uint2 raw_t;
+  static constexpr int WU = 16;
+  __device__ __forceinline__ static raw_t load(const void* base, int64_t idx) {
+    return *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(base) + idx);
   }
-}
+  __device__ __forceinline__ static void unpack(raw_t u, float* v) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  }
+  __device__ __forceinline__ static raw_t zero() { return make_uint2(0u, 0u); }
+};
+template <>
+struct WinTraits<false> {  // 4 fp32 per lane
+  typedef float4 raw_t;
+  static constexpr int WU = 8;
+  __device__ __forceinline__ static raw_t load(const void* base, int64_t idx) {
+    return *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx);
+  }
+  __device__ __forceinline__ static void unpack(raw_t u, float* v) { v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w; }
+  __device__ __forceinline__ static raw_t zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+};
 
 template <bool BF16>
 __global__ void __launch_bounds__(128) window_attn(WindowArgs w) {
+  typedef WinTraits<BF16> Tr;
+  constexpr int WU = Tr::WU;
   const int row = blockIdx.x, b = blockIdx.y;
   const int tt = row / w.H, h = row % w.H, t = w.t0 + tt;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -147,43 +160,55 @@ __global__ void __launch_bounds__(128) window_attn(WindowArgs w) {
   float m = -INFINITY, l = 0.f;
   const int64_t seq = (int64_t)b * w.wins_b;
   for (int g0 = warp * WU; g0 < w.n_win; g0 += 4 * WU) {
-    float kk[WU][4], vv[WU][4];
+    typename Tr::raw_t kr[WU], vr[WU];
 #pragma unroll
     for (int u = 0; u < WU; ++u) {
       const int idx = g0 + u;
       if (dv && idx < w.n_win) {
         const int slot = (w.win_start + idx) % w.Wcap;
         const int64_t base = seq + (((int64_t)t * w.Wcap + slot) * w.H + h) * w.d_h + d0;
-        load4<BF16>(w.wk, base, kk[u]);
-        load4<BF16>(w.wv, base, vv[u]);
+        kr[u] = Tr::load(w.wk, base);
+        vr[u] = Tr::load(w.wv, base);
       } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) kk[u][e] = vv[u][e] = 0.f;
+        kr[u] = Tr::zero();
+        vr[u] = Tr::zero();
       }
     }
     float sc[WU];
 #pragma unroll
     for (int u = 0; u < WU; ++u) {
+      float kk[4];
+      Tr::unpack(kr[u], kk);
       float part = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) part = fmaf(qv[e], kk[u][e], part);
+      for (int e = 0; e < 4; ++e) part = fmaf(qv[e], kk[e], part);
       sc[u] = part;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
       for (int u = 0; u < WU; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
+    // one max per group of tokens, then a single rescale of the running state
+    float gm = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < WU; ++u)
+      if (g0 + u < w.n_win) gm = fmaxf(gm, sc[u]);
+    const float mn = fmaxf(m, gm);
+    const float al = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+    l *= al;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] *= al;
 #pragma unroll
     for (int u = 0; u < WU; ++u) {
       if (g0 + u >= w.n_win) break;
-      const float mn = fmaxf(m, sc[u]);
-      const float al = (m == -INFINITY) ? 0.f : exp2f(m - mn);
       const float p = exp2f(sc[u] - mn);
-      l = l * al + p;
+      float vv[4];
+      Tr::unpack(vr[u], vv);
+      l += p;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[e] = fmaf(p, vv[u][e], acc[e] * al);
-      m = mn;
+      for (int e = 0; e < 4; ++e) acc[e] = fmaf(p, vv[e], acc[e]);
     }
+    m = mn;
   }
   __shared__ float sm_m[4], sm_l[4], sm_y[4][128];
   if (lane == 0) { sm_m[warp] = m; sm_l[warp] = l; }

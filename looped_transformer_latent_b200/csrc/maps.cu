@@ -5,8 +5,8 @@
 //
 // Both are, for every query row (loop t, head h), a [B x K] x [K x N] product
 // with that row's own codec matrix W_row = A_{t,h} (K = d_h, N = r_k) or
-// B_{t,h} (K = r_v, N = d_h).  One CTA computes a 32-sequence x 64-column tile
-// of one row: K is walked in chunks of 32 staged in shared memory (both the
+// B_{t,h} (K = r_v, N = d_h).  One CTA computes a 16- or 32-sequence x
+// 64-column tile of one row: K is walked in chunks of 64 staged in shared memory (both the
 // activations and the codec tile), the next chunk is fetched into registers
 // while the current one is multiplied, and each thread owns one column pair
 // (so the query map can rotate the pair in its epilogue) for four sequences.
@@ -19,7 +19,6 @@ namespace lla {
 namespace {
 
 constexpr int GN = 64;      // columns per tile (32 pairs)
-constexpr int GK = 32;      // reduction chunk
 constexpr int GT = 256;     // threads
 constexpr int MAXS = 16;    // split partials the output map can combine
 
@@ -28,7 +27,7 @@ __device__ __forceinline__ int64_t qbf_index(int b, int row, int k, int r_k) {
   return (int64_t)b * (r_k >> 6) * 4096 + kb * 4096 + row * 64 + ((((e >> 3) ^ (row & 7)) << 3) | (e & 7));
 }
 
-template <int MODE, int GB>
+template <int MODE, int GB, int GK>
 __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
   constexpr int BPW = GB / (GT / 32);   // sequences per warp
   constexpr int LX = GB * GK / GT;      // activation loads per thread
@@ -98,8 +97,9 @@ __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
   const float* Wr = g.W + (int64_t)row * g.K * g.N;
   // loader coordinates
   const int xb = tid / (GK / LX), xk = (tid % (GK / LX)) * LX;   // X: GB sequences x 32 k
-  const int wk = tid >> 3, wn = (tid & 7) * 8;      // W: 32 k x 64 columns
-  float xr[LX], wr[8];
+  constexpr int LW = GK * GN / GT;                  // codec loads per thread
+  const int wk = tid / (GN / LW), wn = (tid % (GN / LW)) * LW;   // W: GK k x 64 columns
+  float xr[LX], wr[LW];
   auto load = [&](int k0) {
     const int b = b0 + xb;
 #pragma unroll
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
     }
     const int k = k0 + wk;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < LW; ++u) {
       const int n = n0 + wn + u;
       wr[u] = (k < g.K && n < g.N) ? __ldg(Wr + (int64_t)k * g.N + n) : 0.f;
     }
@@ -127,8 +127,9 @@ __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
   auto stash = [&](int buf) {
 #pragma unroll
     for (int u = 0; u < LX; ++u) Xs[buf][xk + u][xb] = xr[u];
-    *reinterpret_cast<float4*>(&Ws[buf][wk][wn]) = make_float4(wr[0], wr[1], wr[2], wr[3]);
-    *reinterpret_cast<float4*>(&Ws[buf][wk][wn + 4]) = make_float4(wr[4], wr[5], wr[6], wr[7]);
+#pragma unroll
+    for (int u = 0; u < LW; u += 4)
+      *reinterpret_cast<float4*>(&Ws[buf][wk][wn + u]) = make_float4(wr[u], wr[u + 1], wr[u + 2], wr[u + 3]);
   };
 
   float acc[BPW][2] = {};
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
   for (int kc = 0; kc < nk; ++kc) {
     const int buf = kc & 1;
     if (kc + 1 < nk) load((kc + 1) * GK);
-#pragma unroll 8
+#pragma unroll 16
     for (int k = 0; k < GK; ++k) {
       const float2 w = *reinterpret_cast<const float2*>(&Ws[buf][k][2 * tn]);
 #pragma unroll
@@ -196,17 +197,17 @@ int map_max_splits() { return MAXS; }
 cudaError_t launch_query_map(const MapArgs& g, cudaStream_t st) {
   const int ntile = (g.N + GN - 1) / GN;
   dim3 grid(g.use_tc ? 64 : g.rows, ntile + 1, (g.B + 31) / 32);
-  row_gemm<0, 32><<<grid, GT, 0, st>>>(g);
+  row_gemm<0, 32, 32><<<grid, GT, 0, st>>>(g);
   return cudaGetLastError();
 }
 
 cudaError_t launch_output_map(const MapArgs& g, cudaStream_t st) {
   if (g.B <= 64) {
     dim3 grid(g.rows, (g.N + GN - 1) / GN, (g.B + 15) / 16);
-    row_gemm<1, 16><<<grid, GT, 0, st>>>(g);
+    row_gemm<1, 16, 32><<<grid, GT, 0, st>>>(g);
   } else {
     dim3 grid(g.rows, (g.N + GN - 1) / GN, (g.B + 31) / 32);
-    row_gemm<1, 32><<<grid, GT, 0, st>>>(g);
+    row_gemm<1, 32, 32><<<grid, GT, 0, st>>>(g);
   }
   return cudaGetLastError();
 }

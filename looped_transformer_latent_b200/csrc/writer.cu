@@ -10,7 +10,7 @@
 namespace lla {
 namespace {
 
-constexpr int BK = 16, WT = 256;
+constexpr int BK = 32, WT = 256;
 
 struct Slice {
   const float* X;
@@ -67,7 +67,7 @@ __device__ __forceinline__ Slice slice_of(const WriterArgs& a, int z) {
 }
 
 // Phase 1: C_part[z][split][m][n] = sum over this split's k-chunks.  Tile
-// TM x TN (64 x 64, or 32 x 128 for decode-size batches), 16-deep k-chunks
+// TM x TN (64 x 64, or 32 x 128 for decode-size batches), 32-deep k-chunks
 // staged in shared memory, the next chunk prefetched into registers while the
 // current one is multiplied; each thread owns a 4 x 4 block of outputs.
 template <int TM, int TN>
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(WT) writer_gemm(WriterArgs a) {
   const int n0 = blockIdx.x * TN, m0 = blockIdx.y * TM;
   if (n0 >= s.N) return;
   const int K = s.K_outer * s.d_in;
-  const int nk = K / BK;
+  const int nk = (K + BK - 1) / BK;
   const int kc0 = (int)((int64_t)nk * split / a.S), kc1 = (int)((int64_t)nk * (split + 1) / a.S);
 
   __shared__ float As[2][BK][TM + 4];
@@ -99,16 +99,20 @@ __global__ void __launch_bounds__(WT) writer_gemm(WriterArgs a) {
   const int n = n0 + br;
   const bool nval = n < s.N;
   float ra[LA], rb[LB];
+  // Each thread's run of LA (LB) consecutive k values is aligned and no longer
+  // than 16, and feature blocks (d_in) are multiples of 16, so a run never
+  // crosses from one (loop, head) block into the next.
   auto load = [&](int kc) {
-    const int k = kc * BK;
-    const int o = k / s.d_in, d = k % s.d_in;
-    const int64_t xo = (int64_t)(o / s.o_h) * s.x_o_t + (int64_t)(o % s.o_h) * s.x_o_h;
-    const float* xp = s.X + xrow + xo + d + ak;
-    const float* ep = s.E + (int64_t)o * s.e_o + (int64_t)n * s.e_n + d + bk;
+    const int ka = kc * BK + ak, kb = kc * BK + bk;
+    const bool av = mval && ka < K, bvld = nval && kb < K;
+    const int oa = av ? ka / s.d_in : 0, da = av ? ka % s.d_in : 0;
+    const int ob = bvld ? kb / s.d_in : 0, db = bvld ? kb % s.d_in : 0;
+    const float* xp = s.X + xrow + (int64_t)(oa / s.o_h) * s.x_o_t + (int64_t)(oa % s.o_h) * s.x_o_h + da;
+    const float* ep = s.E + (int64_t)ob * s.e_o + (int64_t)n * s.e_n + db;
 #pragma unroll
-    for (int u = 0; u < LA; ++u) ra[u] = mval ? __ldg(xp + u) : 0.f;
+    for (int u = 0; u < LA; ++u) ra[u] = av ? __ldg(xp + u) : 0.f;
 #pragma unroll
-    for (int u = 0; u < LB; ++u) rb[u] = nval ? __ldg(ep + u) : 0.f;
+    for (int u = 0; u < LB; ++u) rb[u] = bvld ? __ldg(ep + u) : 0.f;
   };
   auto stash = [&](int buf) {
 #pragma unroll
@@ -194,17 +198,17 @@ size_t writer_workspace_floats(const WriterArgs& a) {
 static bool small_batch(const WriterArgs& a) { return a.M <= 32; }
 
 int writer_pick_splits(const WriterArgs& a, int num_sms) {
-  // enough CTAs for two waves; never more splits than 16-wide k-chunks
+  // about four CTAs per SM; never more splits than k-chunks
   const int tm = small_batch(a) ? 32 : 64, tn = small_batch(a) ? 128 : 64;
   const int tiles = ceil_div(a.Nmax, tn) * ceil_div(a.M, tm) * a.Z;
   int K = 0;
   if (a.mode == LLA_WRITE_HLA) K = a.D;  // smallest GEMM depth (loop-1)
   else if (a.mode == LLA_WRITE_PERHEAD) K = a.T * a.d_h;
   else K = a.T * a.H * a.d_h;
-  const int nk = K / BK;
-  int S = ceil_div(2 * num_sms, tiles > 0 ? tiles : 1);
+  const int nk = ceil_div(K, BK);
+  int S = ceil_div(4 * num_sms, tiles > 0 ? tiles : 1);
   if (S > nk) S = nk;
-  if (S > 64) S = 64;
+  if (S > 96) S = 96;
   if (S < 1) S = 1;
   return S;
 }

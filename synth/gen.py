@@ -93,7 +93,7 @@ def hla_hidden(P, n, seed, D, device="cpu", dtype=torch.float32):
     T, R = P.shape
     P = P.to(device=device, dtype=dtype)
     u = torch.randn(n, R, D, generator=g, device=device, dtype=dtype)
-    h = torch.einsum("ts,nsd->ntd", P, u)
+    h = torch.einsum("ts,nsd->ntd", P, u).contiguous()
     h += NOISE * torch.randn(n, T, D, generator=g, device=device, dtype=dtype)
     return h
 
@@ -173,7 +173,7 @@ def lla_kv(P, n, d_h, seed, device="cpu", dtype=torch.float32):
     out = []
     for _ in range(2):
         u = torch.randn(n, H, R, d_h, generator=g, device=device, dtype=dtype)
-        x = torch.einsum("hts,nhsd->nthd", P, u)
+        x = torch.einsum("hts,nhsd->nthd", P, u).contiguous()
         x += NOISE * torch.randn(n, T, H, d_h, generator=g, device=device, dtype=dtype)
         out.append(x)
     return out[0], out[1]
