@@ -95,7 +95,9 @@ WriterArgs writer_args(const lla_write_params& p) {
     a.Z = 2; a.Nmax = std::max(p.r_k, p.r_v);
   }
   a.Nmax += a.Nmax % 2;
-  a.S = writer_pick_splits(a, 148);
+  // tensor cores (3xTF32, fp32-accurate) when the rows are stored as bf16
+  a.use_tc = p.out_dtype == LLA_BF16 && writer_tc_ok(a);
+  a.S = a.use_tc ? writer_tc_splits(a, kNumSms) : writer_pick_splits(a, kNumSms);
   return a;
 }
 
@@ -161,8 +163,8 @@ int check_lla(const lla_decode_params& p) {
 
 // Workspace layout of the absorbed read.
 struct HlaPlan {
-  int rows, n_lat, win_start, n_win, S, tps, use_tc, rows_pad;
-  size_t o_qlat, o_qwin, o_pml, o_py, o_wml, o_wy, o_qbf, o_err, bytes;
+  int rows, n_lat, win_start, n_win, S, tps, use_tc, rows_pad, Sw, cpt, HG;
+  size_t o_qlat, o_pml, o_py, o_wml, o_wy, o_qbf, o_err, bytes;
 };
 
 HlaPlan plan_hla(const hla_decode_params& p) {
@@ -190,15 +192,15 @@ HlaPlan plan_hla(const hla_decode_params& p) {
   } else {
     pl.S = 0; pl.tps = 0;
   }
+  pl.Sw = window_chunks(p.B, p.nt, p.H, pl.n_win, p.win_dtype, p.d_h, kNumSms, &pl.cpt, &pl.HG);
   const size_t br = (size_t)p.B * pl.rows;
   Carve c;
+  pl.o_qbf = c.take(pl.use_tc ? (size_t)p.B * 64 * p.r_k * 2 : 0);
   pl.o_qlat = c.take(pl.use_tc ? 0 : br * p.r_k * 4);
-  pl.o_qwin = c.take(br * p.d_h * 4);
   pl.o_pml = c.take((size_t)pl.S * br * 2 * 4);
   pl.o_py = c.take((size_t)pl.S * br * p.r_v * 4);
-  pl.o_wml = c.take(br * 2 * 4);
-  pl.o_wy = c.take(br * p.d_h * 4);
-  pl.o_qbf = c.take(pl.use_tc ? (size_t)p.B * 64 * p.r_k * 2 : 0);
+  pl.o_wml = c.take((size_t)pl.Sw * br * 2 * 4);
+  pl.o_wy = c.take((size_t)pl.Sw * br * p.d_h * 4);
   pl.o_err = c.take(sizeof(int));
   pl.bytes = c.off;
   return pl;
@@ -221,14 +223,15 @@ HlaPlan plan_lla(const lla_decode_params& p) {
   } else {
     pl.S = 0; pl.tps = 0;
   }
+  pl.Sw = window_chunks(p.B, p.nt, p.H, pl.n_win, p.win_dtype, p.d_h, kNumSms, &pl.cpt, &pl.HG);
   const size_t br = (size_t)p.B * pl.rows;
   Carve c;
   pl.o_qlat = 0;
-  pl.o_qwin = 0;
   pl.o_pml = c.take((size_t)pl.S * br * 2 * 4);
   pl.o_py = c.take((size_t)pl.S * br * p.d_h * 4);
-  pl.o_wml = c.take(br * 2 * 4);
-  pl.o_wy = c.take(br * p.d_h * 4);
+  pl.o_wml = c.take((size_t)pl.Sw * br * 2 * 4);
+  pl.o_wy = c.take((size_t)pl.Sw * br * p.d_h * 4);
+  pl.o_err = c.take(sizeof(int));
   pl.bytes = c.off;
   return pl;
 }
@@ -325,12 +328,11 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
   const float scale = p->scale > 0.f ? p->scale : 1.0f / std::sqrt((float)p->d_h);
   a.qmul = scale * kLog2e;
   a.qlat = reinterpret_cast<float*>(w + pl.o_qlat);
-  a.qwin = reinterpret_cast<float*>(w + pl.o_qwin);
   a.part_ml = reinterpret_cast<float*>(w + pl.o_pml);
   a.part_y = reinterpret_cast<float*>(w + pl.o_py);
   a.win_ml = reinterpret_cast<float*>(w + pl.o_wml);
   a.win_y = reinterpret_cast<float*>(w + pl.o_wy);
-  a.S = pl.S; a.tps = pl.tps;
+  a.S = pl.S; a.tps = pl.tps; a.Sw = pl.Sw; a.cpt = pl.cpt;
   a.use_tc = pl.use_tc; a.rows_pad = pl.rows_pad;
   a.qbf = reinterpret_cast<__nv_bfloat16*>(w + pl.o_qbf);
   a.err = reinterpret_cast<int*>(w + pl.o_err);
@@ -340,10 +342,10 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
   qm.B = a.B; qm.rows = a.rows; qm.K = a.d_h; qm.N = a.r_k; qm.d_h = a.d_h;
   qm.W = a.A; qm.X = a.q; qm.xs_b = a.qs_b; qm.xs_row = a.d_h;
   qm.rotate = a.rotate; qm.pos = a.N - 1; qm.use_tc = a.use_tc; qm.base = a.base; qm.qmul = a.qmul;
-  qm.qlat = a.qlat; qm.qwin = a.qwin; qm.qbf = a.qbf;
+  qm.qlat = a.qlat; qm.qbf = a.qbf;
   cudaError_t e = cudaSuccess;
-  if (a.use_tc) e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
-  if (e == cudaSuccess) e = launch_query_map(qm, s);
+  e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = query_map_tc_ok(qm) ? launch_query_map_tc(qm, a.err, s) : launch_query_map(qm, s);
   if (e == cudaSuccess) e = mark(p->timing_events, 0, s);
   if (e == cudaSuccess && a.n_lat > 0)
     e = a.use_tc ? launch_absorb_split_tc(a, s) : launch_absorb_split_simt(a, s);
@@ -351,10 +353,11 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
   if (e == cudaSuccess) {
     WindowArgs wa;
     wa.B = a.B; wa.rows = a.rows; wa.H = a.H; wa.d_h = a.d_h; wa.t0 = a.t0; wa.Wcap = a.Wcap;
-    wa.win_start = a.win_start; wa.n_win = a.n_win; wa.wk = a.wk; wa.wv = a.wv;
-    wa.dtype = a.win_dtype; wa.wins_b = a.wins_b;
-    wa.q = a.qwin; wa.q_sb = (int64_t)a.rows * a.d_h; wa.q_srow = a.d_h; wa.qmul = 1.f;
-    wa.win_ml = a.win_ml; wa.win_y = a.win_y;
+    wa.win_start = a.win_start; wa.n_win = a.n_win; wa.Sw = a.Sw; wa.cpt = a.cpt; wa.HG = pl.HG;
+    wa.wk = a.wk; wa.wv = a.wv; wa.dtype = a.win_dtype; wa.wins_b = a.wins_b;
+    wa.q = a.q; wa.q_sb = a.qs_b; wa.q_srow = a.d_h; wa.qmul = a.qmul;
+    wa.rotate = a.rotate; wa.pos = a.N - 1; wa.base = a.base;
+    wa.win_ml = a.win_ml; wa.win_y = a.win_y; wa.err = a.err;
     e = launch_window(wa, s);
   }
   if (e == cudaSuccess) {
@@ -362,8 +365,9 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
     std::memset(&om, 0, sizeof(om));
     om.B = a.B; om.rows = a.rows; om.K = a.r_v; om.N = a.d_h; om.d_h = a.d_h; om.W = a.Bm;
     om.part_ml = a.part_ml; om.part_y = a.part_y; om.win_ml = a.win_ml; om.win_y = a.win_y; om.S = a.S;
-    om.out = a.out; om.outs_b = a.outs_b; om.err = a.use_tc ? a.err : nullptr;
-    e = launch_output_map(om, s);
+    om.Sw = a.Sw;
+    om.out = a.out; om.outs_b = a.outs_b; om.err = a.err;
+    e = (a.use_tc && output_map_tc_ok(om)) ? launch_output_map_tc(om, s) : launch_output_map(om, s);
   }
   return cuda_status(e);
 }
@@ -399,25 +403,28 @@ int lla_decode_attn(const lla_decode_params* p, void* ws, size_t ws_bytes, lla_s
   a.part_y = reinterpret_cast<float*>(w + pl.o_py);
   a.win_ml = reinterpret_cast<float*>(w + pl.o_wml);
   a.win_y = reinterpret_cast<float*>(w + pl.o_wy);
-  a.S = pl.S; a.tps = pl.tps;
+  a.S = pl.S; a.tps = pl.tps; a.Sw = pl.Sw; a.cpt = pl.cpt;
+  int* err = reinterpret_cast<int*>(w + pl.o_err);
 
-  cudaError_t e = mark(p->timing_events, 0, s);
+  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = mark(p->timing_events, 0, s);
   if (e == cudaSuccess && a.n_lat > 0) e = launch_recon_split_simt(a, s);
   if (e == cudaSuccess) e = mark(p->timing_events, 1, s);
   if (e == cudaSuccess) {
     WindowArgs wa;
     wa.B = a.B; wa.rows = a.rows; wa.H = a.H; wa.d_h = a.d_h; wa.t0 = a.t0; wa.Wcap = a.Wcap;
-    wa.win_start = a.win_start; wa.n_win = a.n_win; wa.wk = a.wk; wa.wv = a.wv;
-    wa.dtype = a.win_dtype; wa.wins_b = a.wins_b;
+    wa.win_start = a.win_start; wa.n_win = a.n_win; wa.Sw = a.Sw; wa.cpt = a.cpt; wa.HG = pl.HG;
+    wa.wk = a.wk; wa.wv = a.wv; wa.dtype = a.win_dtype; wa.wins_b = a.wins_b;
     wa.q = a.q; wa.q_sb = a.qs_b; wa.q_srow = a.d_h; wa.qmul = a.qmul;
-    wa.win_ml = a.win_ml; wa.win_y = a.win_y;
+    wa.rotate = 0; wa.pos = a.N - 1; wa.base = 0.0;
+    wa.win_ml = a.win_ml; wa.win_y = a.win_y; wa.err = err;
     e = launch_window(wa, s);
   }
   if (e == cudaSuccess) {
     MergeArgs g;
-    g.B = a.B; g.rows = a.rows; g.H = a.H; g.d_h = a.d_h; g.S = a.S; g.Y = a.d_h;
+    g.B = a.B; g.rows = a.rows; g.H = a.H; g.d_h = a.d_h; g.S = a.S; g.Sw = a.Sw; g.Y = a.d_h;
     g.part_ml = a.part_ml; g.part_y = a.part_y; g.win_ml = a.win_ml; g.win_y = a.win_y;
-    g.Bm = nullptr; g.out = a.out; g.outs_b = a.outs_b; g.err = nullptr;
+    g.Bm = nullptr; g.out = a.out; g.outs_b = a.outs_b; g.err = err;
     e = launch_merge(g, s);
   }
   return cuda_status(e);

@@ -3,7 +3,10 @@
 // reconstruct-on-read, exact-window attention, and the split merge with the
 // B_t^T map back to head space.  Scores are kept in base-2 units: every query
 // is pre-multiplied by scale * log2(e) so the softmax uses exp2.
+#include <algorithm>
+
 #include "kernels.cuh"
+#include "tc_ptx.cuh"
 
 namespace lla {
 namespace {
@@ -110,11 +113,14 @@ __global__ void __launch_bounds__(256) absorb_split_simt(AbsorbArgs a) {
 }
 
 // --------------------------------------------------------------- window --
-// Exact attention over the window ring for one (row, sequence).  Each lane
-// holds 4 consecutive elements of the head dimension (one 8- or 16-byte load
-// per token), each warp takes every 4th group of WU tokens and issues all of a
-// group's K and V loads before using them, keeps its own online softmax, and
-// the four warps are combined at the end.  Emits (max, sum, y_w) in base-2 units.
+// Exact attention over the window ring (eq. 4, second term) as partial
+// softmax states.  One CTA per (token chunk, loop, sequence) covers every
+// head: warp w takes heads w, w+8, ..., so at any moment the CTA's warps read
+// neighbouring heads of the same tokens and each token's ring row [H][d_h] is
+// fetched as one contiguous block.  Each lane holds 4 consecutive elements of
+// the head dimension; a warp issues all K and V loads of WU tokens before
+// using them.  The query is rotated here (R_i in head space, when asked) and
+// scaled into base-2 units.  Emits (max, sum, y_w) per (chunk, sequence, row).
 template <bool BF16>
 struct WinTraits;
 template <>
@@ -142,43 +148,201 @@ struct WinTraits<false> {  // 4 fp32 per lane
   __device__ __forceinline__ static raw_t zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
 };
 
-template <bool BF16>
-__global__ void __launch_bounds__(128) window_attn(WindowArgs w) {
+// WU tokens per group: the full group for long windows, 4 for windows of a
+// few tokens (fewer registers, so more CTAs per SM).
+template <bool BF16, int WU, int MINB>
+__global__ void __launch_bounds__(256, MINB) window_part(WindowArgs w) {
   typedef WinTraits<BF16> Tr;
-  constexpr int WU = Tr::WU;
-  const int row = blockIdx.x, b = blockIdx.y;
-  const int tt = row / w.H, h = row % w.H, t = w.t0 + tt;
+  const int chunk = blockIdx.x, tt = blockIdx.y, b = blockIdx.z;
+  const int t = w.t0 + tt;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int d0 = 4 * lane;
   const bool dv = d0 < w.d_h;
+  const int j0 = chunk * w.cpt, j1 = min(w.n_win, j0 + w.cpt);
+  // the lane's two pairs (2 lane, 2 lane + 1) share their angles across heads
+  float c0 = 1.f, s0 = 0.f, c1 = 1.f, s1 = 0.f;
+  if (w.rotate && dv) {
+    rope_cs(2 * lane, w.d_h, w.d_h, w.base, (double)w.pos, &c0, &s0);
+    rope_cs(2 * lane + 1, w.d_h, w.d_h, w.base, (double)w.pos, &c1, &s1);
+  }
+  const int64_t seq = (int64_t)b * w.wins_b;
+  for (int h = warp; h < w.H; h += 8) {
+    const int row = tt * w.H + h;
+    float qv[4] = {0.f, 0.f, 0.f, 0.f}, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (dv) {
+      const float* q = w.q + (int64_t)b * w.q_sb + (int64_t)row * w.q_srow + d0;
+      const float x0 = q[0], y0 = q[1], x1 = q[2], y1 = q[3];
+      qv[0] = (x0 * c0 - y0 * s0) * w.qmul;
+      qv[1] = (x0 * s0 + y0 * c0) * w.qmul;
+      qv[2] = (x1 * c1 - y1 * s1) * w.qmul;
+      qv[3] = (x1 * s1 + y1 * c1) * w.qmul;
+    }
+    float m = -INFINITY, l = 0.f;
+    for (int g0 = j0; g0 < j1; g0 += WU) {
+      typename Tr::raw_t kr[WU], vr[WU];
+#pragma unroll
+      for (int u = 0; u < WU; ++u) {
+        const int idx = g0 + u;
+        if (dv && idx < j1) {
+          const int slot = (w.win_start + idx) % w.Wcap;
+          const int64_t base = seq + (((int64_t)t * w.Wcap + slot) * w.H + h) * w.d_h + d0;
+          kr[u] = Tr::load(w.wk, base);
+          vr[u] = Tr::load(w.wv, base);
+        } else {
+          kr[u] = Tr::zero();
+          vr[u] = Tr::zero();
+        }
+      }
+      float sc[WU];
+#pragma unroll
+      for (int u = 0; u < WU; ++u) {
+        float kk[4];
+        Tr::unpack(kr[u], kk);
+        float part = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) part = fmaf(qv[e], kk[e], part);
+        sc[u] = part;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int u = 0; u < WU; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
+      // one max per group of tokens, then a single rescale of the running state
+      float gm = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < WU; ++u)
+        if (g0 + u < j1) gm = fmaxf(gm, sc[u]);
+      const float mn = fmaxf(m, gm);
+      const float al = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+      l *= al;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] *= al;
+#pragma unroll
+      for (int u = 0; u < WU; ++u) {
+        if (g0 + u >= j1) break;
+        const float p = exp2f(sc[u] - mn);
+        float vv[4];
+        Tr::unpack(vr[u], vv);
+        l += p;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = fmaf(p, vv[e], acc[e]);
+      }
+      m = mn;
+    }
+    const int64_t o = ((int64_t)chunk * w.B + b) * w.rows + row;
+    if (lane == 0) {
+      w.win_ml[o * 2] = m;
+      w.win_ml[o * 2 + 1] = l;
+    }
+    if (dv) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) w.win_y[o * w.d_h + d0 + e] = acc[e];
+    }
+  }
+}
+
+// Large windows: the same partial states, with the ring rows staged in shared
+// memory by bulk copies (the TMA engine) instead of registers.  One CTA per
+// (token chunk, loop x group of 8 heads, sequence), one warp per head.  A
+// token's slice for the head group is contiguous in the ring (heads are
+// adjacent), so each token costs one bulk copy for K and one for V; stages of
+// WB_TS tokens go through a WB_NST-deep ring, so a CTA keeps up to WB_NST
+// stages in flight while its warps reduce the previous one from shared memory.
+constexpr int WB_HEADS = 8;
+constexpr int WB_NST = 3;
+constexpr long long WB_WAIT = 1ll << 32;
+
+template <bool BF16>
+struct WbTraits { static constexpr int TS = BF16 ? 8 : 4; };
+
+template <bool BF16>
+__global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(WindowArgs w) {
+  typedef WinTraits<BF16> Tr;
+  constexpr int TS = WbTraits<BF16>::TS;
+  constexpr int ES = BF16 ? 2 : 4;
+  extern __shared__ __align__(128) uint8_t wsm[];
+  const int chunk = blockIdx.x, tt = blockIdx.y / w.HG, hg = blockIdx.y % w.HG, b = blockIdx.z;
+  const int t = w.t0 + tt, h0 = hg * WB_HEADS;
+  const int nh = min(WB_HEADS, w.H - h0);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t hbytes = (uint32_t)w.d_h * ES;
+  const uint32_t tok_bytes = nh * hbytes;                         // one token's head-group slice
+  const uint32_t half = (uint32_t)TS * WB_HEADS * hbytes;          // K (or V) part of a stage
+  uint64_t* full = reinterpret_cast<uint64_t*>(wsm + WB_NST * 2 * half);
+  const int j0 = chunk * w.cpt, j1 = min(w.n_win, j0 + w.cpt);
+  const int nsub = (j1 - j0 + TS - 1) / TS;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < WB_NST; ++i) ptx::mbar_init(ptx::smem_u32(&full[i]), 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  const char* kbase = reinterpret_cast<const char*>(w.wk) + ((int64_t)b * w.wins_b) * ES;
+  const char* vbase = reinterpret_cast<const char*>(w.wv) + ((int64_t)b * w.wins_b) * ES;
+  auto issue = [&](int i) {        // sub-chunk i into stage i % WB_NST (thread 0)
+    const int st = i % WB_NST;
+    const int jj = j0 + i * TS, nt = min(TS, j1 - jj);
+    const uint32_t bar = ptx::smem_u32(&full[st]);
+    ptx::mbar_arrive_tx(bar, 2u * nt * tok_bytes);
+    const uint32_t dk = ptx::smem_u32(wsm + st * 2 * half), dv = dk + half;
+    for (int u = 0; u < nt; ++u) {
+      const int slot = (w.win_start + jj + u) % w.Wcap;
+      const int64_t off = (((int64_t)t * w.Wcap + slot) * w.H + h0) * (int64_t)hbytes;
+      ptx::bulk_load(dk + u * WB_HEADS * hbytes, kbase + off, tok_bytes, bar);
+      ptx::bulk_load(dv + u * WB_HEADS * hbytes, vbase + off, tok_bytes, bar);
+    }
+  };
+  if (threadIdx.x == 0)
+    for (int i = 0; i < WB_NST && i < nsub; ++i) issue(i);
+
+  const int d0 = 4 * lane;
+  const bool dv = warp < nh && d0 < w.d_h;
+  const int row = tt * w.H + h0 + warp;
+  float c0 = 1.f, s0 = 0.f, c1 = 1.f, s1 = 0.f;
+  if (w.rotate && dv) {
+    rope_cs(2 * lane, w.d_h, w.d_h, w.base, (double)w.pos, &c0, &s0);
+    rope_cs(2 * lane + 1, w.d_h, w.d_h, w.base, (double)w.pos, &c1, &s1);
+  }
   float qv[4] = {0.f, 0.f, 0.f, 0.f}, acc[4] = {0.f, 0.f, 0.f, 0.f};
   if (dv) {
     const float* q = w.q + (int64_t)b * w.q_sb + (int64_t)row * w.q_srow + d0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) qv[e] = q[e] * w.qmul;
+    const float x0 = q[0], y0 = q[1], x1 = q[2], y1 = q[3];
+    qv[0] = (x0 * c0 - y0 * s0) * w.qmul;
+    qv[1] = (x0 * s0 + y0 * c0) * w.qmul;
+    qv[2] = (x1 * c1 - y1 * s1) * w.qmul;
+    qv[3] = (x1 * s1 + y1 * c1) * w.qmul;
   }
   float m = -INFINITY, l = 0.f;
-  const int64_t seq = (int64_t)b * w.wins_b;
-  for (int g0 = warp * WU; g0 < w.n_win; g0 += 4 * WU) {
-    typename Tr::raw_t kr[WU], vr[WU];
-#pragma unroll
-    for (int u = 0; u < WU; ++u) {
-      const int idx = g0 + u;
-      if (dv && idx < w.n_win) {
-        const int slot = (w.win_start + idx) % w.Wcap;
-        const int64_t base = seq + (((int64_t)t * w.Wcap + slot) * w.H + h) * w.d_h + d0;
-        kr[u] = Tr::load(w.wk, base);
-        vr[u] = Tr::load(w.wv, base);
-      } else {
-        kr[u] = Tr::zero();
-        vr[u] = Tr::zero();
+  int failed_at = -1;
+  for (int i = 0; i < nsub; ++i) {
+    const int st = i % WB_NST;
+    const uint32_t bar = ptx::smem_u32(&full[st]);
+    const uint32_t par = (uint32_t)(i / WB_NST) & 1u;
+    bool ok = ptx::mbar_try_wait(bar, par);
+    if (!ok) {
+      const long long t0c = clock64();
+      while (!(ok = ptx::mbar_try_wait(bar, par)) && clock64() - t0c <= WB_WAIT) {
       }
     }
-    float sc[WU];
+    // every thread leaves together, so no warp is left at a barrier
+    if (__syncthreads_or(!ok)) {
+      failed_at = i;
+      break;
+    }
+    const int jj = j0 + i * TS, nt = min(TS, j1 - jj);
+    const uint8_t* ks = wsm + st * 2 * half + (size_t)warp * hbytes + (size_t)d0 * ES;
+    const uint8_t* vs = ks + half;
+    float sc[TS];
+    typename Tr::raw_t vr[TS];
 #pragma unroll
-    for (int u = 0; u < WU; ++u) {
+    for (int u = 0; u < TS; ++u) {
       float kk[4];
-      Tr::unpack(kr[u], kk);
+      typename Tr::raw_t kr = Tr::zero();
+      vr[u] = Tr::zero();
+      if (dv && u < nt) {
+        kr = *reinterpret_cast<const typename Tr::raw_t*>(ks + (size_t)u * WB_HEADS * hbytes);
+        vr[u] = *reinterpret_cast<const typename Tr::raw_t*>(vs + (size_t)u * WB_HEADS * hbytes);
+      }
+      Tr::unpack(kr, kk);
       float part = 0.f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) part = fmaf(qv[e], kk[e], part);
@@ -187,20 +351,19 @@ __global__ void __launch_bounds__(128) window_attn(WindowArgs w) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-      for (int u = 0; u < WU; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
-    // one max per group of tokens, then a single rescale of the running state
+      for (int u = 0; u < TS; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
     float gm = -INFINITY;
 #pragma unroll
-    for (int u = 0; u < WU; ++u)
-      if (g0 + u < w.n_win) gm = fmaxf(gm, sc[u]);
+    for (int u = 0; u < TS; ++u)
+      if (u < nt) gm = fmaxf(gm, sc[u]);
     const float mn = fmaxf(m, gm);
     const float al = (m == -INFINITY) ? 0.f : exp2f(m - mn);
     l *= al;
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[e] *= al;
 #pragma unroll
-    for (int u = 0; u < WU; ++u) {
-      if (g0 + u >= w.n_win) break;
+    for (int u = 0; u < TS; ++u) {
+      if (u >= nt) break;
       const float p = exp2f(sc[u] - mn);
       float vv[4];
       Tr::unpack(vr[u], vv);
@@ -209,28 +372,32 @@ __global__ void __launch_bounds__(128) window_attn(WindowArgs w) {
       for (int e = 0; e < 4; ++e) acc[e] = fmaf(p, vv[e], acc[e]);
     }
     m = mn;
+    __syncthreads();   // every warp is done with this stage
+    if (threadIdx.x == 0 && i + WB_NST < nsub) issue(i + WB_NST);
   }
-  __shared__ float sm_m[4], sm_l[4], sm_y[4][128];
-  if (lane == 0) { sm_m[warp] = m; sm_l[warp] = l; }
-  if (dv) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) sm_y[warp][d0 + e] = acc[e];
+  if (failed_at >= 0) {
+    if (threadIdx.x == 0) {
+      if (w.err) atomicExch(w.err, ERR_WINDOW_TIMEOUT);
+      // leave no copy in flight: wait (bounded) for the stages still owed
+      for (int i = failed_at; i < nsub && i < failed_at + WB_NST; ++i) {
+        const uint32_t bar = ptx::smem_u32(&full[i % WB_NST]);
+        const long long t0c = clock64();
+        while (!ptx::mbar_try_wait(bar, (uint32_t)(i / WB_NST) & 1u) && clock64() - t0c < WB_WAIT) {
+        }
+      }
+    }
+    return;
   }
-  __syncthreads();
-  const float M = fmaxf(fmaxf(sm_m[0], sm_m[1]), fmaxf(sm_m[2], sm_m[3]));
-  float wgt[4], L = 0.f;
+  if (warp < nh) {
+    const int64_t o = ((int64_t)chunk * w.B + b) * w.rows + row;
+    if (lane == 0) {
+      w.win_ml[o * 2] = m;
+      w.win_ml[o * 2 + 1] = l;
+    }
+    if (dv) {
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    wgt[u] = (sm_m[u] == -INFINITY) ? 0.f : exp2f(sm_m[u] - M);
-    L += wgt[u] * sm_l[u];
-  }
-  const int64_t o = (int64_t)b * w.rows + row;
-  if (threadIdx.x == 0) { w.win_ml[o * 2] = M; w.win_ml[o * 2 + 1] = L; }
-  for (int d = threadIdx.x; d < w.d_h; d += 128) {
-    float y = 0.f;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) y += wgt[u] * sm_y[u][d];
-    w.win_y[o * w.d_h + d] = y;
+      for (int e = 0; e < 4; ++e) w.win_y[o * w.d_h + d0 + e] = acc[e];
+    }
   }
 }
 
@@ -242,22 +409,29 @@ __global__ void __launch_bounds__(128) window_attn(WindowArgs w) {
 __global__ void __launch_bounds__(128) merge_plain(MergeArgs g) {
   const int row = blockIdx.x, b = blockIdx.y;
   const int64_t br = (int64_t)b * g.rows + row;
-  float M = g.win_ml[br * 2];
-  for (int s = 0; s < g.S; ++s) M = fmaxf(M, g.part_ml[((int64_t)s * g.B * g.rows + br) * 2]);
-  const float ww = exp2f(g.win_ml[br * 2] - M);
-  float L = ww * g.win_ml[br * 2 + 1];
+  const int64_t bstride = (int64_t)g.B * g.rows;   // between partials of consecutive splits / chunks
+  float M = -INFINITY;
+  for (int c = 0; c < g.Sw; ++c) M = fmaxf(M, g.win_ml[(c * bstride + br) * 2]);
+  for (int s = 0; s < g.S; ++s) M = fmaxf(M, g.part_ml[(s * bstride + br) * 2]);
+  float L = 0.f;
+  for (int c = 0; c < g.Sw; ++c) {
+    const float mc = g.win_ml[(c * bstride + br) * 2];
+    if (mc != -INFINITY) L += exp2f(mc - M) * g.win_ml[(c * bstride + br) * 2 + 1];
+  }
   for (int s = 0; s < g.S; ++s) {
-    const float ms = g.part_ml[((int64_t)s * g.B * g.rows + br) * 2];
-    if (ms == -INFINITY) continue;
-    L += exp2f(ms - M) * g.part_ml[((int64_t)s * g.B * g.rows + br) * 2 + 1];
+    const float ms = g.part_ml[(s * bstride + br) * 2];
+    if (ms != -INFINITY) L += exp2f(ms - M) * g.part_ml[(s * bstride + br) * 2 + 1];
   }
   const float li = 1.f / L;
   for (int d = threadIdx.x; d < g.d_h; d += blockDim.x) {
-    float y = ww * g.win_y[br * g.d_h + d];
+    float y = 0.f;
+    for (int c = 0; c < g.Sw; ++c) {
+      const float mc = g.win_ml[(c * bstride + br) * 2];
+      if (mc != -INFINITY) y = fmaf(exp2f(mc - M), g.win_y[(c * bstride + br) * g.d_h + d], y);
+    }
     for (int s = 0; s < g.S; ++s) {
-      const float ms = g.part_ml[((int64_t)s * g.B * g.rows + br) * 2];
-      if (ms == -INFINITY) continue;
-      y = fmaf(exp2f(ms - M), g.part_y[((int64_t)s * g.B * g.rows + br) * g.d_h + d], y);
+      const float ms = g.part_ml[(s * bstride + br) * 2];
+      if (ms != -INFINITY) y = fmaf(exp2f(ms - M), g.part_y[(s * bstride + br) * g.d_h + d], y);
     }
     g.out[(int64_t)b * g.outs_b + (int64_t)row * g.d_h + d] = (g.err && *g.err) ? NAN : y * li;
   }
@@ -397,12 +571,54 @@ cudaError_t launch_absorb_split_simt(const AbsorbArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+bool window_bulk_ok(int dtype, int d_h) {
+  const int es = dtype == LLA_BF16 ? 2 : 4;
+  return (d_h * es) % 16 == 0;
+}
+
+int window_chunks(int B, int nt, int H, int n_win, int dtype, int d_h, int num_sms, int* cpt, int* HG) {
+  // about four CTAs per SM; chunks of a multiple of 8 tokens.  Windows of at
+  // least 16 tokens use the bulk-copy kernel (groups of 8 heads per CTA).
+  const bool bulk = n_win >= 16 && window_bulk_ok(dtype, d_h);
+  *HG = bulk ? (H + WB_HEADS - 1) / WB_HEADS : 0;
+  const long ctas = (long)B * nt * (bulk ? *HG : 1);
+  long S = ctas > 0 ? (4L * num_sms + ctas - 1) / ctas : 1;
+  S = std::max(1L, std::min(S, std::min((long)kMaxWindowChunks, (long)((n_win + 7) / 8))));
+  int c = (int)((n_win + S - 1) / S);
+  c = (c + 7) / 8 * 8;
+  *cpt = c;
+  return (n_win + c - 1) / c;
+}
+
 cudaError_t launch_window(const WindowArgs& w, cudaStream_t st) {
-  dim3 grid(w.rows, w.B);
-  if (w.dtype == LLA_BF16)
-    window_attn<true><<<grid, 128, 0, st>>>(w);
-  else
-    window_attn<false><<<grid, 128, 0, st>>>(w);
+  if (w.n_win <= 0 || w.B == 0) return cudaSuccess;
+  const int nt = w.rows / w.H;
+  if (w.HG > 0) {
+    const int es = w.dtype == LLA_BF16 ? 2 : 4;
+    const int ts = w.dtype == LLA_BF16 ? WbTraits<true>::TS : WbTraits<false>::TS;
+    const size_t smem = (size_t)WB_NST * 2 * ts * WB_HEADS * w.d_h * es + 8 * WB_NST + 16;
+    dim3 grid(w.Sw, nt * w.HG, w.B);
+    cudaError_t e;
+    if (w.dtype == LLA_BF16) {
+      e = cudaFuncSetAttribute(window_bulk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      window_bulk<true><<<grid, 32 * WB_HEADS, smem, st>>>(w);
+    } else {
+      e = cudaFuncSetAttribute(window_bulk<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      window_bulk<false><<<grid, 32 * WB_HEADS, smem, st>>>(w);
+    }
+    return cudaGetLastError();
+  }
+  dim3 grid(w.Sw, nt, w.B);
+  const bool small = w.cpt <= 8;
+  if (w.dtype == LLA_BF16) {
+    if (small) window_part<true, 4, 4><<<grid, 256, 0, st>>>(w);
+    else window_part<true, WinTraits<true>::WU, 1><<<grid, 256, 0, st>>>(w);
+  } else {
+    if (small) window_part<false, 4, 4><<<grid, 256, 0, st>>>(w);
+    else window_part<false, WinTraits<false>::WU, 1><<<grid, 256, 0, st>>>(w);
+  }
   return cudaGetLastError();
 }
 

@@ -1,0 +1,608 @@
+// The dense contractions around the latent read, on the tensor cores
+// (tcgen05, kind::tf32, accumulators in TMEM):
+//
+//   query map  (HLA eq. 3):  q~[b][row] = s*log2e * R~_i A_row^T q[b][row]        (bf16 out)
+//   output map (eq. 4):      o[b][row]  = (B_row^T sum_s w_s y~_s + sum_c w_c y_c) / l
+//   writer     (eq. 2, LLA encoders): fp32 partial sums of each writer slice
+//
+// Every one is a set of GEMMs D = A_g * X_g^T with a per-group codec matrix
+// A_g (the M side, 128 rows per tile: the latent / head-dimension columns of
+// the codec) and the activations X_g (the N side: sequences or tokens, BN per
+// tile), so a decode batch of 32 and one of 768 both map onto the MMA's N.
+//
+// Operands are fp32 in HBM.  Four producer warps copy each 32-deep k-chunk
+// into 128-byte-swizzled shared memory with cp.async (zero-filling anything
+// out of range), then round their own pieces in place to tf32 (round to
+// nearest, ties away) and, for PREC = 3, store the remainder x - tf32(x) as a
+// second tf32 tile.  PREC = 3 issues hi*hi + hi*lo + lo*hi ("3xTF32"), whose
+// error is that of fp32 arithmetic; PREC = 1 issues hi*hi (relative error
+// about 2^-11 per product).  One thread of a fifth warp issues the MMAs into
+// TMEM and releases stages with tcgen05.commit; the producer warps then read
+// the accumulators back (tcgen05.ld) for the epilogue.  Waits are bounded:
+// on a timeout the CTA records an error code (outputs become NaN downstream).
+#include <cuda.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "tc_ptx.cuh"
+#include "writer_slice.cuh"
+
+namespace lla {
+namespace {
+
+using namespace ptx;
+
+constexpr int GM = 128;                 // M of every MMA (codec rows per tile)
+constexpr int KCH = 32;                 // k per chunk: 32 fp32 = one 128-byte row
+constexpr int A_BYTES = GM * KCH * 4;   // 16 KB
+constexpr int NPROD = 256;              // producer + epilogue threads (warps 0-7)
+constexpr int NTHR = NPROD + 32;        // + warp 8: TMEM allocation, MMA issue
+constexpr int MMA_WARP = NPROD / 32;
+constexpr int SMEM_MAX = 232448;
+constexpr long long WAIT_CYCLES = 1ll << 32;
+
+enum : int { KIND_QMAP = 0, KIND_OMAP = 1, KIND_WRITER = 2 };
+enum : int { ERR_GEMM_EMPTY = 11, ERR_GEMM_FULL = 12, ERR_GEMM_DONE = 13 };
+
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn_major) {
+  return (1u << 4)                          // D format: fp32
+         | (2u << 7)                        // A format: tf32
+         | (2u << 10)                       // B format: tf32
+         | ((a_mn_major ? 1u : 0u) << 15)   // B is always K-major
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 16-byte global -> shared copy; src_bytes = 0 fills the 16 bytes with zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ float4 lds4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(a)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err,
+                                         int code, bool honour_abort = true) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (honour_abort && *abort_flag) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > WAIT_CYCLES) {
+      *abort_flag = 1;
+      if (err) atomicExch(err, code);
+      return false;
+    }
+  }
+}
+
+// Offset of 16-byte piece c (k = 4c .. 4c+3) of row r in a K-major SW128 tile.
+__device__ __forceinline__ uint32_t kmajor_off(int r, int c) {
+  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+// Offset of the 16-byte piece holding rows 4c32 .. 4c32+3 at depth kk in an
+// MN-major tf32 tile of 128 rows x 32 k, in the 128-byte swizzle with 32-byte
+// granules (the one layout the tensor cores accept for MN-major tf32): atoms
+// of 4 k-rows x 128 bytes (512 B) whose 32-byte granule index is XORed with
+// the k-row (mod 4); k-groups 512 B apart, 32-row MN atoms 4 KB apart.
+__device__ __forceinline__ uint32_t mnmajor_off(int kk, int c32) {
+  const int c = c32 & 7;
+  return (uint32_t)((c32 >> 3) * 4096 + (kk >> 2) * 512 + (kk & 3) * 128 + (((c >> 1) ^ (kk & 3)) << 5) +
+                    ((c & 1) << 4));
+}
+
+__device__ __forceinline__ int64_t qbf_index(int b, int row, int k, int r_k) {
+  const int kb = k >> 6, e = k & 63;
+  return (int64_t)b * (r_k >> 6) * 4096 + kb * 4096 + row * 64 + ((((e >> 3) ^ (row & 7)) << 3) | (e & 7));
+}
+
+// Per-tile geometry, resolved from blockIdx for each kind.
+struct Tile {
+  int g;            // group: map row, or writer slice
+  int split;        // writer k-split
+  int m0, n0;       // tile origin (codec rows, activation rows)
+  int Mv, Nv, K;    // valid extents of the group and its depth
+  int kc0, kc1;     // chunk range
+};
+
+template <int KIND, int BN, int PREC, int DEPTH>
+__global__ void __launch_bounds__(NTHR, 1) tc_gemm(const TcGemmArgs a) {
+  constexpr int NST = DEPTH + 1;
+  constexpr bool A_MN = KIND != KIND_WRITER;   // codec operand MN-major (maps) or K-major (writer)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- tile ------------------------------------------------------------
+  Tile t;
+  const int mt = (int)blockIdx.x / a.ntiles, nti = (int)blockIdx.x % a.ntiles;
+  t.m0 = mt * GM;
+  t.n0 = nti * BN;
+  Slice sl;
+  if (KIND == KIND_WRITER) {
+    t.g = (int)blockIdx.y / a.S;
+    t.split = (int)blockIdx.y % a.S;
+    sl = slice_of(a.w, t.g);
+    t.Mv = sl.N;
+    t.Nv = a.w.M;
+    t.K = sl.K_outer * sl.d_in;
+    const int nk = (t.K + KCH - 1) / KCH;
+    t.kc0 = (int)((int64_t)nk * t.split / a.S);
+    t.kc1 = (int)((int64_t)nk * (t.split + 1) / a.S);
+    if (t.m0 >= t.Mv) return;   // this slice is narrower than the widest one
+  } else {
+    t.g = blockIdx.y;
+    t.split = 0;
+    t.Mv = a.Mtot;
+    t.Nv = a.B;
+    t.K = a.K;
+    t.kc0 = 0;
+    t.kc1 = (t.K + KCH - 1) / KCH;
+    if (KIND == KIND_QMAP && t.g >= a.rows) {
+      // rows of the bf16 query operand past the last query row are zero
+      for (int idx = tid; idx < GM * BN; idx += NTHR) {
+        const int m = t.m0 + (idx % GM), n = t.n0 + idx / GM;
+        if (m < t.Mv && n < t.Nv) a.qbf[qbf_index(n, t.g, m, a.Mtot)] = __float2bfloat16_rn(0.f);
+      }
+      return;
+    }
+  }
+  const int nb = KIND == KIND_OMAP ? a.NB : 1;
+  const int nchunks = t.kc1 - t.kc0;
+
+  // ---- shared memory ------------------------------------------------------
+  const uint32_t b_tile = (uint32_t)BN * 128;
+  const uint32_t a_part = (uint32_t)A_BYTES * (PREC == 3 ? 2 : 1);
+  const uint32_t stage_bytes = a_part + b_tile * nb * (PREC == 3 ? 2 : 1);
+  const uint32_t sbase = smem_u32(base);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + NST * stage_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + NST;
+  uint64_t* done = bars + 2 * NST;
+  uint8_t* misc = reinterpret_cast<uint8_t*>(bars + 2 * NST + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  float* wts = reinterpret_cast<float*>(misc + 16);   // output map: [BN][NB + Sw + 1]
+
+  if (tid == 0) {
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(smem_u32(&full[i]), NPROD);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    mbar_init(smem_u32(done), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  uint32_t ncols = 32;
+  while (ncols < (uint32_t)(nb * BN)) ncols <<= 1;
+  if (warp == MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < NPROD / 32) {
+    // ---- producers ---------------------------------------------------------
+    // A thread's pieces of a chunk share one k (K-major: column c of every
+    // row r0 + 32u) or one codec row (MN-major: rows m .. m+3 at depths
+    // kk0 + 8u), so their addresses are a fixed base plus u times a stride,
+    // and moving to the next chunk only advances one running position.
+    constexpr int PA = A_BYTES / 16 / NPROD;   // A pieces per thread
+    constexpr int PB = BN * 8 / NPROD;         // pieces per thread of each B operand
+    const int c8 = tid & 7, r0 = tid >> 3;                 // K-major piece: column, first row
+    const int c32 = tid & 31, kk0 = tid >> 5;              // MN-major piece: row group, first depth
+    const uint32_t a_off0 = A_MN ? mnmajor_off(kk0, c32) : kmajor_off(r0, c8);
+    constexpr uint32_t A_OFF_U = A_MN ? 1024u * (NPROD / 256) : 4096u * (NPROD / 256);
+    const uint32_t b_off0 = kmajor_off(r0, c8);
+    constexpr uint32_t B_OFF_U = 4096u * (NPROD / 256);
+    // rows of the operands for this thread
+    const int a_row = A_MN ? t.m0 + 4 * c32 : t.m0 + r0;   // + 32u for K-major
+    // running k position of this thread's K-major pieces (the writer's
+    // (outer block, feature) decomposition is tracked incrementally)
+    int kpos = t.kc0 * KCH + 4 * c8;
+    int ob = 0, od = 0, ot = 0, oh = 0;
+    if (KIND == KIND_WRITER) {
+      ob = kpos / sl.d_in;
+      od = kpos % sl.d_in;
+      ot = ob / sl.o_h;
+      oh = ob % sl.o_h;
+    }
+    int64_t xrow[PB > 0 ? PB : 1];
+#pragma unroll
+    for (int u = 0; u < PB; ++u) {
+      const int n = t.n0 + r0 + 32 * (NPROD / 256) * u;
+      xrow[u] = 0;
+      if (n < t.Nv) {
+        if (KIND == KIND_WRITER) xrow[u] = writer_xrow(a.w, n);
+        else if (KIND == KIND_QMAP) xrow[u] = (int64_t)n * a.xs_b + (int64_t)t.g * t.K;
+        else xrow[u] = ((int64_t)n * a.rows + t.g) * t.K;
+      }
+    }
+    const int64_t b_jb_stride = (int64_t)a.B * a.rows * t.K;   // output map: between split partials
+    bool aborted = false;
+    auto issue = [&](int i) {
+      if (!aborted) {
+        const int st = i % NST;
+        if (i >= NST &&
+            !wait_bar(smem_u32(&empty[st]), ((i / NST) - 1) & 1, abort_flag, a.err, ERR_GEMM_EMPTY))
+          aborted = true;
+        if (!aborted) {
+          const uint32_t s0 = sbase + st * stage_bytes;
+          const int k0 = (t.kc0 + i) * KCH;
+          if (A_MN) {
+            // codec [g][k][m]: rows m .. m+3 at depth k0 + kk0 + 8u
+            const bool mok = a_row < t.Mv;
+            const float* src0 = a.Aw + ((int64_t)t.g * t.K + k0 + kk0) * t.Mv + a_row;
+#pragma unroll
+            for (int u = 0; u < PA; ++u) {
+              const int k = k0 + kk0 + 8 * (NPROD / 256) * u;
+              const bool ok = mok && k < t.K;
+              cp_async16(s0 + a_off0 + u * A_OFF_U, ok ? src0 + (int64_t)8 * (NPROD / 256) * u * t.Mv : a.Aw,
+                         ok ? 16u : 0u);
+            }
+          } else {
+            // writer codec E(n, k) at E + ob * e_o + n * e_n + od
+            const bool kok = kpos < t.K;
+            const float* src0 = sl.E + (int64_t)ob * sl.e_o + (int64_t)a_row * sl.e_n + od;
+#pragma unroll
+            for (int u = 0; u < PA; ++u) {
+              const bool ok = kok && a_row + 32 * (NPROD / 256) * u < t.Mv;
+              cp_async16(s0 + a_off0 + u * A_OFF_U, ok ? src0 + (int64_t)32 * (NPROD / 256) * u * sl.e_n : sl.E,
+                         ok ? 16u : 0u);
+            }
+          }
+          const bool kok = kpos < t.K;
+          int64_t koff;
+          if (KIND == KIND_WRITER) koff = (int64_t)ot * sl.x_o_t + (int64_t)oh * sl.x_o_h + od;
+          else koff = kpos;
+          const float* xbase = KIND == KIND_WRITER ? sl.X : a.X;
+          for (int jb = 0; jb < nb; ++jb) {
+            const uint32_t bt = s0 + a_part + jb * b_tile;
+#pragma unroll
+            for (int u = 0; u < PB; ++u) {
+              const bool ok = kok && t.n0 + r0 + 32 * (NPROD / 256) * u < t.Nv;
+              cp_async16(bt + b_off0 + u * B_OFF_U, ok ? xbase + jb * b_jb_stride + xrow[u] + koff : xbase,
+                         ok ? 16u : 0u);
+            }
+          }
+        }
+      }
+      cp_async_commit();
+      // advance this thread's k position by one chunk
+      kpos += KCH;
+      if (KIND == KIND_WRITER) {
+        od += KCH;
+        while (od >= sl.d_in) {
+          od -= sl.d_in;
+          ++ob;
+          if (++oh == sl.o_h) {
+            oh = 0;
+            ++ot;
+          }
+        }
+      }
+    };
+    auto convert = [&](uint32_t addr, uint32_t lo_addr) {
+      const float4 v = lds4(addr);
+      const uint32_t hx = to_tf32(v.x), hy = to_tf32(v.y), hz = to_tf32(v.z), hw = to_tf32(v.w);
+      sts4(addr, hx, hy, hz, hw);
+      if (PREC == 3)
+        sts4(lo_addr, to_tf32(v.x - __uint_as_float(hx)), to_tf32(v.y - __uint_as_float(hy)),
+             to_tf32(v.z - __uint_as_float(hz)), to_tf32(v.w - __uint_as_float(hw)));
+    };
+#pragma unroll 1
+    for (int i = 0; i < DEPTH; ++i) {
+      if (i < nchunks) issue(i);
+      else cp_async_commit();
+    }
+#pragma unroll 1
+    for (int i = 0; i < nchunks; ++i) {
+      cp_async_wait<DEPTH - 1>();
+      if (aborted || *abort_flag) {
+        aborted = true;
+        break;
+      }
+      const int st = i % NST;
+      const uint32_t s0 = sbase + st * stage_bytes;
+#pragma unroll
+      for (int u = 0; u < PA; ++u) convert(s0 + a_off0 + u * A_OFF_U, s0 + A_BYTES + a_off0 + u * A_OFF_U);
+      for (int jb = 0; jb < nb; ++jb) {
+        const uint32_t bt = s0 + a_part + jb * b_tile;
+#pragma unroll
+        for (int u = 0; u < PB; ++u) convert(bt + b_off0 + u * B_OFF_U, bt + nb * b_tile + b_off0 + u * B_OFF_U);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&full[st]));
+      if (i + DEPTH < nchunks) issue(i + DEPTH);
+      else cp_async_commit();
+    }
+    cp_async_wait<0>();
+
+    // ---- output-map weights (while the last MMAs run) ---------------------
+    if (KIND == KIND_OMAP) {
+      const int ld = a.NB + a.Sw + 1;
+      const int64_t bstride = (int64_t)a.B * a.rows;
+      for (int bb = tid; bb < BN; bb += NPROD) {
+        const int b = t.n0 + bb;
+        float* w = wts + bb * ld;
+        if (b >= a.B) {
+          for (int j = 0; j < ld; ++j) w[j] = 0.f;
+          continue;
+        }
+        const int64_t br = (int64_t)b * a.rows + t.g;
+        float M = -INFINITY, L = 0.f;
+        for (int s = 0; s < a.NB; ++s) M = fmaxf(M, a.part_ml[(s * bstride + br) * 2]);
+        for (int c = 0; c < a.Sw; ++c) M = fmaxf(M, a.win_ml[(c * bstride + br) * 2]);
+        for (int s = 0; s < a.NB; ++s) {
+          const float ms = a.part_ml[(s * bstride + br) * 2];
+          const float ws = ms == -INFINITY ? 0.f : exp2f(ms - M);
+          w[s] = ws;
+          L += ws * a.part_ml[(s * bstride + br) * 2 + 1];
+        }
+        for (int c = 0; c < a.Sw; ++c) {
+          const float mc = a.win_ml[(c * bstride + br) * 2];
+          const float wc = mc == -INFINITY ? 0.f : exp2f(mc - M);
+          w[a.NB + c] = wc;
+          L += wc * a.win_ml[(c * bstride + br) * 2 + 1];
+        }
+        w[a.NB + a.Sw] = 1.f / L;
+      }
+      named_sync(1, NPROD);
+    }
+
+    // ---- epilogue ------------------------------------------------------------
+    const bool ok = wait_bar(smem_u32(done), 0, abort_flag, a.err, ERR_GEMM_DONE, false) && !*abort_flag;
+    tc_fence_after();
+    // warps w and w + 4 share TMEM lanes 32 (w & 3) .. +31 and split the columns
+    const int quarter = warp & 3, half = warp >> 2;
+    const int m = t.m0 + 32 * quarter + lane;   // this thread's TMEM lane = codec row
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
+    const bool have = nchunks > 0;
+    float cq = 1.f, sq = 0.f;
+    if (KIND == KIND_QMAP && a.rotate && m < t.Mv) rope_cs(m >> 1, a.Mtot, a.d_h, a.base, (double)a.pos, &cq, &sq);
+    const bool bad = !ok || (KIND == KIND_OMAP && a.err && *a.err);
+#pragma unroll 1
+    for (int c = half * (BN / 32); c < (half + 1) * (BN / 32); ++c) {
+      float v[16];
+      if (KIND == KIND_OMAP) {
+        const int ld = a.NB + a.Sw + 1;
+        float acc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+        for (int jb = 0; jb < nb; ++jb) {
+          if (have) {
+            tmem_ld16(lane_addr + jb * BN + 16 * c, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] = fmaf(wts[(16 * c + i) * ld + jb], v[i], acc[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = acc[i];
+      } else if (have) {
+        tmem_ld16(lane_addr + 16 * c, v);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      }
+      if (KIND == KIND_QMAP) {
+        // rotate pair (m even, m + 1) -- neighbouring lanes -- then scale to bf16
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float other = __shfl_xor_sync(0xffffffffu, v[i], 1);
+          const float x = (m & 1) ? other : v[i], y = (m & 1) ? v[i] : other;
+          const float r = (m & 1) ? (x * sq + y * cq) : (x * cq - y * sq);
+          const int n = t.n0 + 16 * c + i;
+          if (m < t.Mv && n < t.Nv)
+            a.qbf[qbf_index(n, t.g, m, a.Mtot)] = __float2bfloat16_rn(bad ? NAN : r * a.qmul);
+        }
+      } else if (KIND == KIND_OMAP) {
+        const int ld = a.NB + a.Sw + 1;
+        const int64_t bstride = (int64_t)a.B * a.rows;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int bb = 16 * c + i, n = t.n0 + bb;
+          if (m >= t.Mv || n >= t.Nv) continue;
+          float y = v[i];
+          const int64_t br = (int64_t)n * a.rows + t.g;
+          for (int cw = 0; cw < a.Sw; ++cw)
+            y = fmaf(wts[bb * ld + a.NB + cw], a.win_y[(cw * bstride + br) * a.Mtot + m], y);
+          a.out[(int64_t)n * a.outs_b + (int64_t)t.g * a.Mtot + m] = bad ? NAN : y * wts[bb * ld + a.NB + a.Sw];
+        }
+      } else {
+        float* P = a.w.part + ((int64_t)(t.g * a.S + t.split) * a.w.M) * a.w.Nmax;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int n = t.n0 + 16 * c + i;
+          if (m < t.Mv && n < t.Nv) P[(int64_t)n * a.w.Nmax + m] = bad ? NAN : v[i];
+        }
+      }
+    }
+    tc_fence_before();
+  } else if (lane == 0) {
+    // ---- MMA issue -------------------------------------------------------------
+    const bool a_mn = KIND != KIND_WRITER;
+    constexpr uint32_t idesc = idesc_tf32(GM, BN, KIND != KIND_WRITER);
+    const uint32_t a_step = a_mn ? (1024u >> 4) : (32u >> 4);   // 8 k: two 4-row groups, or 32 bytes
+    const uint32_t b_step = 32u >> 4;
+#pragma unroll 1
+    for (int i = 0; i < nchunks; ++i) {
+      const int st = i % NST;
+      if (!wait_bar(smem_u32(&full[st]), (i / NST) & 1, abort_flag, a.err, ERR_GEMM_FULL)) break;
+      tc_fence_after();
+      const uint32_t s0 = sbase + st * stage_bytes;
+      const uint64_t ahi = a_mn ? smem_desc_sw128_32b(s0, 4096, 512) : smem_desc_sw128(s0, 16, 1024);
+      const uint64_t alo = a_mn ? smem_desc_sw128_32b(s0 + A_BYTES, 4096, 512) : smem_desc_sw128(s0 + A_BYTES, 16, 1024);
+      for (int jb = 0; jb < nb; ++jb) {
+        const uint32_t bt = s0 + a_part + jb * b_tile;
+        const uint64_t bhi = smem_desc_sw128(bt, 16, 1024);
+        const uint64_t blo = smem_desc_sw128(bt + nb * b_tile, 16, 1024);
+        const uint32_t d = tmem + jb * BN;
+#pragma unroll
+        for (int j = 0; j < KCH / 8; ++j) {
+          if (PREC == 3) {
+            mma_tf32(d, alo + j * a_step, bhi + j * b_step, idesc, (i > 0 || j > 0) ? 1u : 0u);
+            mma_tf32(d, ahi + j * a_step, blo + j * b_step, idesc, 1u);
+            mma_tf32(d, ahi + j * a_step, bhi + j * b_step, idesc, 1u);
+          } else {
+            mma_tf32(d, ahi + j * a_step, bhi + j * b_step, idesc, (i > 0 || j > 0) ? 1u : 0u);
+          }
+        }
+      }
+      mma_commit(smem_u32(&empty[st]));
+    }
+    mma_commit(smem_u32(done));
+  }
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, ncols);
+  }
+}
+
+template <int KIND, int BN, int PREC, int DEPTH>
+cudaError_t launch_one(const TcGemmArgs& a, int grid_y, int nb, cudaStream_t st) {
+  const int stage = (A_BYTES * (PREC == 3 ? 2 : 1)) + BN * 128 * nb * (PREC == 3 ? 2 : 1);
+  const int wts = KIND == KIND_OMAP ? BN * (nb + a.Sw + 1) * 4 : 0;
+  size_t smem = 1024 + (size_t)(DEPTH + 1) * stage + 8 * (2 * (DEPTH + 1) + 1) + 16 + wts;
+  // keep the CTAs an SM can hold (228 KB of shared memory, 1 KB reserved per
+  // CTA) within its 512 TMEM columns, so that no allocation ever waits
+  int ncols = 32;
+  while (ncols < nb * BN) ncols <<= 1;
+  const int max_ctas = 512 / ncols;
+  const size_t floor_smem = (size_t)233472 / (max_ctas + 1) - 1024 + 16;
+  if (smem < floor_smem) smem = floor_smem;
+  if (smem > (size_t)SMEM_MAX) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(tc_gemm<KIND, BN, PREC, DEPTH>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.mtiles * a.ntiles, grid_y);
+  tc_gemm<KIND, BN, PREC, DEPTH><<<grid, NTHR, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+int pick_bn(int n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : 256; }
+
+template <int KIND, int PREC, int DEPTH>
+cudaError_t launch_bn(TcGemmArgs a, int Nv, int grid_y, int nb, int bn_cap, cudaStream_t st) {
+  const int bn = std::min(pick_bn(Nv), bn_cap);
+  a.ntiles = (Nv + bn - 1) / bn;
+  switch (bn) {
+    case 32: return launch_one<KIND, 32, PREC, DEPTH>(a, grid_y, nb, st);
+    case 64: return launch_one<KIND, 64, PREC, DEPTH>(a, grid_y, nb, st);
+    case 128: return launch_one<KIND, 128, PREC, DEPTH>(a, grid_y, nb, st);
+    default: return launch_one<KIND, 256, PREC, DEPTH>(a, grid_y, nb, st);
+  }
+}
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+// ------------------------------------------------------------- query map --
+bool query_map_tc_ok(const MapArgs& g) {
+  return g.use_tc && al16(g.W) && al16(g.X) && g.xs_b % 4 == 0 && g.xs_row == g.K && g.K % 4 == 0 &&
+         g.N % 64 == 0 && g.N <= 1024;
+}
+
+cudaError_t launch_query_map_tc(const MapArgs& g, int* err, cudaStream_t st) {
+  TcGemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = g.B; a.rows = g.rows; a.Mtot = g.N; a.K = g.K; a.mtiles = (g.N + GM - 1) / GM;
+  a.Aw = g.W; a.X = g.X; a.xs_b = g.xs_b;
+  a.rotate = g.rotate; a.pos = g.pos; a.d_h = g.d_h; a.base = g.base; a.qmul = g.qmul; a.qbf = g.qbf;
+  a.err = err; a.NB = 1; a.S = 1;
+  return launch_bn<KIND_QMAP, 1, 3>(a, g.B, 64, 1, 256, st);
+}
+
+// ------------------------------------------------------------ output map --
+bool output_map_tc_ok(const MapArgs& g) {
+  // one TMEM accumulator per latent split: at most 8 splits of 32 columns
+  return al16(g.W) && g.N % 4 == 0 && g.N <= GM && g.K % 4 == 0 && g.S >= 1 && g.S <= 8 &&
+         g.Sw <= kMaxWindowChunks;
+}
+
+cudaError_t launch_output_map_tc(const MapArgs& g, cudaStream_t st) {
+  TcGemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = g.B; a.rows = g.rows; a.Mtot = g.N; a.K = g.K; a.mtiles = 1;
+  a.Aw = g.W; a.X = g.part_y;
+  a.part_ml = g.part_ml; a.win_ml = g.win_ml; a.win_y = g.win_y; a.Sw = g.Sw;
+  a.out = g.out; a.outs_b = g.outs_b; a.err = const_cast<int*>(g.err);
+  a.NB = g.S; a.S = 1;
+  int bn_cap = 256;
+  while (bn_cap > 32 && g.S * bn_cap > 256) bn_cap >>= 1;
+  return launch_bn<KIND_OMAP, 1, 3>(a, g.B, g.rows, g.S, bn_cap, st);
+}
+
+// ---------------------------------------------------------------- writer --
+bool writer_tc_ok(const WriterArgs& w) {
+  if (!al16(w.x) || (w.xv && !al16(w.xv))) return false;
+  if (w.xs_b % 4 || w.xs_n % 4 || w.xs_t % 4) return false;
+  const float* es[4] = {w.E_main, w.E_1, w.E_K, w.E_V};
+  for (const float* e : es)
+    if (e && !al16(e)) return false;
+  if (w.mode == LLA_WRITE_HLA) return w.D % 4 == 0;
+  return w.d_h % 4 == 0;
+}
+
+int writer_tc_splits(const WriterArgs& w, int num_sms) {
+  const int bn = std::min(pick_bn(w.M), 128);
+  int tiles = 0, nk_min = 1 << 30;
+  for (int z = 0; z < w.Z; ++z) {
+    const Slice s = slice_of(w, z);
+    tiles += ((s.N + GM - 1) / GM) * ((w.M + bn - 1) / bn);
+    nk_min = std::min(nk_min, (s.K_outer * s.d_in + KCH - 1) / KCH);
+  }
+  int S = num_sms / std::max(tiles, 1);        // one wave of CTAs (one per SM)
+  S = std::min(S, std::max(1, nk_min / 4));   // at least four chunks per split
+  return std::max(1, std::min(S, 64));
+}
+
+cudaError_t launch_writer_tc(const WriterArgs& w, int* err, cudaStream_t st) {
+  TcGemmArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.w = w; a.err = err; a.S = w.S; a.NB = 1;
+  a.mtiles = (w.Nmax + GM - 1) / GM;
+  return launch_bn<KIND_WRITER, 3, 2>(a, w.M, w.Z * w.S, 1, 128, st);
+}
+
+}  // namespace lla

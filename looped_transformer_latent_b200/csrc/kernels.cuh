@@ -6,6 +6,8 @@
 
 namespace lla {
 
+constexpr int kMaxWindowChunks = 16;   // window partials one call can produce
+
 // ---------------------------------------------------------------- writer --
 struct WriterArgs {
   int mode, B, n_tok, pos0, T, H, d_h, D, r_k, r_v, r_1, rotate;
@@ -20,11 +22,17 @@ struct WriterArgs {
   int Z;       // independent GEMMs (HLA: 2; PERHEAD: 2H; FOLDED: 2)
   int Nmax;    // largest output width over the Z GEMMs
   int S;       // split-K factor
+  int use_tc;  // phase 1 on the tensor cores (3xTF32)
   float* part; // [Z][S][M][Nmax] fp32 partial sums
+  int* err;    // tensor-core phase: set on a timed-out wait; the stores are then NaN
 };
 size_t writer_workspace_floats(const WriterArgs& a);
 int writer_pick_splits(const WriterArgs& a, int num_sms);
 cudaError_t launch_writer(const WriterArgs& a, cudaStream_t st);
+// tensor-core writer phase 1 (gemm_tc.cu)
+bool writer_tc_ok(const WriterArgs& w);
+int writer_tc_splits(const WriterArgs& w, int num_sms);
+cudaError_t launch_writer_tc(const WriterArgs& w, int* err, cudaStream_t st);
 
 // ------------------------------------------------------ absorbed decode --
 struct AbsorbArgs {
@@ -45,12 +53,12 @@ struct AbsorbArgs {
   float qmul;          // scale * log2(e): scores are kept in base-2 units
   // workspace views
   float *qlat;         // [B][rows][r_k]  (scaled, rotated)
-  float *qwin;         // [B][rows][d_h]  (scaled, rotated)
   float *part_ml;      // [S][B][rows][2] (running max, sum) per split
   float *part_y;       // [S][B][rows][r_v]
-  float *win_ml;       // [B][rows][2]
-  float *win_y;        // [B][rows][d_h]
+  float *win_ml;       // [Sw][B][rows][2] per window chunk
+  float *win_y;        // [Sw][B][rows][d_h]
   int S, tps;          // splits of the latent range, tokens per split
+  int Sw, cpt;         // window chunks, tokens per chunk
   // tensor-core path
   int use_tc;
   int rows_pad;        // rows rounded up to 16 (N of the accumulate MMA)
@@ -74,22 +82,34 @@ struct ReconArgs {
   int64_t outs_b;
   float qmul;
   float *part_ml, *part_y, *win_ml, *win_y;
-  int S, tps;
+  int S, tps, Sw, cpt;
 };
 
 // Shared pieces.
+// Window partials: one per (token chunk of cpt tokens, sequence, row).  The
+// query is the raw q [B][rows][d_h] (strides q_sb, q_srow), rotated by R_pos
+// in head space when `rotate` is set and multiplied by qmul.
 struct WindowArgs {
   int B, rows, H, d_h, t0, Wcap, win_start, n_win;
+  int Sw, cpt, HG;         // chunks, tokens per chunk, head groups (0: register kernel)
   const void *wk, *wv;
   int dtype;
   int64_t wins_b;
   const float* q;
   int64_t q_sb, q_srow;
   float qmul;
-  float *win_ml, *win_y;
+  int rotate, pos;
+  double base;
+  float *win_ml, *win_y;   // [Sw][B][rows][2], [Sw][B][rows][d_h]
+  int* err;                // optional: set to ERR_WINDOW_TIMEOUT if a copy never lands
 };
+constexpr int ERR_WINDOW_TIMEOUT = 21;
+// Kernel choice and chunking of the window for launch_window: returns the
+// chunk count, sets *cpt (tokens per chunk) and *HG (head groups of the
+// bulk-copy kernel, 0 for the register kernel).
+int window_chunks(int B, int nt, int H, int n_win, int dtype, int d_h, int num_sms, int* cpt, int* HG);
 struct MergeArgs {
-  int B, rows, H, d_h, S, Y;
+  int B, rows, H, d_h, S, Sw, Y;
   const float *part_ml, *part_y, *win_ml, *win_y;
   const float* Bm;   // [rows][Y][d_h] when mapping latent space back; else null
   float* out;
@@ -107,11 +127,12 @@ struct MapArgs {
   int rotate, pos, use_tc;
   double base;
   float qmul;
-  float *qlat, *qwin;
+  float* qlat;
   __nv_bfloat16* qbf;
-  // output map: X = sum over splits of the partials (K = r_v, N = d_h)
+  // output map: X = sum over splits of the partials (K = r_v, N = d_h), plus
+  // Sw window partials in head space
   const float *part_ml, *part_y, *win_ml, *win_y;
-  int S;
+  int S, Sw;
   float* out;
   int64_t outs_b;
   const int* err;
@@ -119,6 +140,26 @@ struct MapArgs {
 int map_max_splits();
 cudaError_t launch_query_map(const MapArgs& g, cudaStream_t st);
 cudaError_t launch_output_map(const MapArgs& g, cudaStream_t st);
+
+// Tensor-core maps (gemm_tc.cu): used with the tensor-core latent read.
+struct TcGemmArgs {
+  int B, rows, Mtot, K, mtiles, ntiles, S, NB, Sw;
+  const float *Aw, *X;     // codec [group][K][Mtot]; activations (per kind)
+  int64_t xs_b;
+  int rotate, pos, d_h;    // query map epilogue
+  double base;
+  float qmul;
+  __nv_bfloat16* qbf;
+  const float *part_ml, *win_ml, *win_y;   // output map epilogue
+  float* out;
+  int64_t outs_b;
+  int* err;
+  WriterArgs w;            // writer slices
+};
+bool query_map_tc_ok(const MapArgs& g);
+cudaError_t launch_query_map_tc(const MapArgs& g, int* err, cudaStream_t st);
+bool output_map_tc_ok(const MapArgs& g);
+cudaError_t launch_output_map_tc(const MapArgs& g, cudaStream_t st);
 
 cudaError_t launch_absorb_split_simt(const AbsorbArgs& a, cudaStream_t st);
 cudaError_t launch_window(const WindowArgs& w, cudaStream_t st);

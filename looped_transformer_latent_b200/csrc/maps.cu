@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
   constexpr int LX = GB * GK / GT;      // activation loads per thread
   __shared__ float Xs[2][GK][GB + 1];
   __shared__ __align__(16) float Ws[2][GK][GN];
-  __shared__ float wsplit[GB][MAXS + 1];   // MODE 1: split weights (last = window)
+  __shared__ float wsplit[GB][MAXS + kMaxWindowChunks];   // MODE 1: split, then window weights
   __shared__ float linv[GB];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x;
@@ -53,38 +53,27 @@ __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
       }
       return;
     }
-    if ((int)blockIdx.y == ntile) {
-      // window query: q_w = s*log2e * R_i q (head space)
-      const int hp = g.K / 2;
-      for (int idx = tid; idx < nb * hp; idx += GT) {
-        const int bb = idx / hp, p = idx % hp;
-        const float* q = g.X + (int64_t)(b0 + bb) * g.xs_b + (int64_t)row * g.xs_row;
-        float c = 1.f, s = 0.f;
-        if (g.rotate) rope_cs(p, g.K, g.K, g.base, (double)g.pos, &c, &s);
-        const float x = q[2 * p], y = q[2 * p + 1];
-        float* dst = g.qwin + ((int64_t)(b0 + bb) * g.rows + row) * g.K + 2 * p;
-        dst[0] = (x * c - y * s) * g.qmul;
-        dst[1] = (x * s + y * c) * g.qmul;
-      }
-      return;
-    }
   } else {
-    // split weights of this tile's sequences
+    // weights of this tile's sequences: splits, then window chunks
+    const int64_t bstride = (int64_t)g.B * g.rows;
     for (int bb = tid; bb < GB; bb += GT) {
       float M = -INFINITY, L = 0.f;
       if (bb < nb) {
         const int64_t br = (int64_t)(b0 + bb) * g.rows + row;
-        M = g.win_ml[br * 2];
-        for (int s = 0; s < g.S; ++s) M = fmaxf(M, g.part_ml[((int64_t)s * g.B * g.rows + br) * 2]);
+        for (int c = 0; c < g.Sw; ++c) M = fmaxf(M, g.win_ml[(c * bstride + br) * 2]);
+        for (int s = 0; s < g.S; ++s) M = fmaxf(M, g.part_ml[(s * bstride + br) * 2]);
         for (int s = 0; s < g.S; ++s) {
-          const float ms = g.part_ml[((int64_t)s * g.B * g.rows + br) * 2];
+          const float ms = g.part_ml[(s * bstride + br) * 2];
           const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
           wsplit[bb][s] = w;
-          L += w * g.part_ml[((int64_t)s * g.B * g.rows + br) * 2 + 1];
+          L += w * g.part_ml[(s * bstride + br) * 2 + 1];
         }
-        const float ww = exp2f(g.win_ml[br * 2] - M);
-        wsplit[bb][MAXS] = ww;
-        L += ww * g.win_ml[br * 2 + 1];
+        for (int c = 0; c < g.Sw; ++c) {
+          const float mc = g.win_ml[(c * bstride + br) * 2];
+          const float w = mc == -INFINITY ? 0.f : exp2f(mc - M);
+          wsplit[bb][MAXS + c] = w;
+          L += w * g.win_ml[(c * bstride + br) * 2 + 1];
+        }
       }
       linv[bb] = bb < nb ? 1.f / L : 0.f;
     }
@@ -181,11 +170,16 @@ __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
       if (bb >= nb) break;
       const int b = b0 + bb;
       const int64_t br = (int64_t)b * g.rows + row;
-      const float ww = wsplit[bb][MAXS], li = linv[bb];
+      const float li = linv[bb];
+      float y0 = acc[j][0], y1 = acc[j][1];
+      for (int c = 0; c < g.Sw; ++c) {
+        const float* yw = g.win_y + ((int64_t)c * g.B * g.rows + br) * g.N + n;
+        y0 = fmaf(wsplit[bb][MAXS + c], yw[0], y0);
+        y1 = fmaf(wsplit[bb][MAXS + c], yw[1], y1);
+      }
       float* dst = g.out + (int64_t)b * g.outs_b + (int64_t)row * g.N + n;
-      const float* yw = g.win_y + br * g.N + n;
-      dst[0] = bad ? NAN : (acc[j][0] + ww * yw[0]) * li;
-      dst[1] = bad ? NAN : (acc[j][1] + ww * yw[1]) * li;
+      dst[0] = bad ? NAN : y0 * li;
+      dst[1] = bad ? NAN : y1 * li;
     }
   }
 }
@@ -196,7 +190,7 @@ int map_max_splits() { return MAXS; }
 
 cudaError_t launch_query_map(const MapArgs& g, cudaStream_t st) {
   const int ntile = (g.N + GN - 1) / GN;
-  dim3 grid(g.use_tc ? 64 : g.rows, ntile + 1, (g.B + 31) / 32);
+  dim3 grid(g.use_tc ? 64 : g.rows, ntile, (g.B + 31) / 32);
   row_gemm<0, 32, 32><<<grid, GT, 0, st>>>(g);
   return cudaGetLastError();
 }

@@ -5,66 +5,12 @@
 // split-K SIMT fp32 GEMM writing partial sums to the workspace; phase 2 adds
 // the partials in a fixed order (deterministic), rotates key pairs by
 // R~_pos (HLA), rounds once to the storage type and stores the cache rows.
-#include "kernels.cuh"
+#include "writer_slice.cuh"
 
 namespace lla {
 namespace {
 
 constexpr int BK = 32, WT = 256;
-
-struct Slice {
-  const float* X;
-  int64_t x_o_t, x_o_h;
-  int o_h;
-  const float* E;
-  int64_t e_o, e_n;
-  int K_outer, d_in, N;
-  void* out;
-  int64_t os_b, os_n, col0;
-  int rot_dim;
-};
-
-__device__ __forceinline__ Slice slice_of(const WriterArgs& a, int z) {
-  Slice s;
-  if (a.mode == LLA_WRITE_HLA) {
-    if (z == 0) {  // c_j = sum_{t=2..T} E_t h_{j,t}
-      s.X = a.x + a.xs_t; s.x_o_t = a.xs_t; s.x_o_h = 0; s.o_h = 1;
-      s.N = a.r_k + a.r_v;
-      s.E = a.E_main; s.e_o = (int64_t)s.N * a.D; s.e_n = a.D;
-      s.K_outer = a.T - 1; s.d_in = a.D;
-      s.out = a.out0; s.os_b = a.os_b; s.os_n = a.os_n; s.col0 = 0;
-      s.rot_dim = a.rotate ? a.r_k : 0;
-    } else {       // c^(1)_j = E_1 h_{j,1}
-      s.X = a.x; s.x_o_t = 0; s.x_o_h = 0; s.o_h = 1;
-      s.N = 2 * a.r_1;
-      s.E = a.E_1; s.e_o = 0; s.e_n = a.D;
-      s.K_outer = 1; s.d_in = a.D;
-      s.out = a.out1; s.os_b = a.o1s_b; s.os_n = a.o1s_n; s.col0 = 0;
-      s.rot_dim = a.rotate ? a.r_1 : 0;
-    }
-  } else if (a.mode == LLA_WRITE_PERHEAD) {  // c_{j,h} = sum_t E_{t,h} k_{j,t,h}
-    const int part = z / a.H, h = z % a.H;
-    const int r = part ? a.r_v : a.r_k;
-    s.X = (part ? a.xv : a.x) + (int64_t)h * a.d_h; s.x_o_t = a.xs_t; s.x_o_h = 0; s.o_h = 1;
-    s.N = r;
-    s.E = (part ? a.E_V : a.E_K) + (int64_t)h * r * a.d_h;
-    s.e_o = (int64_t)a.H * r * a.d_h; s.e_n = a.d_h;
-    s.K_outer = a.T; s.d_in = a.d_h;
-    s.out = part ? a.out1 : a.out0; s.os_b = a.os_b; s.os_n = a.os_n;
-    s.col0 = (int64_t)h * a.os_h;
-    s.rot_dim = 0;
-  } else {  // FOLDED: c_j = sum_{t,h} E_{t,h} k_{j,t,h}
-    const int part = z;
-    const int r = part ? a.r_v : a.r_k;
-    s.X = part ? a.xv : a.x; s.x_o_t = a.xs_t; s.x_o_h = a.d_h; s.o_h = a.H;
-    s.N = r;
-    s.E = part ? a.E_V : a.E_K; s.e_o = (int64_t)r * a.d_h; s.e_n = a.d_h;
-    s.K_outer = a.T * a.H; s.d_in = a.d_h;
-    s.out = a.out0; s.os_b = a.os_b; s.os_n = a.os_n; s.col0 = part ? a.r_k : 0;
-    s.rot_dim = 0;
-  }
-  return s;
-}
 
 // Phase 1: C_part[z][split][m][n] = sum over this split's k-chunks.  Tile
 // TM x TN (64 x 64, or 32 x 128 for decode-size batches), 32-deep k-chunks
@@ -175,6 +121,7 @@ __global__ void writer_epilogue(WriterArgs a) {
       x += P[n];
       y += P[n + 1];
     }
+    if (*a.err) x = y = NAN;
     const int b = m / a.n_tok, j = m % a.n_tok;
     const int pos = a.pos0 + j;
     if (n < s.rot_dim) {
@@ -191,8 +138,9 @@ __global__ void writer_epilogue(WriterArgs a) {
 
 }  // namespace
 
+// Partial sums, then (16 bytes) the tensor-core error flag.
 size_t writer_workspace_floats(const WriterArgs& a) {
-  return (size_t)a.Z * a.S * a.M * a.Nmax;
+  return (size_t)a.Z * a.S * a.M * a.Nmax + 4;
 }
 
 static bool small_batch(const WriterArgs& a) { return a.M <= 32; }
@@ -213,16 +161,22 @@ int writer_pick_splits(const WriterArgs& a, int num_sms) {
   return S;
 }
 
-cudaError_t launch_writer(const WriterArgs& a, cudaStream_t st) {
+cudaError_t launch_writer(const WriterArgs& a_in, cudaStream_t st) {
+  WriterArgs a = a_in;
   if (a.M == 0) return cudaSuccess;
-  if (small_batch(a)) {
+  a.err = reinterpret_cast<int*>(a.part + (size_t)a.Z * a.S * a.M * a.Nmax);
+  cudaError_t e0 = cudaMemsetAsync(a.err, 0, sizeof(int), st);
+  if (e0 != cudaSuccess) return e0;
+  if (a.use_tc) {
+    e0 = launch_writer_tc(a, a.err, st);
+  } else if (small_batch(a)) {
     dim3 grid(ceil_div(a.Nmax, 128), ceil_div(a.M, 32), a.Z * a.S);
     writer_gemm<32, 128><<<grid, WT, 0, st>>>(a);
   } else {
     dim3 grid(ceil_div(a.Nmax, 64), ceil_div(a.M, 64), a.Z * a.S);
     writer_gemm<64, 64><<<grid, WT, 0, st>>>(a);
   }
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = a.use_tc ? e0 : cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t total = (int64_t)a.Z * a.M * (a.Nmax / 2);
   int blocks = (int)((total + 255) / 256);

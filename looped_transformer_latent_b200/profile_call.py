@@ -1,13 +1,17 @@
-"""Run one absorbed-read call of a configuration's latent on synthetic inputs.
+"""Run one call of the hot path on synthetic inputs of a configuration's shapes.
 
     python -m looped_transformer_latent_b200.profile_call --config ouro_hla_4k \
         --group main --batch 16 --iters 3
+    python -m looped_transformer_latent_b200.profile_call --op write \
+        --config ouro_lla2d_768 --batch 768 --iters 3
 
-A small, self-contained workload for profilers (ncu): it builds random bf16
-latents and fp32 codecs/queries of the configuration's shapes on the device,
-then calls hla_decode_attn `iters` times on one stream and synchronises.
-`--group main` reads the main latent (loops 2..T share it), `--group loop1`
-the loop-1 latent, `--group folded` an LLA-2D latent (no rotation).
+A small, self-contained workload for profilers (ncu).  `--op read` (default)
+builds random bf16 latents and fp32 codecs/queries on the device and calls
+hla_decode_attn `iters` times: `--group main` reads the main latent (loops
+2..T share it), `--group loop1` the loop-1 latent, `--group folded` an LLA-2D
+latent (no rotation).  `--op write` calls lla_write_latents for one decode
+token per sequence in the configuration's writer mode (HLA, LLA-2D folded or
+LLA per-head).
 """
 
 import argparse
@@ -31,19 +35,23 @@ def main():
     ap.add_argument("--group", default="main", choices=["main", "loop1", "folded"])
     ap.add_argument("--batch", type=int, default=16)
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--op", default="read", choices=["read", "write"])
+    ap.add_argument("--context", type=int, default=0, help="override the context length N (read)")
     args = ap.parse_args()
     c = synth.CONFIGS[args.config]
     dev = torch.device("cuda", 0)
     g = torch.Generator(device=dev)
     g.manual_seed(7)
     B = args.batch
+    if args.op == "write":
+        return write(L, c, B, args.iters, g, dev)
     if args.group == "main":
         t0, nt, r_k, r_v, rotate = 1, c.T - 1, c.r_k, c.r_v, True
     elif args.group == "loop1":
         t0, nt, r_k, r_v, rotate = 0, 1, c.r_1, c.r_1, True
     else:
         t0, nt, r_k, r_v, rotate = 0, c.T, c.r_k, c.r_v, False
-    H, d_h, N, W = c.H, c.d_h, c.N, c.W
+    H, d_h, N, W = c.H, c.d_h, (args.context or c.N), c.W
     Wcap = W + 1
     lat = (torch.randn(B, N, r_k + r_v, generator=g, device=dev) * math.sqrt(d_h / r_k)).to(torch.bfloat16)
     A = torch.randn(nt, H, d_h, r_k, generator=g, device=dev) / math.sqrt(d_h)
@@ -60,6 +68,37 @@ def main():
     torch.cuda.synchronize()
     print(f"ok: {args.config} {args.group} B={B} N={N} rows={nt * H} r_k={r_k} r_v={r_v}, "
           f"latent bytes per call {lat[:, :max(0, N - 1 - W)].numel() * 2 / 1e6:.1f} MB")
+
+
+def write(L, c, B, iters, g, dev):
+    pos = 0   # the row written does not change the work; row 0 keeps the buffers small
+    if c.kind == "hla":
+        h = torch.randn(B, 1, c.T, c.D, generator=g, device=dev)
+        E = torch.randn(c.T - 1, c.r_k + c.r_v, c.D, generator=g, device=dev) / math.sqrt(c.D)
+        E1 = torch.randn(2 * c.r_1, c.D, generator=g, device=dev) / math.sqrt(c.D)
+        out0 = torch.empty(B, pos + 1, c.r_k + c.r_v, dtype=torch.bfloat16, device=dev)
+        out1 = torch.empty(B, pos + 1, 2 * c.r_1, dtype=torch.bfloat16, device=dev)
+        kw = dict(x=h, E_main=E, E_1=E1, out0=out0, out1=out1, r_k=c.r_k, d_h=c.d_h, pos0=pos, rope_base=c.base)
+        mode = L.LLA_WRITE_HLA
+    else:
+        k = torch.randn(B, 1, c.T, c.H, c.d_h, generator=g, device=dev)
+        v = torch.randn(B, 1, c.T, c.H, c.d_h, generator=g, device=dev)
+        EK = torch.randn(c.T, c.H, c.r_k, c.d_h, generator=g, device=dev) / math.sqrt(c.d_h)
+        EV = torch.randn(c.T, c.H, c.r_v, c.d_h, generator=g, device=dev) / math.sqrt(c.d_h)
+        if c.kind == "lla2d":
+            out0 = torch.empty(B, pos + 1, c.r_k + c.r_v, dtype=torch.bfloat16, device=dev)
+            kw = dict(x=k, xv=v, E_K=EK, E_V=EV, out0=out0, pos0=pos)
+            mode = L.LLA_WRITE_FOLDED
+        else:
+            out0 = torch.empty(B, c.H, pos + 1, c.r_k, dtype=torch.bfloat16, device=dev)
+            out1 = torch.empty(B, c.H, pos + 1, c.r_v, dtype=torch.bfloat16, device=dev)
+            kw = dict(x=k, xv=v, E_K=EK, E_V=EV, out0=out0, out1=out1, pos0=pos)
+            mode = L.LLA_WRITE_PERHEAD
+    ws = torch.empty(max(256, L.lla_write_workspace_bytes(mode, **kw)), dtype=torch.uint8, device=dev)
+    for _ in range(iters):
+        L.lla_write_latents(mode, workspace=ws, **kw)
+    torch.cuda.synchronize()
+    print(f"ok: write {c.name} B={B} mode={mode}")
 
 
 if __name__ == "__main__":

@@ -237,9 +237,23 @@ def test_writer_lla_layout_bit_exact(cuda_device, mode):
         assert torch.equal(lat.cpu(), e.to(torch.bfloat16))
 
 
+def _accumulation_bound(x_blocks, e_blocks):
+    """Bound on the fp32 accumulation error of each written value: the sum of
+    the magnitudes of its K products times sqrt(K) 2^-22 (a few fp32 roundings
+    per product, random-walk growth), widened over each rotated pair (a
+    rotation mixes the two members with |cos| + |sin| <= 2)."""
+    ax = np.abs(np.concatenate([np.asarray(b, np.float64) for b in x_blocks], axis=1))
+    ae = np.abs(np.concatenate([np.asarray(b, np.float64) for b in e_blocks], axis=1))
+    s = ax @ ae.T
+    s = np.maximum(s[:, 0::2], s[:, 1::2]).repeat(2, axis=1) * 2.0
+    return np.sqrt(ax.shape[1]) * 2.0 ** -22 * s
+
+
 def test_writer_rotation_and_rounding(cuda_device):
-    """Rotated bf16 writes: each value within one bf16 rounding of the
-    oracle's (fp32 accumulation order may move a value across a tie)."""
+    """Rotated bf16 writes: each value within one bf16 ulp of the oracle's plus
+    the fp32 accumulation error bound (where a value cancels to far below its
+    terms, fp32 summation alone can move it by more than one bf16 ulp), and
+    at least 95 % of the values equal to the oracle's rounded value."""
     c = synth.CONFIGS["tiny_hla"]
     x = synth.tiny_hla(1)
     dev = cuda_device
@@ -253,9 +267,12 @@ def test_writer_rotation_and_rounding(cuda_device):
                         d_h=c.d_h, pos0=pos0, rope_base=c.base)
     torch.cuda.synchronize()
     ce, c1e = hla.write(x["h"][:n], x["E_main"], x["E_1"], pos0, c.r_k, c.r_v, c.r_1, c.d_h, c.base)
-    for got, exact in ((f64(lat[0, pos0:]), ce), (f64(lat1[0, pos0:]), c1e)):
+    hx = x["h"][:n]
+    acc_main = _accumulation_bound([hx[:, t] for t in range(1, c.T)], list(x["E_main"]))
+    acc_1 = _accumulation_bound([hx[:, 0]], [x["E_1"]])
+    for got, exact, acc in ((f64(lat[0, pos0:]), ce, acc_main), (f64(lat1[0, pos0:]), c1e, acc_1)):
         ulp = np.abs(rounding.to_bf16(exact)) * 2.0 ** -7 + 1e-30
-        assert np.all(np.abs(got - exact) <= ulp)
+        assert np.all(np.abs(got - exact) <= ulp + acc)
         assert np.mean(got == rounding.to_bf16(exact)) > 0.95
 
 
