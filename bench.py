@@ -470,20 +470,29 @@ def run_reference(args, cfg):
 
 
 # DRAM traffic (read + write) per latent token of the tensor-core latent read,
-# from one ncu capture of the Ouro main latent (profiles/absorb_split_tc_ouro_main_b16.md),
-# keyed by the sha256 prefix of the kernel source it was taken on: a changed
-# kernel reports no traffic until it is captured again.
-TC_TRAFFIC_PER_TOKEN = {"5163ad08b2a9e31d": 2122.7}
+# from ncu captures (profiles/absorb_split_tc_*.md), keyed by the sha256 prefix
+# of the kernel source it was taken on and the latent row width in bytes: a
+# changed kernel, or a row width never captured, reports no traffic.
+TC_TRAFFIC_PER_TOKEN = {("5163ad08b2a9e31d", 2048): 2122.7}
 
 
-def tc_traffic_per_token():
+def tc_traffic_per_token(row_bytes):
     import hashlib
     src = os.path.join(ROOT, "looped_transformer_latent_b200", "csrc", "decode_tc.cu")
     try:
         h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     except OSError:
         return None
-    return TC_TRAFFIC_PER_TOKEN.get(h)
+    return TC_TRAFFIC_PER_TOKEN.get((h, row_bytes))
+
+
+def reduce_max(dist, value, device):
+    """Max of a per-rank float over all ranks (the value itself on one rank)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def main():
@@ -553,10 +562,8 @@ def main():
     clocks = sampler.stop()
     ms = t0.elapsed_time(t1) / args.steps
     split_ms = [a.elapsed_time(b) for a, b in evs]       # last replay of the timed region
+    ms = reduce_max(dist, ms, dev)
     if dist is not None:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
         dist.barrier()
 
     # end to end: pinned host inputs -> device, step, outputs -> host
@@ -588,10 +595,7 @@ def main():
         e1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1) / args.steps
-    if dist is not None:
-        tt = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_e2e = float(tt.item())
+    ms_e2e = reduce_max(dist, ms_e2e, dev)
 
     hbm, tflops, src = peaks()
     lb = step.read_latent_bytes()
@@ -601,11 +605,10 @@ def main():
     mean_ms = sum(main_ms) / max(1, len(main_ms))
     achieved = (sum(main_bytes) / 1e9) / (sum(main_ms) / 1e3) if sum(main_ms) > 0 else 0.0
     all_gbs = (sum(lb) / 1e9) / (sum(split_ms) / 1e3) if sum(split_ms) > 0 else 0.0
-    per_tok = tc_traffic_per_token() if cfg.kind != "lla" else None
+    per_tok = tc_traffic_per_token((cfg.r_k + cfg.r_v) * 2) if cfg.kind != "lla" else None
     traffic = None
     if per_tok is not None and main_ix:
-        c0 = cfg
-        traffic = per_tok * c0.B * step.n_lat
+        traffic = per_tok * cfg.B * step.n_lat
     step_bytes = step.step_bytes()
     tokens = cfg.B * world
     srt = sorted(main_ms)

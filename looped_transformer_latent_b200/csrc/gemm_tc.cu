@@ -138,7 +138,7 @@ struct Tile {
 
 template <int KIND, int BN, int PREC, int DEPTH>
 __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const TcGemmArgs a) {
-  constexpr int NST = DEPTH + 1;
+  const int NST = a.nst;   // stages in the ring (> DEPTH; the host sizes it to shared memory)
   constexpr bool A_MN = KIND != KIND_WRITER;   // codec operand MN-major (maps) or K-major (writer)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -352,41 +352,88 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const TcGemmArgs a) {
     }
     cp_async_wait<0>();
 
-    // ---- output-map weights (while the last MMAs run) ---------------------
-    if (KIND == KIND_OMAP) {
-      const int ld = a.NB + a.Sw + 1;
-      const int64_t bstride = (int64_t)a.B * a.rows;
-      for (int bb = tid; bb < BN; bb += NPROD) {
-        const int b = t.n0 + bb;
-        float* w = wts + bb * ld;
-        if (b >= a.B) {
-          for (int j = 0; j < ld; ++j) w[j] = 0.f;
-          continue;
-        }
-        const int64_t br = (int64_t)b * a.rows + t.g;
-        float M = -INFINITY, L = 0.f;
-        for (int s = 0; s < a.NB; ++s) M = fmaxf(M, a.part_ml[(s * bstride + br) * 2]);
-        for (int c = 0; c < a.Sw; ++c) M = fmaxf(M, a.win_ml[(c * bstride + br) * 2]);
-        for (int s = 0; s < a.NB; ++s) {
-          const float ms = a.part_ml[(s * bstride + br) * 2];
-          const float ws = ms == -INFINITY ? 0.f : exp2f(ms - M);
-          w[s] = ws;
-          L += ws * a.part_ml[(s * bstride + br) * 2 + 1];
-        }
-        for (int c = 0; c < a.Sw; ++c) {
-          const float mc = a.win_ml[(c * bstride + br) * 2];
-          const float wc = mc == -INFINITY ? 0.f : exp2f(mc - M);
-          w[a.NB + c] = wc;
-          L += wc * a.win_ml[(c * bstride + br) * 2 + 1];
-        }
-        w[a.NB + a.Sw] = 1.f / L;
-      }
-      named_sync(1, NPROD);
-    }
-
     // ---- epilogue ------------------------------------------------------------
     const bool ok = wait_bar(smem_u32(done), 0, abort_flag, a.err, ERR_GEMM_DONE, false) && !*abort_flag;
     tc_fence_after();
+    // Output map, now that every MMA has completed and the stage memory is
+    // free: (1) gather the (max, sum) of every split and window partial of the
+    // tile's sequences with all producer threads; (2) one thread per sequence
+    // turns them into weights 2^(m - M) and 1 / l; (3) gather the window term
+    // sum_c w_c y_c of every (sequence, column) with coalesced loads.
+    float* ywin = reinterpret_cast<float*>(base);              // [BN][GM]
+    if (KIND == KIND_OMAP) {
+      const int ne = a.NB + a.Sw;                              // partials per sequence
+      const int ld = ne + 1;
+      const int64_t bstride = (int64_t)a.B * a.rows;
+      float2* mls = reinterpret_cast<float2*>(base + (size_t)BN * GM * 4);   // [BN][ne]
+#pragma unroll 4
+      for (int idx = tid; idx < BN * ne; idx += NPROD) {
+        const int bb = idx / ne, e = idx % ne;
+        const int n = t.n0 + bb;
+        float2 v = make_float2(-INFINITY, 0.f);
+        if (n < t.Nv) {
+          const int64_t br = (int64_t)n * a.rows + t.g;
+          const float* src = e < a.NB ? a.part_ml + (e * bstride + br) * 2 : a.win_ml + ((e - a.NB) * bstride + br) * 2;
+          v = make_float2(src[0], src[1]);
+        }
+        mls[idx] = v;
+      }
+      named_sync(1, NPROD);
+      for (int bb = tid; bb < BN; bb += NPROD) {
+        const float2* e = mls + bb * ne;
+        float* w = wts + bb * ld;
+        float M = -INFINITY;
+        for (int j = 0; j < ne; ++j) M = fmaxf(M, e[j].x);
+        float L = 0.f;
+        for (int j = 0; j < ne; ++j) {
+          const float wj = e[j].x == -INFINITY ? 0.f : exp2f(e[j].x - M);
+          w[j] = wj;
+          L += wj * e[j].y;
+        }
+        w[ne] = t.n0 + bb < t.Nv ? 1.f / L : 0.f;
+      }
+      named_sync(1, NPROD);
+      // float4 groups of 4 columns; per pass each thread keeps 4 groups and
+      // loops over the window chunks outermost, so its loads of a chunk are
+      // independent and in flight together
+      constexpr int G4 = BN * GM / 4;                 // float4 groups in the tile
+      for (int base4 = 0; base4 < G4; base4 += 4 * NPROD) {
+        float4 acc4[4];
+        int64_t off4[4];
+        bool live[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx4 = base4 + u * NPROD + tid;
+          const int bb = idx4 / (GM / 4), mm = 4 * (idx4 % (GM / 4));
+          const int n = t.n0 + bb, m = t.m0 + mm;
+          live[u] = idx4 < G4 && n < t.Nv && m < t.Mv;
+          off4[u] = live[u] ? ((int64_t)n * a.rows + t.g) * a.Mtot + m : 0;
+          acc4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int cw = 0; cw < a.Sw; ++cw) {
+          float4 v4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            v4[u] = live[u] ? *reinterpret_cast<const float4*>(a.win_y + cw * bstride * a.Mtot + off4[u])
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int idx4 = base4 + u * NPROD + tid;
+            const float w = live[u] ? wts[(idx4 / (GM / 4)) * ld + a.NB + cw] : 0.f;
+            acc4[u].x = fmaf(w, v4[u].x, acc4[u].x);
+            acc4[u].y = fmaf(w, v4[u].y, acc4[u].y);
+            acc4[u].z = fmaf(w, v4[u].z, acc4[u].z);
+            acc4[u].w = fmaf(w, v4[u].w, acc4[u].w);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx4 = base4 + u * NPROD + tid;
+          if (idx4 < G4) reinterpret_cast<float4*>(ywin)[idx4] = acc4[u];
+        }
+      }
+      named_sync(1, NPROD);
+    }
     // warps w and w + 4 share TMEM lanes 32 (w & 3) .. +31 and split the columns
     const int quarter = warp & 3, half = warp >> 2;
     const int m = t.m0 + 32 * quarter + lane;   // this thread's TMEM lane = codec row
@@ -428,23 +475,22 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const TcGemmArgs a) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float other = __shfl_xor_sync(0xffffffffu, v[i], 1);
+          // even lanes hold x of the pair, odd lanes y; the even lane stores both
           const float x = (m & 1) ? other : v[i], y = (m & 1) ? v[i] : other;
-          const float r = (m & 1) ? (x * sq + y * cq) : (x * cq - y * sq);
           const int n = t.n0 + 16 * c + i;
-          if (m < t.Mv && n < t.Nv)
-            a.qbf[qbf_index(n, t.g, m, a.Mtot)] = __float2bfloat16_rn(bad ? NAN : r * a.qmul);
+          if (!(m & 1) && m < t.Mv && n < t.Nv) {
+            const float rx = bad ? NAN : (x * cq - y * sq) * a.qmul;
+            const float ry = bad ? NAN : (x * sq + y * cq) * a.qmul;
+            *reinterpret_cast<__nv_bfloat162*>(a.qbf + qbf_index(n, t.g, m, a.Mtot)) = __floats2bfloat162_rn(rx, ry);
+          }
         }
       } else if (KIND == KIND_OMAP) {
         const int ld = a.NB + a.Sw + 1;
-        const int64_t bstride = (int64_t)a.B * a.rows;
 #pragma unroll 4
         for (int i = 0; i < 16; ++i) {
           const int bb = 16 * c + i, n = t.n0 + bb;
           if (m >= t.Mv || n >= t.Nv) continue;
-          float y = v[i];
-          const int64_t br = (int64_t)n * a.rows + t.g;
-          for (int cw = 0; cw < a.Sw; ++cw)
-            y = fmaf(wts[bb * ld + a.NB + cw], a.win_y[(cw * bstride + br) * a.Mtot + m], y);
+          const float y = v[i] + ywin[bb * GM + (m - t.m0)];
           a.out[(int64_t)n * a.outs_b + (int64_t)t.g * a.Mtot + m] = bad ? NAN : y * wts[bb * ld + a.NB + a.Sw];
         }
       } else {
@@ -499,10 +545,19 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const TcGemmArgs a) {
 }
 
 template <int KIND, int BN, int PREC, int DEPTH>
-cudaError_t launch_one(const TcGemmArgs& a, int grid_y, int nb, cudaStream_t st) {
+cudaError_t launch_one(TcGemmArgs a, int grid_y, int nb, size_t smem_budget, cudaStream_t st) {
   const int stage = (A_BYTES * (PREC == 3 ? 2 : 1)) + BN * 128 * nb * (PREC == 3 ? 2 : 1);
   const int wts = KIND == KIND_OMAP ? BN * (nb + a.Sw + 1) * 4 : 0;
-  size_t smem = 1024 + (size_t)(DEPTH + 1) * stage + 8 * (2 * (DEPTH + 1) + 1) + 16 + wts;
+  // stages: at least DEPTH + 1, up to DEPTH + 3 (slack between the copies in
+  // flight and the stage the MMA is still reading) as the budget allows
+  const size_t fixed = 1024 + 16 + wts;
+  int nst = DEPTH + 1;
+  while (nst < DEPTH + 3 && fixed + (size_t)(nst + 1) * (stage + 16) + 8 <= smem_budget) ++nst;
+  a.nst = nst;
+  // the output map's epilogue tiles (window term, partial maxima) reuse the stages
+  if (KIND == KIND_OMAP && (size_t)BN * GM * 4 + (size_t)BN * (nb + a.Sw) * 8 > (size_t)nst * stage)
+    return cudaErrorInvalidConfiguration;
+  size_t smem = fixed + (size_t)nst * stage + 8 * (2 * nst + 1);
   // keep the CTAs an SM can hold (228 KB of shared memory, 1 KB reserved per
   // CTA) within its 512 TMEM columns, so that no allocation ever waits
   int ncols = 32;
@@ -522,14 +577,14 @@ cudaError_t launch_one(const TcGemmArgs& a, int grid_y, int nb, cudaStream_t st)
 int pick_bn(int n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : 256; }
 
 template <int KIND, int PREC, int DEPTH>
-cudaError_t launch_bn(TcGemmArgs a, int Nv, int grid_y, int nb, int bn_cap, cudaStream_t st) {
+cudaError_t launch_bn(TcGemmArgs a, int Nv, int grid_y, int nb, int bn_cap, size_t smem_budget, cudaStream_t st) {
   const int bn = std::min(pick_bn(Nv), bn_cap);
   a.ntiles = (Nv + bn - 1) / bn;
   switch (bn) {
-    case 32: return launch_one<KIND, 32, PREC, DEPTH>(a, grid_y, nb, st);
-    case 64: return launch_one<KIND, 64, PREC, DEPTH>(a, grid_y, nb, st);
-    case 128: return launch_one<KIND, 128, PREC, DEPTH>(a, grid_y, nb, st);
-    default: return launch_one<KIND, 256, PREC, DEPTH>(a, grid_y, nb, st);
+    case 32: return launch_one<KIND, 32, PREC, DEPTH>(a, grid_y, nb, smem_budget, st);
+    case 64: return launch_one<KIND, 64, PREC, DEPTH>(a, grid_y, nb, smem_budget, st);
+    case 128: return launch_one<KIND, 128, PREC, DEPTH>(a, grid_y, nb, smem_budget, st);
+    default: return launch_one<KIND, 256, PREC, DEPTH>(a, grid_y, nb, smem_budget, st);
   }
 }
 
@@ -550,7 +605,7 @@ cudaError_t launch_query_map_tc(const MapArgs& g, int* err, cudaStream_t st) {
   a.Aw = g.W; a.X = g.X; a.xs_b = g.xs_b;
   a.rotate = g.rotate; a.pos = g.pos; a.d_h = g.d_h; a.base = g.base; a.qmul = g.qmul; a.qbf = g.qbf;
   a.err = err; a.NB = 1; a.S = 1;
-  return launch_bn<KIND_QMAP, 1, 3>(a, g.B, 64, 1, 256, st);
+  return launch_bn<KIND_QMAP, 1, 2>(a, g.B, 64, 1, 128, SMEM_MAX / 2 - 1024, st);
 }
 
 // ------------------------------------------------------------ output map --
@@ -570,7 +625,7 @@ cudaError_t launch_output_map_tc(const MapArgs& g, cudaStream_t st) {
   a.NB = g.S; a.S = 1;
   int bn_cap = 256;
   while (bn_cap > 32 && g.S * bn_cap > 256) bn_cap >>= 1;
-  return launch_bn<KIND_OMAP, 1, 3>(a, g.B, g.rows, g.S, bn_cap, st);
+  return launch_bn<KIND_OMAP, 1, 3>(a, g.B, g.rows, g.S, bn_cap, SMEM_MAX, st);
 }
 
 // ---------------------------------------------------------------- writer --
@@ -602,7 +657,7 @@ cudaError_t launch_writer_tc(const WriterArgs& w, int* err, cudaStream_t st) {
   std::memset(&a, 0, sizeof(a));
   a.w = w; a.err = err; a.S = w.S; a.NB = 1;
   a.mtiles = (w.Nmax + GM - 1) / GM;
-  return launch_bn<KIND_WRITER, 3, 2>(a, w.M, w.Z * w.S, 1, 128, st);
+  return launch_bn<KIND_WRITER, 3, 2>(a, w.M, w.Z * w.S, 1, 128, SMEM_MAX, st);
 }
 
 }  // namespace lla

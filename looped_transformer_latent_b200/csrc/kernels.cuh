@@ -144,6 +144,7 @@ cudaError_t launch_output_map(const MapArgs& g, cudaStream_t st);
 // Tensor-core maps (gemm_tc.cu): used with the tensor-core latent read.
 struct TcGemmArgs {
   int B, rows, Mtot, K, mtiles, ntiles, S, NB, Sw;
+  int nst;                 // shared-memory stages (set by the launcher)
   const float *Aw, *X;     // codec [group][K][Mtot]; activations (per kind)
   int64_t xs_b;
   int rotate, pos, d_h;    // query map epilogue
