@@ -345,7 +345,11 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
   qm.qlat = a.qlat; qm.qbf = a.qbf;
   cudaError_t e = cudaSuccess;
   e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
-  if (e == cudaSuccess) e = query_map_tc_ok(qm) ? launch_query_map_tc(qm, a.err, s) : launch_query_map(qm, s);
+  if (e == cudaSuccess) {
+    // tensor-core map when the shapes allow a tensor-map view, else the SIMT map
+    e = query_map_tc_ok(qm) ? launch_query_map_tc(qm, a.err, s) : cudaErrorNotSupported;
+    if (e == cudaErrorNotSupported) e = launch_query_map(qm, s);
+  }
   if (e == cudaSuccess) e = mark(p->timing_events, 0, s);
   if (e == cudaSuccess && a.n_lat > 0)
     e = a.use_tc ? launch_absorb_split_tc(a, s) : launch_absorb_split_simt(a, s);
@@ -367,7 +371,8 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
     om.part_ml = a.part_ml; om.part_y = a.part_y; om.win_ml = a.win_ml; om.win_y = a.win_y; om.S = a.S;
     om.Sw = a.Sw;
     om.out = a.out; om.outs_b = a.outs_b; om.err = a.err;
-    e = (a.use_tc && output_map_tc_ok(om)) ? launch_output_map_tc(om, s) : launch_output_map(om, s);
+    e = (a.use_tc && output_map_tc_ok(om)) ? launch_output_map_tc(om, s) : cudaErrorNotSupported;
+    if (e == cudaErrorNotSupported) e = launch_output_map(om, s);
   }
   return cuda_status(e);
 }

@@ -10,22 +10,26 @@
 // the codec) and the activations X_g (the N side: sequences or tokens, BN per
 // tile), so a decode batch of 32 and one of 768 both map onto the MMA's N.
 //
-// Operands are fp32 in HBM.  Four producer warps copy each 32-deep k-chunk
-// into 128-byte-swizzled shared memory with cp.async (zero-filling anything
-// out of range), then round their own pieces in place to tf32 (round to
-// nearest, ties away) and, for PREC = 3, store the remainder x - tf32(x) as a
-// second tf32 tile.  PREC = 3 issues hi*hi + hi*lo + lo*hi ("3xTF32"), whose
-// error is that of fp32 arithmetic; PREC = 1 issues hi*hi (relative error
-// about 2^-11 per product).  One thread of a fifth warp issues the MMAs into
-// TMEM and releases stages with tcgen05.commit; the producer warps then read
-// the accumulators back (tcgen05.ld) for the epilogue.  Waits are bounded:
-// on a timeout the CTA records an error code (outputs become NaN downstream).
+// Operands are fp32 in HBM.  One thread of a TMA warp copies each 32-deep
+// k-chunk of both operands into shared memory with tensor-map boxes that land
+// directly in the MMA layouts (128-byte swizzle; for the MN-major codec of the
+// maps the 128-byte swizzle with 32-byte atoms, the one layout the tensor
+// cores take for MN-major tf32); out-of-range elements arrive as zeros.  Eight
+// converter warps round each landed stage in place to tf32 (round to nearest,
+// ties away) and, for PREC = 3, store the remainder x - tf32(x) as a second
+// tf32 tile.  PREC = 3 issues hi*hi + hi*lo + lo*hi ("3xTF32"), whose error is
+// that of fp32 arithmetic; PREC = 1 issues hi*hi (relative error about 2^-11
+// per product).  One thread of an MMA warp issues the MMAs into TMEM and
+// releases stages with tcgen05.commit; the converter warps then read the
+// accumulators back (tcgen05.ld) for the epilogue.  Waits are bounded: on a
+// timeout the CTA records an error code (outputs become NaN downstream).
 #include <cuda.h>
 
 #include <algorithm>
 #include <cstring>
 
 #include "tc_ptx.cuh"
+#include "tmap.cuh"
 #include "writer_slice.cuh"
 
 namespace lla {
@@ -36,14 +40,21 @@ using namespace ptx;
 constexpr int GM = 128;                 // M of every MMA (codec rows per tile)
 constexpr int KCH = 32;                 // k per chunk: 32 fp32 = one 128-byte row
 constexpr int A_BYTES = GM * KCH * 4;   // 16 KB
-constexpr int NPROD = 256;              // producer + epilogue threads (warps 0-7)
-constexpr int NTHR = NPROD + 32;        // + warp 8: TMEM allocation, MMA issue
-constexpr int MMA_WARP = NPROD / 32;
+constexpr int NPROD = 256;              // converter + epilogue threads (warps 0-7)
+constexpr int MMA_WARP = NPROD / 32;    // warp 8: TMEM allocation, MMA issue
+constexpr int TMA_WARP = MMA_WARP + 1;  // warp 9: tensor-map copies
+constexpr int NTHR = NPROD + 64;
 constexpr int SMEM_MAX = 232448;
 constexpr long long WAIT_CYCLES = 1ll << 32;
 
 enum : int { KIND_QMAP = 0, KIND_OMAP = 1, KIND_WRITER = 2 };
-enum : int { ERR_GEMM_EMPTY = 11, ERR_GEMM_FULL = 12, ERR_GEMM_DONE = 13 };
+enum : int { ERR_GEMM_EMPTY = 11, ERR_GEMM_FULL = 12, ERR_GEMM_DONE = 13, ERR_GEMM_LOAD = 14 };
+
+// Tensor maps of one launch: codec operand(s) and activation operand(s).
+struct TcMaps {
+  CUtensorMap a[2];
+  CUtensorMap x[2];
+};
 
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn_major) {
   return (1u << 4)                          // D format: fp32
@@ -62,16 +73,6 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint6
       "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
-}
-
-// 16-byte global -> shared copy; src_bytes = 0 fills the 16 bytes with zeros.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
@@ -107,20 +108,12 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
-// Offset of 16-byte piece c (k = 4c .. 4c+3) of row r in a K-major SW128 tile.
-__device__ __forceinline__ uint32_t kmajor_off(int r, int c) {
-  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
-}
-// Offset of the 16-byte piece holding rows 4c32 .. 4c32+3 at depth kk in an
-// MN-major tf32 tile of 128 rows x 32 k, in the 128-byte swizzle with 32-byte
-// granules (the one layout the tensor cores accept for MN-major tf32): atoms
-// of 4 k-rows x 128 bytes (512 B) whose 32-byte granule index is XORed with
-// the k-row (mod 4); k-groups 512 B apart, 32-row MN atoms 4 KB apart.
-__device__ __forceinline__ uint32_t mnmajor_off(int kk, int c32) {
-  const int c = c32 & 7;
-  return (uint32_t)((c32 >> 3) * 4096 + (kk >> 2) * 512 + (kk & 3) * 128 + (((c >> 1) ^ (kk & 3)) << 5) +
-                    ((c & 1) << 4));
-}
+// Shared-memory operand layouts (written by the tensor-map copies):
+//   K-major tile (rows x 32 k): 128-byte rows, 8-row atoms of 1 KB, 16-byte
+//   pieces swizzled by row mod 8 -- descriptor LBO 16, SBO 1024;
+//   MN-major tf32 codec tile (128 rows x 32 k): four 32-row atoms 4 KB apart,
+//   each 32 k-rows of 128 bytes whose 32-byte granules are swizzled by k-row
+//   mod 4 -- descriptor layout type 1, LBO 4096 (atoms), SBO 512 (4 k-rows).
 
 __device__ __forceinline__ int64_t qbf_index(int b, int row, int k, int r_k) {
   const int kb = k >> 6, e = k & 63;
@@ -136,10 +129,9 @@ struct Tile {
   int kc0, kc1;     // chunk range
 };
 
-template <int KIND, int BN, int PREC, int DEPTH>
-__global__ void __launch_bounds__(NTHR, 1) tc_gemm(const TcGemmArgs a) {
-  const int NST = a.nst;   // stages in the ring (> DEPTH; the host sizes it to shared memory)
-  constexpr bool A_MN = KIND != KIND_WRITER;   // codec operand MN-major (maps) or K-major (writer)
+template <int KIND, int BN, int PREC>
+__global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMaps maps, const TcGemmArgs a) {
+  const int NST = a.nst;   // stages in the ring (the host sizes it to shared memory)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -187,16 +179,18 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const TcGemmArgs a) {
   const uint32_t stage_bytes = a_part + b_tile * nb * (PREC == 3 ? 2 : 1);
   const uint32_t sbase = smem_u32(base);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + NST * stage_bytes);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + NST;
-  uint64_t* done = bars + 2 * NST;
-  uint8_t* misc = reinterpret_cast<uint8_t*>(bars + 2 * NST + 1);
+  uint64_t* loaded = bars;            // [NST] TMA bytes landed
+  uint64_t* full = bars + NST;        // [NST] converted (all converter threads)
+  uint64_t* empty = bars + 2 * NST;   // [NST] MMAs reading the stage completed
+  uint64_t* done = bars + 3 * NST;
+  uint8_t* misc = reinterpret_cast<uint8_t*>(bars + 3 * NST + 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   float* wts = reinterpret_cast<float*>(misc + 16);   // output map: [BN][NB + Sw + 1]
 
   if (tid == 0) {
     for (int i = 0; i < NST; ++i) {
+      mbar_init(smem_u32(&loaded[i]), 1);
       mbar_init(smem_u32(&full[i]), NPROD);
       mbar_init(smem_u32(&empty[i]), 1);
     }
@@ -216,106 +210,8 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const TcGemmArgs a) {
   const uint32_t tmem = *tmem_slot;
 
   if (warp < NPROD / 32) {
-    // ---- producers ---------------------------------------------------------
-    // A thread's pieces of a chunk share one k (K-major: column c of every
-    // row r0 + 32u) or one codec row (MN-major: rows m .. m+3 at depths
-    // kk0 + 8u), so their addresses are a fixed base plus u times a stride,
-    // and moving to the next chunk only advances one running position.
-    constexpr int PA = A_BYTES / 16 / NPROD;   // A pieces per thread
-    constexpr int PB = BN * 8 / NPROD;         // pieces per thread of each B operand
-    const int c8 = tid & 7, r0 = tid >> 3;                 // K-major piece: column, first row
-    const int c32 = tid & 31, kk0 = tid >> 5;              // MN-major piece: row group, first depth
-    const uint32_t a_off0 = A_MN ? mnmajor_off(kk0, c32) : kmajor_off(r0, c8);
-    constexpr uint32_t A_OFF_U = A_MN ? 1024u * (NPROD / 256) : 4096u * (NPROD / 256);
-    const uint32_t b_off0 = kmajor_off(r0, c8);
-    constexpr uint32_t B_OFF_U = 4096u * (NPROD / 256);
-    // rows of the operands for this thread
-    const int a_row = A_MN ? t.m0 + 4 * c32 : t.m0 + r0;   // + 32u for K-major
-    // running k position of this thread's K-major pieces (the writer's
-    // (outer block, feature) decomposition is tracked incrementally)
-    int kpos = t.kc0 * KCH + 4 * c8;
-    int ob = 0, od = 0, ot = 0, oh = 0;
-    if (KIND == KIND_WRITER) {
-      ob = kpos / sl.d_in;
-      od = kpos % sl.d_in;
-      ot = ob / sl.o_h;
-      oh = ob % sl.o_h;
-    }
-    int64_t xrow[PB > 0 ? PB : 1];
-#pragma unroll
-    for (int u = 0; u < PB; ++u) {
-      const int n = t.n0 + r0 + 32 * (NPROD / 256) * u;
-      xrow[u] = 0;
-      if (n < t.Nv) {
-        if (KIND == KIND_WRITER) xrow[u] = writer_xrow(a.w, n);
-        else if (KIND == KIND_QMAP) xrow[u] = (int64_t)n * a.xs_b + (int64_t)t.g * t.K;
-        else xrow[u] = ((int64_t)n * a.rows + t.g) * t.K;
-      }
-    }
-    const int64_t b_jb_stride = (int64_t)a.B * a.rows * t.K;   // output map: between split partials
-    bool aborted = false;
-    auto issue = [&](int i) {
-      if (!aborted) {
-        const int st = i % NST;
-        if (i >= NST &&
-            !wait_bar(smem_u32(&empty[st]), ((i / NST) - 1) & 1, abort_flag, a.err, ERR_GEMM_EMPTY))
-          aborted = true;
-        if (!aborted) {
-          const uint32_t s0 = sbase + st * stage_bytes;
-          const int k0 = (t.kc0 + i) * KCH;
-          if (A_MN) {
-            // codec [g][k][m]: rows m .. m+3 at depth k0 + kk0 + 8u
-            const bool mok = a_row < t.Mv;
-            const float* src0 = a.Aw + ((int64_t)t.g * t.K + k0 + kk0) * t.Mv + a_row;
-#pragma unroll
-            for (int u = 0; u < PA; ++u) {
-              const int k = k0 + kk0 + 8 * (NPROD / 256) * u;
-              const bool ok = mok && k < t.K;
-              cp_async16(s0 + a_off0 + u * A_OFF_U, ok ? src0 + (int64_t)8 * (NPROD / 256) * u * t.Mv : a.Aw,
-                         ok ? 16u : 0u);
-            }
-          } else {
-            // writer codec E(n, k) at E + ob * e_o + n * e_n + od
-            const bool kok = kpos < t.K;
-            const float* src0 = sl.E + (int64_t)ob * sl.e_o + (int64_t)a_row * sl.e_n + od;
-#pragma unroll
-            for (int u = 0; u < PA; ++u) {
-              const bool ok = kok && a_row + 32 * (NPROD / 256) * u < t.Mv;
-              cp_async16(s0 + a_off0 + u * A_OFF_U, ok ? src0 + (int64_t)32 * (NPROD / 256) * u * sl.e_n : sl.E,
-                         ok ? 16u : 0u);
-            }
-          }
-          const bool kok = kpos < t.K;
-          int64_t koff;
-          if (KIND == KIND_WRITER) koff = (int64_t)ot * sl.x_o_t + (int64_t)oh * sl.x_o_h + od;
-          else koff = kpos;
-          const float* xbase = KIND == KIND_WRITER ? sl.X : a.X;
-          for (int jb = 0; jb < nb; ++jb) {
-            const uint32_t bt = s0 + a_part + jb * b_tile;
-#pragma unroll
-            for (int u = 0; u < PB; ++u) {
-              const bool ok = kok && t.n0 + r0 + 32 * (NPROD / 256) * u < t.Nv;
-              cp_async16(bt + b_off0 + u * B_OFF_U, ok ? xbase + jb * b_jb_stride + xrow[u] + koff : xbase,
-                         ok ? 16u : 0u);
-            }
-          }
-        }
-      }
-      cp_async_commit();
-      // advance this thread's k position by one chunk
-      kpos += KCH;
-      if (KIND == KIND_WRITER) {
-        od += KCH;
-        while (od >= sl.d_in) {
-          od -= sl.d_in;
-          ++ob;
-          if (++oh == sl.o_h) {
-            oh = 0;
-            ++ot;
-          }
-        }
-      }
-    };
+    // ---- converters: round each landed stage to tf32 in place ---------------
+    // (the hi and lo tiles share one layout, so pieces are plain 16-byte slots)
     auto convert = [&](uint32_t addr, uint32_t lo_addr) {
       const float4 v = lds4(addr);
       const uint32_t hx = to_tf32(v.x), hy = to_tf32(v.y), hz = to_tf32(v.z), hw = to_tf32(v.w);
@@ -324,33 +220,22 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const TcGemmArgs a) {
         sts4(lo_addr, to_tf32(v.x - __uint_as_float(hx)), to_tf32(v.y - __uint_as_float(hy)),
              to_tf32(v.z - __uint_as_float(hz)), to_tf32(v.w - __uint_as_float(hw)));
     };
-#pragma unroll 1
-    for (int i = 0; i < DEPTH; ++i) {
-      if (i < nchunks) issue(i);
-      else cp_async_commit();
-    }
+    const int b_pieces = nb * BN * 8;
 #pragma unroll 1
     for (int i = 0; i < nchunks; ++i) {
-      cp_async_wait<DEPTH - 1>();
-      if (aborted || *abort_flag) {
-        aborted = true;
-        break;
-      }
       const int st = i % NST;
+      if (!wait_bar(smem_u32(&loaded[st]), (i / NST) & 1, abort_flag, a.err, ERR_GEMM_LOAD)) break;
       const uint32_t s0 = sbase + st * stage_bytes;
 #pragma unroll
-      for (int u = 0; u < PA; ++u) convert(s0 + a_off0 + u * A_OFF_U, s0 + A_BYTES + a_off0 + u * A_OFF_U);
-      for (int jb = 0; jb < nb; ++jb) {
-        const uint32_t bt = s0 + a_part + jb * b_tile;
-#pragma unroll
-        for (int u = 0; u < PB; ++u) convert(bt + b_off0 + u * B_OFF_U, bt + nb * b_tile + b_off0 + u * B_OFF_U);
+      for (int u = 0; u < A_BYTES / 16 / NPROD; ++u) {
+        const uint32_t off = 16u * (tid + NPROD * u);
+        convert(s0 + off, s0 + A_BYTES + off);
       }
+      const uint32_t bt = s0 + a_part;
+      for (int p = tid; p < b_pieces; p += NPROD) convert(bt + 16u * p, bt + nb * b_tile + 16u * p);
       fence_proxy_async_smem();
       mbar_arrive(smem_u32(&full[st]));
-      if (i + DEPTH < nchunks) issue(i + DEPTH);
-      else cp_async_commit();
     }
-    cp_async_wait<0>();
 
     // ---- epilogue ------------------------------------------------------------
     const bool ok = wait_bar(smem_u32(done), 0, abort_flag, a.err, ERR_GEMM_DONE, false) && !*abort_flag;
@@ -503,6 +388,48 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const TcGemmArgs a) {
       }
     }
     tc_fence_before();
+  } else if (warp == TMA_WARP) {
+    // ---- tensor-map copies ------------------------------------------------------
+    if (lane == 0) {
+#pragma unroll 1
+      for (int i = 0; i < nchunks; ++i) {
+        const int st = i % NST;
+        if (i >= NST &&
+            !wait_bar(smem_u32(&empty[st]), ((i / NST) - 1) & 1, abort_flag, a.err, ERR_GEMM_EMPTY))
+          break;
+        const uint32_t s0 = sbase + st * stage_bytes;
+        const uint32_t bar = smem_u32(&loaded[st]);
+        mbar_arrive_tx(bar, (uint32_t)A_BYTES + nb * b_tile);
+        const int k0 = (t.kc0 + i) * KCH;
+        if (KIND == KIND_WRITER) {
+          // chunk k0 lies in one (outer block, feature) run: outer o, feature d
+          const int o = k0 / sl.d_in, d = k0 % sl.d_in;
+          int ai = 0, ta = 0, ha = 0, tx = 0, hx = 0;
+          if (a.w.mode == LLA_WRITE_HLA) {
+            ai = t.g;                       // E_main or E_1
+            ta = o;
+            tx = t.g == 0 ? 1 + o : 0;      // loops 2..T, or loop 1
+          } else if (a.w.mode == LLA_WRITE_PERHEAD) {
+            ai = t.g / a.w.H;               // K or V
+            ha = hx = t.g % a.w.H;
+            ta = tx = o;
+          } else {
+            ai = t.g;
+            ta = tx = o / a.w.H;
+            ha = hx = o % a.w.H;
+          }
+          tma_load_4d(s0, &maps.a[ai], bar, d, t.m0, ha, ta);
+          tma_load_4d(s0 + a_part, &maps.x[ai], bar, d, hx, tx, t.n0);
+        } else if (KIND == KIND_QMAP) {
+          tma_load_4d(s0, &maps.a[0], bar, 0, k0, t.m0 / 32, t.g);
+          tma_load_3d(s0 + a_part, &maps.x[0], bar, k0, t.g, t.n0);
+        } else {
+          tma_load_4d(s0, &maps.a[0], bar, 0, k0, t.m0 / 32, t.g);
+          for (int jb = 0; jb < nb; ++jb)
+            tma_load_4d(s0 + a_part + jb * b_tile, &maps.x[0], bar, k0, t.g, t.n0, jb);
+        }
+      }
+    }
   } else if (lane == 0) {
     // ---- MMA issue -------------------------------------------------------------
     const bool a_mn = KIND != KIND_WRITER;
@@ -544,20 +471,19 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const TcGemmArgs a) {
   }
 }
 
-template <int KIND, int BN, int PREC, int DEPTH>
-cudaError_t launch_one(TcGemmArgs a, int grid_y, int nb, size_t smem_budget, cudaStream_t st) {
+template <int KIND, int BN, int PREC>
+cudaError_t launch_one(const TcMaps& maps, TcGemmArgs a, int grid_y, int nb, size_t smem_budget, cudaStream_t st) {
   const int stage = (A_BYTES * (PREC == 3 ? 2 : 1)) + BN * 128 * nb * (PREC == 3 ? 2 : 1);
   const int wts = KIND == KIND_OMAP ? BN * (nb + a.Sw + 1) * 4 : 0;
-  // stages: at least DEPTH + 1, up to DEPTH + 3 (slack between the copies in
-  // flight and the stage the MMA is still reading) as the budget allows
-  const size_t fixed = 1024 + 16 + wts;
-  int nst = DEPTH + 1;
-  while (nst < DEPTH + 3 && fixed + (size_t)(nst + 1) * (stage + 16) + 8 <= smem_budget) ++nst;
+  // stages: 2 to 6, as many as the budget allows
+  const size_t fixed = 1024 + 16 + wts + 8;
+  int nst = 2;
+  while (nst < 6 && fixed + (size_t)(nst + 1) * (stage + 24) <= smem_budget) ++nst;
   a.nst = nst;
   // the output map's epilogue tiles (window term, partial maxima) reuse the stages
   if (KIND == KIND_OMAP && (size_t)BN * GM * 4 + (size_t)BN * (nb + a.Sw) * 8 > (size_t)nst * stage)
-    return cudaErrorInvalidConfiguration;
-  size_t smem = fixed + (size_t)nst * stage + 8 * (2 * nst + 1);
+    return cudaErrorNotSupported;
+  size_t smem = fixed + (size_t)nst * stage + 8 * (3 * nst + 1);
   // keep the CTAs an SM can hold (228 KB of shared memory, 1 KB reserved per
   // CTA) within its 512 TMEM columns, so that no allocation ever waits
   int ncols = 32;
@@ -565,30 +491,93 @@ cudaError_t launch_one(TcGemmArgs a, int grid_y, int nb, size_t smem_budget, cud
   const int max_ctas = 512 / ncols;
   const size_t floor_smem = (size_t)233472 / (max_ctas + 1) - 1024 + 16;
   if (smem < floor_smem) smem = floor_smem;
-  if (smem > (size_t)SMEM_MAX) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(tc_gemm<KIND, BN, PREC, DEPTH>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (smem > (size_t)SMEM_MAX) return cudaErrorNotSupported;
+  cudaError_t e = cudaFuncSetAttribute(tc_gemm<KIND, BN, PREC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.mtiles * a.ntiles, grid_y);
-  tc_gemm<KIND, BN, PREC, DEPTH><<<grid, NTHR, smem, st>>>(a);
+  tc_gemm<KIND, BN, PREC><<<grid, NTHR, smem, st>>>(maps, a);
   return cudaGetLastError();
 }
 
 int pick_bn(int n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : 256; }
 
-template <int KIND, int PREC, int DEPTH>
-cudaError_t launch_bn(TcGemmArgs a, int Nv, int grid_y, int nb, int bn_cap, size_t smem_budget, cudaStream_t st) {
+// Codec of the maps, [groups][K][Mtot] fp32, as an MN-major tf32 operand:
+// 4-D view (32 rows, k, 32-row atom, group), boxes of 32 x 32 x 4 atoms.
+bool map_codec_tmap(CUtensorMap* m, const float* W, int groups, int K, int Mtot) {
+  if (Mtot % 32 || K % 4) return false;
+  const cuuint64_t dims[4] = {32, (cuuint64_t)K, (cuuint64_t)(Mtot / 32), (cuuint64_t)groups};
+  const cuuint64_t strides[3] = {(cuuint64_t)Mtot * 4, 128, (cuuint64_t)K * Mtot * 4};
+  const cuuint32_t box[4] = {32, KCH, GM / 32, 1};
+  return tmap_f32(m, W, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
+}
+
+template <int KIND, int PREC>
+cudaError_t launch_bn(TcMaps& maps, TcGemmArgs a, int Nv, int grid_y, int nb, int bn_cap, size_t smem_budget,
+                      bool (*x_map)(TcMaps&, const TcGemmArgs&, int), cudaStream_t st) {
   const int bn = std::min(pick_bn(Nv), bn_cap);
   a.ntiles = (Nv + bn - 1) / bn;
+  if (!x_map(maps, a, bn)) return cudaErrorNotSupported;
   switch (bn) {
-    case 32: return launch_one<KIND, 32, PREC, DEPTH>(a, grid_y, nb, smem_budget, st);
-    case 64: return launch_one<KIND, 64, PREC, DEPTH>(a, grid_y, nb, smem_budget, st);
-    case 128: return launch_one<KIND, 128, PREC, DEPTH>(a, grid_y, nb, smem_budget, st);
-    default: return launch_one<KIND, 256, PREC, DEPTH>(a, grid_y, nb, smem_budget, st);
+    case 32: return launch_one<KIND, 32, PREC>(maps, a, grid_y, nb, smem_budget, st);
+    case 64: return launch_one<KIND, 64, PREC>(maps, a, grid_y, nb, smem_budget, st);
+    case 128: return launch_one<KIND, 128, PREC>(maps, a, grid_y, nb, smem_budget, st);
+    default: return launch_one<KIND, 256, PREC>(maps, a, grid_y, nb, smem_budget, st);
   }
 }
 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// q [B][rows][K] (batch stride xs_b): 3-D view (k, row, sequence), boxes of 32 x 1 x BN.
+bool qmap_x(TcMaps& maps, const TcGemmArgs& a, int bn) {
+  const cuuint64_t dims[3] = {(cuuint64_t)a.K, (cuuint64_t)a.rows, (cuuint64_t)a.B};
+  const cuuint64_t strides[2] = {(cuuint64_t)a.K * 4, (cuuint64_t)a.xs_b * 4};
+  const cuuint32_t box[3] = {KCH, 1, (cuuint32_t)bn};
+  return tmap_f32(&maps.x[0], a.X, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// split partials y~ [S][B][rows][K]: 4-D view (k, row, sequence, split).
+bool omap_x(TcMaps& maps, const TcGemmArgs& a, int bn) {
+  const cuuint64_t dims[4] = {(cuuint64_t)a.K, (cuuint64_t)a.rows, (cuuint64_t)a.B, (cuuint64_t)a.NB};
+  const cuuint64_t strides[3] = {(cuuint64_t)a.K * 4, (cuuint64_t)a.rows * a.K * 4,
+                                 (cuuint64_t)a.B * a.rows * a.K * 4};
+  const cuuint32_t box[4] = {KCH, 1, (cuuint32_t)bn, 1};
+  return tmap_f32(&maps.x[0], a.X, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Writer: codec E(n, k) and activations X(m, k) of both slices' operands as
+// 4-D views (feature, n, head, outer) and (feature, head, loop, token).
+bool writer_x(TcMaps& maps, const TcGemmArgs& a, int bn) {
+  const WriterArgs& w = a.w;
+  const int64_t mstride = w.n_tok == 1 ? w.xs_b : w.xs_n;
+  const cuuint32_t boxa[4] = {KCH, GM, 1, 1};
+  const cuuint32_t boxx[4] = {KCH, 1, 1, (cuuint32_t)bn};
+  if (w.mode == LLA_WRITE_HLA) {
+    const int N0 = w.r_k + w.r_v, N1 = 2 * w.r_1;
+    const cuuint64_t d0[4] = {(cuuint64_t)w.D, (cuuint64_t)N0, 1, (cuuint64_t)(w.T - 1)};
+    const cuuint64_t s0[3] = {(cuuint64_t)w.D * 4, (cuuint64_t)N0 * w.D * 4, (cuuint64_t)N0 * w.D * 4};
+    const cuuint64_t d1[4] = {(cuuint64_t)w.D, (cuuint64_t)N1, 1, 1};
+    const cuuint64_t s1[3] = {(cuuint64_t)w.D * 4, (cuuint64_t)N1 * w.D * 4, (cuuint64_t)N1 * w.D * 4};
+    const cuuint64_t dx[4] = {(cuuint64_t)w.D, 1, (cuuint64_t)w.T, (cuuint64_t)w.M};
+    const cuuint64_t sx[3] = {(cuuint64_t)w.xs_t * 4, (cuuint64_t)w.xs_t * 4, (cuuint64_t)mstride * 4};
+    return (w.T < 2 || tmap_f32(&maps.a[0], w.E_main, 4, d0, s0, boxa, CU_TENSOR_MAP_SWIZZLE_128B)) &&
+           tmap_f32(&maps.a[1], w.E_1, 4, d1, s1, boxa, CU_TENSOR_MAP_SWIZZLE_128B) &&
+           tmap_f32(&maps.x[0], w.x, 4, dx, sx, boxx, CU_TENSOR_MAP_SWIZZLE_128B) &&
+           tmap_f32(&maps.x[1], w.x, 4, dx, sx, boxx, CU_TENSOR_MAP_SWIZZLE_128B);
+  }
+  const float* E[2] = {w.E_K, w.E_V};
+  const float* X[2] = {w.x, w.xv};
+  const int r[2] = {w.r_k, w.r_v};
+  for (int p = 0; p < 2; ++p) {
+    const cuuint64_t da[4] = {(cuuint64_t)w.d_h, (cuuint64_t)r[p], (cuuint64_t)w.H, (cuuint64_t)w.T};
+    const cuuint64_t sa[3] = {(cuuint64_t)w.d_h * 4, (cuuint64_t)r[p] * w.d_h * 4, (cuuint64_t)w.H * r[p] * w.d_h * 4};
+    const cuuint64_t dx[4] = {(cuuint64_t)w.d_h, (cuuint64_t)w.H, (cuuint64_t)w.T, (cuuint64_t)w.M};
+    const cuuint64_t sx[3] = {(cuuint64_t)w.d_h * 4, (cuuint64_t)w.xs_t * 4, (cuuint64_t)mstride * 4};
+    if (!tmap_f32(&maps.a[p], E[p], 4, da, sa, boxa, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !tmap_f32(&maps.x[p], X[p], 4, dx, sx, boxx, CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+  }
+  return true;
+}
 
 }  // namespace
 
@@ -605,13 +594,16 @@ cudaError_t launch_query_map_tc(const MapArgs& g, int* err, cudaStream_t st) {
   a.Aw = g.W; a.X = g.X; a.xs_b = g.xs_b;
   a.rotate = g.rotate; a.pos = g.pos; a.d_h = g.d_h; a.base = g.base; a.qmul = g.qmul; a.qbf = g.qbf;
   a.err = err; a.NB = 1; a.S = 1;
-  return launch_bn<KIND_QMAP, 1, 2>(a, g.B, 64, 1, 128, SMEM_MAX / 2 - 1024, st);
+  TcMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if (!map_codec_tmap(&maps.a[0], g.W, g.rows, g.K, g.N)) return cudaErrorNotSupported;
+  return launch_bn<KIND_QMAP, 1>(maps, a, g.B, 64, 1, 128, SMEM_MAX / 2 - 1024, qmap_x, st);
 }
 
 // ------------------------------------------------------------ output map --
 bool output_map_tc_ok(const MapArgs& g) {
   // one TMEM accumulator per latent split: at most 8 splits of 32 columns
-  return al16(g.W) && g.N % 4 == 0 && g.N <= GM && g.K % 4 == 0 && g.S >= 1 && g.S <= 8 &&
+  return al16(g.W) && g.N % 32 == 0 && g.N <= GM && g.K % 4 == 0 && g.S >= 1 && g.S <= 8 &&
          g.Sw <= kMaxWindowChunks;
 }
 
@@ -625,18 +617,22 @@ cudaError_t launch_output_map_tc(const MapArgs& g, cudaStream_t st) {
   a.NB = g.S; a.S = 1;
   int bn_cap = 256;
   while (bn_cap > 32 && g.S * bn_cap > 256) bn_cap >>= 1;
-  return launch_bn<KIND_OMAP, 1, 3>(a, g.B, g.rows, g.S, bn_cap, SMEM_MAX, st);
+  TcMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if (!map_codec_tmap(&maps.a[0], g.W, g.rows, g.K, g.N)) return cudaErrorNotSupported;
+  return launch_bn<KIND_OMAP, 1>(maps, a, g.B, g.rows, g.S, bn_cap, SMEM_MAX, omap_x, st);
 }
 
 // ---------------------------------------------------------------- writer --
 bool writer_tc_ok(const WriterArgs& w) {
   if (!al16(w.x) || (w.xv && !al16(w.xv))) return false;
   if (w.xs_b % 4 || w.xs_n % 4 || w.xs_t % 4) return false;
+  if (w.n_tok > 1 && w.xs_b != (int64_t)w.n_tok * w.xs_n) return false;   // tokens must form one strided axis
   const float* es[4] = {w.E_main, w.E_1, w.E_K, w.E_V};
   for (const float* e : es)
     if (e && !al16(e)) return false;
-  if (w.mode == LLA_WRITE_HLA) return w.D % 4 == 0;
-  return w.d_h % 4 == 0;
+  if (w.mode == LLA_WRITE_HLA) return w.D % KCH == 0;
+  return w.d_h % KCH == 0;
 }
 
 int writer_tc_splits(const WriterArgs& w, int num_sms) {
@@ -657,7 +653,9 @@ cudaError_t launch_writer_tc(const WriterArgs& w, int* err, cudaStream_t st) {
   std::memset(&a, 0, sizeof(a));
   a.w = w; a.err = err; a.S = w.S; a.NB = 1;
   a.mtiles = (w.Nmax + GM - 1) / GM;
-  return launch_bn<KIND_WRITER, 3, 2>(a, w.M, w.Z * w.S, 1, 128, SMEM_MAX, st);
+  TcMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  return launch_bn<KIND_WRITER, 3>(maps, a, w.M, w.Z * w.S, 1, 128, SMEM_MAX, writer_x, st);
 }
 
 }  // namespace lla

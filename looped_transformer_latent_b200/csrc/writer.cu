@@ -167,17 +167,22 @@ cudaError_t launch_writer(const WriterArgs& a_in, cudaStream_t st) {
   a.err = reinterpret_cast<int*>(a.part + (size_t)a.Z * a.S * a.M * a.Nmax);
   cudaError_t e0 = cudaMemsetAsync(a.err, 0, sizeof(int), st);
   if (e0 != cudaSuccess) return e0;
+  bool simt = !a.use_tc;
   if (a.use_tc) {
     e0 = launch_writer_tc(a, a.err, st);
-  } else if (small_batch(a)) {
-    dim3 grid(ceil_div(a.Nmax, 128), ceil_div(a.M, 32), a.Z * a.S);
-    writer_gemm<32, 128><<<grid, WT, 0, st>>>(a);
-  } else {
-    dim3 grid(ceil_div(a.Nmax, 64), ceil_div(a.M, 64), a.Z * a.S);
-    writer_gemm<64, 64><<<grid, WT, 0, st>>>(a);
+    if (e0 == cudaErrorNotSupported) simt = true;   // no tensor-map view of these operands
   }
-  cudaError_t e = a.use_tc ? e0 : cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (simt) {
+    if (small_batch(a)) {
+      dim3 grid(ceil_div(a.Nmax, 128), ceil_div(a.M, 32), a.Z * a.S);
+      writer_gemm<32, 128><<<grid, WT, 0, st>>>(a);
+    } else {
+      dim3 grid(ceil_div(a.Nmax, 64), ceil_div(a.M, 64), a.Z * a.S);
+      writer_gemm<64, 64><<<grid, WT, 0, st>>>(a);
+    }
+    e0 = cudaGetLastError();
+  }
+  if (e0 != cudaSuccess) return e0;
   const int64_t total = (int64_t)a.Z * a.M * (a.Nmax / 2);
   int blocks = (int)((total + 255) / 256);
   if (blocks > 148 * 16) blocks = 148 * 16;
