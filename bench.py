@@ -650,20 +650,20 @@ def main():
                                "read after the last replay of the timed region"},
     }
     if cfg.kind == "lla":
-        # reconstruct-on-read is bound by the fp32 reconstruction arithmetic:
-        # per latent token, loop and head 2*2*d_h*r flops (k^ and v^) plus
-        # 2*2*d_h for the score and the weighted sum.  Peak: 148 SMs x 128
-        # fp32 lanes x 2 flops x the maximum SM clock.
+        # reconstruct-on-read rebuilds k^ and v^ for every latent token, loop
+        # and head on the tensor cores: 2*d_h*r flops each, plus 2*d_h for the
+        # score and 2*d_h for the weighted sum (algorithmic count: one product
+        # per term, rank and head dimension unpadded).  Peak: the measured dense
+        # bf16 rate of this machine's B200s.
         flops = cfg.B * cfg.T * cfg.H * step.n_lat * (4.0 * cfg.d_h * cfg.r_k + 4.0 * cfg.d_h)
         tf = flops / 1e12 / (mean_ms / 1e3) if mean_ms > 0 else 0.0
-        max_mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
-        alu_peak = 148 * 128 * 2 * max_mhz * 1e6 / 1e12
-        line["roofline"] = {"bound": "alu", "achieved": tf, "peak": alu_peak, "unit": "TFLOP/s",
-                            "frac": tf / alu_peak, "traffic": None,
-                            "kernel": "LLA reconstruct-on-read (recon_split_simt)",
-                            "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x max SM clock",
-                            "per_launch_ms": mean_ms, "flops_per_launch": flops,
-                            "latent_gbs": achieved, "launches_per_step": len(main_ix)}
+        line["roofline"] = {"bound": "tensor", "achieved": tf, "peak": tflops, "unit": "TFLOP/s",
+                            "frac": tf / tflops, "traffic": None,
+                            "kernel": "LLA reconstruct-on-read (recon_split_tc)",
+                            "peak_source": src + " (dense bf16)", "per_launch_ms": mean_ms,
+                            "flops_per_launch": flops, "latent_gbs": achieved,
+                            "launches_per_step": len(main_ix),
+                            "fp32_alu_equivalent_frac": tf / (148 * 128 * 2 * ((clocks or {}).get("sm_max_mhz") or 1965.0) * 1e6 / 1e12)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg)
     if rank == 0:

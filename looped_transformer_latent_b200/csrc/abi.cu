@@ -213,7 +213,15 @@ HlaPlan plan_lla(const lla_decode_params& p) {
   pl.n_lat = std::max(0, i - p.W);
   pl.win_start = pl.n_lat;
   pl.n_win = i - pl.win_start + 1;
-  if (pl.n_lat > 0) {
+  // tensor-core reconstruction: bf16 latents whose rows and strides allow a
+  // tensor-map view; one CTA per (loop, head, sequence) covers all tokens
+  pl.use_tc = pl.n_lat > 0 && p.lat_dtype == LLA_BF16 && p.r % 8 == 0 && p.d_h % 16 == 0 &&
+              (p.lat_stride_b * 2) % 16 == 0 && (p.lat_stride_h * 2) % 16 == 0;
+  pl.rows_pad = pl.rows;
+  if (pl.use_tc) {
+    pl.S = 1;
+    pl.tps = (pl.n_lat + 31) / 32 * 32;
+  } else if (pl.n_lat > 0) {
     const long ctas = (long)p.B * pl.rows;
     long S = (kTargetCtas + ctas - 1) / ctas;
     const long tiles = (pl.n_lat + 31) / 32;
@@ -413,7 +421,10 @@ int lla_decode_attn(const lla_decode_params* p, void* ws, size_t ws_bytes, lla_s
 
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
   if (e == cudaSuccess) e = mark(p->timing_events, 0, s);
-  if (e == cudaSuccess && a.n_lat > 0) e = launch_recon_split_simt(a, s);
+  if (e == cudaSuccess && a.n_lat > 0) {
+    e = (pl.use_tc && recon_tc_supported(a)) ? launch_recon_split_tc(a, err, s) : cudaErrorNotSupported;
+    if (e == cudaErrorNotSupported) e = launch_recon_split_simt(a, s);   // S = 1 covers every token as well
+  }
   if (e == cudaSuccess) e = mark(p->timing_events, 1, s);
   if (e == cudaSuccess) {
     WindowArgs wa;

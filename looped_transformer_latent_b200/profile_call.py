@@ -35,7 +35,7 @@ def main():
     ap.add_argument("--group", default="main", choices=["main", "loop1", "folded"])
     ap.add_argument("--batch", type=int, default=16)
     ap.add_argument("--iters", type=int, default=3)
-    ap.add_argument("--op", default="read", choices=["read", "write"])
+    ap.add_argument("--op", default="read", choices=["read", "write", "recon"])
     ap.add_argument("--context", type=int, default=0, help="override the context length N (read)")
     args = ap.parse_args()
     c = synth.CONFIGS[args.config]
@@ -45,6 +45,8 @@ def main():
     B = args.batch
     if args.op == "write":
         return write(L, c, B, args.iters, g, dev)
+    if args.op == "recon":
+        return recon(L, c, B, args.iters, g, dev, args.context or c.N)
     if args.group == "main":
         t0, nt, r_k, r_v, rotate = 1, c.T - 1, c.r_k, c.r_v, True
     elif args.group == "loop1":
@@ -68,6 +70,25 @@ def main():
     torch.cuda.synchronize()
     print(f"ok: {args.config} {args.group} B={B} N={N} rows={nt * H} r_k={r_k} r_v={r_v}, "
           f"latent bytes per call {lat[:, :max(0, N - 1 - W)].numel() * 2 / 1e6:.1f} MB")
+
+
+def recon(L, c, B, iters, g, dev, N):
+    """LLA per-head reconstruct-on-read: all T loops of every head, W = 0."""
+    r, T, H, d_h = c.r_k, c.T, c.H, c.d_h
+    cK = torch.randn(B, H, N, r, generator=g, device=dev).to(torch.bfloat16)
+    cV = torch.randn(B, H, N, r, generator=g, device=dev).to(torch.bfloat16)
+    UK = torch.randn(T, H, d_h, r, generator=g, device=dev) / math.sqrt(r)
+    UV = torch.randn(T, H, d_h, r, generator=g, device=dev) / math.sqrt(r)
+    q = torch.randn(B, T, H, d_h, generator=g, device=dev)
+    wk = torch.randn(B, T, 1, H, d_h, generator=g, device=dev).to(torch.bfloat16)
+    wv = torch.randn(B, T, 1, H, d_h, generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty(B, T, H, d_h, device=dev)
+    kw = dict(cK=cK, cV=cV, UK=UK, UV=UV, q=q, win_k=wk, win_v=wv, out=out, N=N, W=0, t0=0)
+    ws = torch.empty(max(256, L.lla_decode_workspace_bytes(**kw)), dtype=torch.uint8, device=dev)
+    for _ in range(iters):
+        L.lla_decode_attn(workspace=ws, **kw)
+    torch.cuda.synchronize()
+    print(f"ok: recon {c.name} B={B} N={N} H={H} T={T} r={r}")
 
 
 def write(L, c, B, iters, g, dev):
