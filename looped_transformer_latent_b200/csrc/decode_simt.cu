@@ -7,6 +7,7 @@
 
 #include "kernels.cuh"
 #include "tc_ptx.cuh"
+#include "tmap.cuh"
 
 namespace lla {
 namespace {
@@ -255,8 +256,15 @@ constexpr long long WB_WAIT = 1ll << 32;
 template <bool BF16>
 struct WbTraits { static constexpr int TS = BF16 ? 8 : 4; };
 
+// Ring tensor maps: 5-D view (feature, head, slot, loop, sequence), boxes of
+// d_h x 8 heads x TS slots -- one copy lands a stage's K (or V) block in the
+// [slot][head][feature] order the warps read.
+struct RingMaps {
+  CUtensorMap k, v;
+};
+
 template <bool BF16>
-__global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(WindowArgs w) {
+__global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(const __grid_constant__ RingMaps maps, WindowArgs w) {
   typedef WinTraits<BF16> Tr;
   constexpr int TS = WbTraits<BF16>::TS;
   constexpr int ES = BF16 ? 2 : 4;
@@ -282,13 +290,22 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(WindowArgs w) {
     const int st = i % WB_NST;
     const int jj = j0 + i * TS, nt = min(TS, j1 - jj);
     const uint32_t bar = ptx::smem_u32(&full[st]);
-    ptx::mbar_arrive_tx(bar, 2u * nt * tok_bytes);
     const uint32_t dk = ptx::smem_u32(wsm + st * 2 * half), dv = dk + half;
-    for (int u = 0; u < nt; ++u) {
-      const int slot = (w.win_start + jj + u) % w.Wcap;
-      const int64_t off = (((int64_t)t * w.Wcap + slot) * w.H + h0) * (int64_t)hbytes;
-      ptx::bulk_load(dk + u * WB_HEADS * hbytes, kbase + off, tok_bytes, bar);
-      ptx::bulk_load(dv + u * WB_HEADS * hbytes, vbase + off, tok_bytes, bar);
+    const int s0 = (w.win_start + jj) % w.Wcap;
+    if (s0 + nt <= w.Wcap) {
+      // the stage's slots are consecutive in the ring: one box each for K and V
+      ptx::mbar_arrive_tx(bar, 2u * half);
+      ptx::tma_load_5d(dk, &maps.k, bar, 0, h0, s0, t, b);
+      ptx::tma_load_5d(dv, &maps.v, bar, 0, h0, s0, t, b);
+    } else {
+      // the stage wraps around the ring's end: one copy per token
+      ptx::mbar_arrive_tx(bar, 2u * nt * tok_bytes);
+      for (int u = 0; u < nt; ++u) {
+        const int slot = (w.win_start + jj + u) % w.Wcap;
+        const int64_t off = (((int64_t)t * w.Wcap + slot) * w.H + h0) * (int64_t)hbytes;
+        ptx::bulk_load(dk + u * WB_HEADS * hbytes, kbase + off, tok_bytes, bar);
+        ptx::bulk_load(dv + u * WB_HEADS * hbytes, vbase + off, tok_bytes, bar);
+      }
     }
   };
   if (threadIdx.x == 0)
@@ -598,18 +615,34 @@ cudaError_t launch_window(const WindowArgs& w, cudaStream_t st) {
     const int ts = w.dtype == LLA_BF16 ? WbTraits<true>::TS : WbTraits<false>::TS;
     const size_t smem = (size_t)WB_NST * 2 * ts * WB_HEADS * w.d_h * es + 8 * WB_NST + 16;
     dim3 grid(w.Sw, nt * w.HG, w.B);
+    RingMaps maps;
+    TmapEncodeFn enc = tmap_encoder();
+    bool mapped = enc != nullptr;
+    const cuuint64_t dims[5] = {(cuuint64_t)w.d_h, (cuuint64_t)w.H, (cuuint64_t)w.Wcap, (cuuint64_t)(w.t0 + nt),
+                                (cuuint64_t)w.B};
+    const cuuint64_t hb = (cuuint64_t)w.d_h * es;
+    const cuuint64_t strides[4] = {hb, hb * w.H, hb * w.H * w.Wcap, (cuuint64_t)w.wins_b * es};
+    const cuuint32_t box[5] = {(cuuint32_t)w.d_h, WB_HEADS, (cuuint32_t)ts, 1, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    const CUtensorMapDataType dt = w.dtype == LLA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    for (int m = 0; m < 2 && mapped; ++m)
+      mapped = enc(m == 0 ? &maps.k : &maps.v, dt, 5, const_cast<void*>(m == 0 ? w.wk : w.wv), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (!mapped) goto register_kernel;   // no tensor-map view: same chunks on the register kernel
     cudaError_t e;
     if (w.dtype == LLA_BF16) {
       e = cudaFuncSetAttribute(window_bulk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      window_bulk<true><<<grid, 32 * WB_HEADS, smem, st>>>(w);
+      window_bulk<true><<<grid, 32 * WB_HEADS, smem, st>>>(maps, w);
     } else {
       e = cudaFuncSetAttribute(window_bulk<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      window_bulk<false><<<grid, 32 * WB_HEADS, smem, st>>>(w);
+      window_bulk<false><<<grid, 32 * WB_HEADS, smem, st>>>(maps, w);
     }
     return cudaGetLastError();
   }
+register_kernel:
   dim3 grid(w.Sw, nt, w.B);
   const bool small = w.cpt <= 8;
   if (w.dtype == LLA_BF16) {
