@@ -45,6 +45,9 @@ constexpr int MMA_WARP = NPROD / 32;    // warp 8: TMEM allocation, MMA issue
 constexpr int TMA_WARP = MMA_WARP + 1;  // warp 9: tensor-map copies
 constexpr int NTHR = NPROD + 64;
 constexpr int SMEM_MAX = 232448;
+constexpr int YW_SMEM_MAX = 65536;      // output map: window term of the column slice kept in smem up to this
+__host__ __device__ constexpr int align8(int x) { return (x + 7) & ~7; }
+__host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
 constexpr long long WAIT_CYCLES = 1ll << 32;
 
 enum : int { KIND_QMAP = 0, KIND_OMAP = 1, KIND_WRITER = 2 };
@@ -138,7 +141,10 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
 
   // ---- tile ------------------------------------------------------------
   Tile t;
-  const int mt = (int)blockIdx.x / a.ntiles, nti = (int)blockIdx.x % a.ntiles;
+  // output map: the k range of a tile is split over a cluster of ks CTAs
+  const int ks = KIND == KIND_OMAP ? (int)blockIdx.x % a.ks : 0;
+  const int tix = KIND == KIND_OMAP ? (int)blockIdx.x / a.ks : (int)blockIdx.x;
+  const int mt = tix / a.ntiles, nti = tix % a.ntiles;
   t.m0 = mt * GM;
   t.n0 = nti * BN;
   Slice sl;
@@ -159,8 +165,9 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
     t.Mv = a.Mtot;
     t.Nv = a.B;
     t.K = a.K;
-    t.kc0 = 0;
-    t.kc1 = (t.K + KCH - 1) / KCH;
+    const int nk = (t.K + KCH - 1) / KCH;
+    t.kc0 = KIND == KIND_OMAP ? (int)((int64_t)nk * ks / a.ks) : 0;
+    t.kc1 = KIND == KIND_OMAP ? (int)((int64_t)nk * (ks + 1) / a.ks) : nk;
     if (KIND == KIND_QMAP && t.g >= a.rows) {
       // rows of the bf16 query operand past the last query row are zero
       for (int idx = tid; idx < GM * BN; idx += NTHR) {
@@ -183,12 +190,58 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
   uint64_t* full = bars + NST;        // [NST] converted (all converter threads)
   uint64_t* empty = bars + 2 * NST;   // [NST] MMAs reading the stage completed
   uint64_t* done = bars + 3 * NST;
-  uint8_t* misc = reinterpret_cast<uint8_t*>(bars + 3 * NST + 1);
+  // misc region on a 16-byte boundary (the window-term tile is read as float4)
+  uint8_t* misc = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bars + 3 * NST + 1) + 15) & ~uintptr_t(15));
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
-  float* wts = reinterpret_cast<float*>(misc + 16);   // output map: [BN][NB + Sw + 1]
+  // output map: split weights, partial maxima and (for narrow column slices)
+  // the window term, in dedicated shared memory (filled while the stages stream)
+  const int ne = KIND == KIND_OMAP ? a.NB + a.Sw : 0;            // partials per sequence
+  const int cols_per = KIND == KIND_OMAP ? (BN + a.ks - 1) / a.ks : BN;
+  const int col_lo = min(BN, ks * cols_per), col_hi = min(BN, col_lo + cols_per);
+  const bool yw_smem = KIND == KIND_OMAP && cols_per * GM * 4 <= YW_SMEM_MAX;
+  float* wts = reinterpret_cast<float*>(misc + 16);                                       // [BN][ne + 1]
+  float2* mls = reinterpret_cast<float2*>(misc + 16 + align8(BN * (ne + 1) * 4));         // [BN][ne]
+  float* ywin_d = reinterpret_cast<float*>(misc + 16 + align8(BN * (ne + 1) * 4) + align16(BN * ne * 8));
 
-  if (tid == 0) {
+  // The copy thread initialises the barriers and issues the first stages at
+  // once, so their latency overlaps the TMEM allocation and the prologue.
+  auto issue_chunk = [&](int i) {
+    const int st = i % NST;
+    const uint32_t s0 = sbase + st * stage_bytes;
+    const uint32_t bar = smem_u32(&loaded[st]);
+    mbar_arrive_tx(bar, (uint32_t)A_BYTES + nb * b_tile);
+    const int k0 = (t.kc0 + i) * KCH;
+    if (KIND == KIND_WRITER) {
+      // chunk k0 lies in one (outer block, feature) run: outer o, feature d
+      const int o = k0 / sl.d_in, d = k0 % sl.d_in;
+      int ai = 0, ta = 0, ha = 0, tx = 0, hx = 0;
+      if (a.w.mode == LLA_WRITE_HLA) {
+        ai = t.g;                       // E_main or E_1
+        ta = o;
+        tx = t.g == 0 ? 1 + o : 0;      // loops 2..T, or loop 1
+      } else if (a.w.mode == LLA_WRITE_PERHEAD) {
+        ai = t.g / a.w.H;               // K or V
+        ha = hx = t.g % a.w.H;
+        ta = tx = o;
+      } else {
+        ai = t.g;
+        ta = tx = o / a.w.H;
+        ha = hx = o % a.w.H;
+      }
+      tma_load_4d(s0, &maps.a[ai], bar, d, t.m0, ha, ta);
+      tma_load_4d(s0 + a_part, &maps.x[ai], bar, d, hx, tx, t.n0);
+    } else if (KIND == KIND_QMAP) {
+      tma_load_4d(s0, &maps.a[0], bar, 0, k0, t.m0 / 32, t.g);
+      tma_load_3d(s0 + a_part, &maps.x[0], bar, k0, t.g, t.n0);
+    } else {
+      tma_load_4d(s0, &maps.a[0], bar, 0, k0, t.m0 / 32, t.g);
+      for (int jb = 0; jb < nb; ++jb)
+        tma_load_4d(s0 + a_part + jb * b_tile, &maps.x[0], bar, k0, t.g, t.n0, jb);
+    }
+  };
+  const int first = min(NST, nchunks);
+  if (warp == TMA_WARP && lane == 0) {
     for (int i = 0; i < NST; ++i) {
       mbar_init(smem_u32(&loaded[i]), 1);
       mbar_init(smem_u32(&full[i]), NPROD);
@@ -197,6 +250,9 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
     mbar_init(smem_u32(done), 1);
     *abort_flag = 0;
     fence_mbar_init();
+    prefetch_tmap(&maps.a[0]);
+    prefetch_tmap(&maps.x[0]);
+    for (int i = 0; i < first; ++i) issue_chunk(i);
   }
   uint32_t ncols = 32;
   while (ncols < (uint32_t)(nb * BN)) ncols <<= 1;
@@ -208,6 +264,9 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // output map with a cluster k-split: this CTA's weighted partial tile, in
+  // the stage memory (free once every MMA is done)
+  float* part_s = reinterpret_cast<float*>(base);                          // [BN][GM]
 
   if (warp < NPROD / 32) {
     // ---- converters: round each landed stage to tf32 in place ---------------
@@ -220,37 +279,13 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
         sts4(lo_addr, to_tf32(v.x - __uint_as_float(hx)), to_tf32(v.y - __uint_as_float(hy)),
              to_tf32(v.z - __uint_as_float(hz)), to_tf32(v.w - __uint_as_float(hw)));
     };
-    const int b_pieces = nb * BN * 8;
-#pragma unroll 1
-    for (int i = 0; i < nchunks; ++i) {
-      const int st = i % NST;
-      if (!wait_bar(smem_u32(&loaded[st]), (i / NST) & 1, abort_flag, a.err, ERR_GEMM_LOAD)) break;
-      const uint32_t s0 = sbase + st * stage_bytes;
-#pragma unroll
-      for (int u = 0; u < A_BYTES / 16 / NPROD; ++u) {
-        const uint32_t off = 16u * (tid + NPROD * u);
-        convert(s0 + off, s0 + A_BYTES + off);
-      }
-      const uint32_t bt = s0 + a_part;
-      for (int p = tid; p < b_pieces; p += NPROD) convert(bt + 16u * p, bt + nb * b_tile + 16u * p);
-      fence_proxy_async_smem();
-      mbar_arrive(smem_u32(&full[st]));
-    }
-
-    // ---- epilogue ------------------------------------------------------------
-    const bool ok = wait_bar(smem_u32(done), 0, abort_flag, a.err, ERR_GEMM_DONE, false) && !*abort_flag;
-    tc_fence_after();
-    // Output map, now that every MMA has completed and the stage memory is
-    // free: (1) gather the (max, sum) of every split and window partial of the
-    // tile's sequences with all producer threads; (2) one thread per sequence
-    // turns them into weights 2^(m - M) and 1 / l; (3) gather the window term
-    // sum_c w_c y_c of every (sequence, column) with coalesced loads.
-    float* ywin = reinterpret_cast<float*>(base);              // [BN][GM]
-    if (KIND == KIND_OMAP) {
-      const int ne = a.NB + a.Sw;                              // partials per sequence
+    if constexpr (KIND == KIND_OMAP) {
+      // while the first stages stream: (1) gather the (max, sum) of every split
+      // and window partial of the tile's sequences; (2) one thread per sequence
+      // turns them into weights 2^(m - M) and 1 / l; (3) for narrow column
+      // slices, the window term sum_c w_c y_c of this CTA's columns
       const int ld = ne + 1;
       const int64_t bstride = (int64_t)a.B * a.rows;
-      float2* mls = reinterpret_cast<float2*>(base + (size_t)BN * GM * 4);   // [BN][ne]
 #pragma unroll 4
       for (int idx = tid; idx < BN * ne; idx += NPROD) {
         const int bb = idx / ne, e = idx % ne;
@@ -278,47 +313,69 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
         w[ne] = t.n0 + bb < t.Nv ? 1.f / L : 0.f;
       }
       named_sync(1, NPROD);
-      // float4 groups of 4 columns; per pass each thread keeps 4 groups and
-      // loops over the window chunks outermost, so its loads of a chunk are
-      // independent and in flight together
-      constexpr int G4 = BN * GM / 4;                 // float4 groups in the tile
-      for (int base4 = 0; base4 < G4; base4 += 4 * NPROD) {
-        float4 acc4[4];
-        int64_t off4[4];
-        bool live[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int idx4 = base4 + u * NPROD + tid;
-          const int bb = idx4 / (GM / 4), mm = 4 * (idx4 % (GM / 4));
-          const int n = t.n0 + bb, m = t.m0 + mm;
-          live[u] = idx4 < G4 && n < t.Nv && m < t.Mv;
-          off4[u] = live[u] ? ((int64_t)n * a.rows + t.g) * a.Mtot + m : 0;
-          acc4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        for (int cw = 0; cw < a.Sw; ++cw) {
-          float4 v4[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            v4[u] = live[u] ? *reinterpret_cast<const float4*>(a.win_y + cw * bstride * a.Mtot + off4[u])
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      if (yw_smem) {
+        // float4 groups of 4 columns; per pass each thread keeps 4 groups and
+        // loops over the window chunks outermost, so its loads of a chunk are
+        // independent and in flight together
+        const int g4_hi = (col_hi - col_lo) * (GM / 4);
+        for (int base4 = 0; base4 < g4_hi; base4 += 4 * NPROD) {
+          float4 acc4[4];
+          int64_t off4[4];
+          bool live[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int idx4 = base4 + u * NPROD + tid;
-            const float w = live[u] ? wts[(idx4 / (GM / 4)) * ld + a.NB + cw] : 0.f;
-            acc4[u].x = fmaf(w, v4[u].x, acc4[u].x);
-            acc4[u].y = fmaf(w, v4[u].y, acc4[u].y);
-            acc4[u].z = fmaf(w, v4[u].z, acc4[u].z);
-            acc4[u].w = fmaf(w, v4[u].w, acc4[u].w);
+            const int bb = col_lo + idx4 / (GM / 4), mm = 4 * (idx4 % (GM / 4));
+            const int n = t.n0 + bb, m = t.m0 + mm;
+            live[u] = idx4 < g4_hi && n < t.Nv && m < t.Mv;
+            off4[u] = live[u] ? ((int64_t)n * a.rows + t.g) * a.Mtot + m : 0;
+            acc4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          for (int cw = 0; cw < a.Sw; ++cw) {
+            float4 v4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              v4[u] = live[u] ? *reinterpret_cast<const float4*>(a.win_y + cw * bstride * a.Mtot + off4[u])
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int idx4 = base4 + u * NPROD + tid;
+              const float w = live[u] ? wts[(col_lo + idx4 / (GM / 4)) * ld + a.NB + cw] : 0.f;
+              acc4[u].x = fmaf(w, v4[u].x, acc4[u].x);
+              acc4[u].y = fmaf(w, v4[u].y, acc4[u].y);
+              acc4[u].z = fmaf(w, v4[u].z, acc4[u].z);
+              acc4[u].w = fmaf(w, v4[u].w, acc4[u].w);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int idx4 = base4 + u * NPROD + tid;
+            if (idx4 < g4_hi) reinterpret_cast<float4*>(ywin_d)[idx4] = acc4[u];
           }
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int idx4 = base4 + u * NPROD + tid;
-          if (idx4 < G4) reinterpret_cast<float4*>(ywin)[idx4] = acc4[u];
-        }
+        named_sync(1, NPROD);
       }
-      named_sync(1, NPROD);
     }
+    const int b_pieces = nb * BN * 8;
+#pragma unroll 1
+    for (int i = 0; i < nchunks; ++i) {
+      const int st = i % NST;
+      if (!wait_bar(smem_u32(&loaded[st]), (i / NST) & 1, abort_flag, a.err, ERR_GEMM_LOAD)) break;
+      const uint32_t s0 = sbase + st * stage_bytes;
+#pragma unroll
+      for (int u = 0; u < A_BYTES / 16 / NPROD; ++u) {
+        const uint32_t off = 16u * (tid + NPROD * u);
+        convert(s0 + off, s0 + A_BYTES + off);
+      }
+      const uint32_t bt = s0 + a_part;
+      for (int p = tid; p < b_pieces; p += NPROD) convert(bt + 16u * p, bt + nb * b_tile + 16u * p);
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&full[st]));
+    }
+
+    // ---- epilogue ------------------------------------------------------------
+    const bool ok = wait_bar(smem_u32(done), 0, abort_flag, a.err, ERR_GEMM_DONE, false) && !*abort_flag;
+    tc_fence_after();
     // warps w and w + 4 share TMEM lanes 32 (w & 3) .. +31 and split the columns
     const int quarter = warp & 3, half = warp >> 2;
     const int m = t.m0 + 32 * quarter + lane;   // this thread's TMEM lane = codec row
@@ -331,7 +388,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
     for (int c = half * (BN / 32); c < (half + 1) * (BN / 32); ++c) {
       float v[16];
       if (KIND == KIND_OMAP) {
-        const int ld = a.NB + a.Sw + 1;
+        const int ld = ne + 1;
         float acc[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc[i] = 0.f;
@@ -370,13 +427,38 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
           }
         }
       } else if (KIND == KIND_OMAP) {
-        const int ld = a.NB + a.Sw + 1;
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-          const int bb = 16 * c + i, n = t.n0 + bb;
-          if (m >= t.Mv || n >= t.Nv) continue;
-          const float y = v[i] + ywin[bb * GM + (m - t.m0)];
-          a.out[(int64_t)n * a.outs_b + (int64_t)t.g * a.Mtot + m] = bad ? NAN : y * wts[bb * ld + a.NB + a.Sw];
+        if (a.ks > 1) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) part_s[(16 * c + i) * GM + (m - t.m0)] = v[i];
+        } else {
+          const int ld = ne + 1;
+          const int64_t bstride = (int64_t)a.B * a.rows;
+          float yw[16];
+          if (yw_smem) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) yw[i] = ywin_d[(16 * c + i) * GM + (m - t.m0)];
+          } else {
+            // window term from global memory: the 16 columns' loads per chunk together
+#pragma unroll
+            for (int i = 0; i < 16; ++i) yw[i] = 0.f;
+            for (int cw = 0; cw < a.Sw; ++cw) {
+              float wv[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int n = t.n0 + 16 * c + i;
+                wv[i] = (m < t.Mv && n < t.Nv)
+                            ? a.win_y[(cw * bstride + (int64_t)n * a.rows + t.g) * a.Mtot + m] : 0.f;
+              }
+#pragma unroll
+              for (int i = 0; i < 16; ++i) yw[i] = fmaf(wts[(16 * c + i) * ld + a.NB + cw], wv[i], yw[i]);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int bb = 16 * c + i, n = t.n0 + bb;
+            if (m < t.Mv && n < t.Nv)
+              a.out[(int64_t)n * a.outs_b + (int64_t)t.g * a.Mtot + m] = bad ? NAN : (v[i] + yw[i]) * wts[bb * ld + ne];
+          }
         }
       } else {
         float* P = a.w.part + ((int64_t)(t.g * a.S + t.split) * a.w.M) * a.w.Nmax;
@@ -391,43 +473,18 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
   } else if (warp == TMA_WARP) {
     // ---- tensor-map copies ------------------------------------------------------
     if (lane == 0) {
+      int issued = first;
 #pragma unroll 1
-      for (int i = 0; i < nchunks; ++i) {
+      for (int i = first; i < nchunks; ++i) {
         const int st = i % NST;
-        if (i >= NST &&
-            !wait_bar(smem_u32(&empty[st]), ((i / NST) - 1) & 1, abort_flag, a.err, ERR_GEMM_EMPTY))
-          break;
-        const uint32_t s0 = sbase + st * stage_bytes;
-        const uint32_t bar = smem_u32(&loaded[st]);
-        mbar_arrive_tx(bar, (uint32_t)A_BYTES + nb * b_tile);
-        const int k0 = (t.kc0 + i) * KCH;
-        if (KIND == KIND_WRITER) {
-          // chunk k0 lies in one (outer block, feature) run: outer o, feature d
-          const int o = k0 / sl.d_in, d = k0 % sl.d_in;
-          int ai = 0, ta = 0, ha = 0, tx = 0, hx = 0;
-          if (a.w.mode == LLA_WRITE_HLA) {
-            ai = t.g;                       // E_main or E_1
-            ta = o;
-            tx = t.g == 0 ? 1 + o : 0;      // loops 2..T, or loop 1
-          } else if (a.w.mode == LLA_WRITE_PERHEAD) {
-            ai = t.g / a.w.H;               // K or V
-            ha = hx = t.g % a.w.H;
-            ta = tx = o;
-          } else {
-            ai = t.g;
-            ta = tx = o / a.w.H;
-            ha = hx = o % a.w.H;
-          }
-          tma_load_4d(s0, &maps.a[ai], bar, d, t.m0, ha, ta);
-          tma_load_4d(s0 + a_part, &maps.x[ai], bar, d, hx, tx, t.n0);
-        } else if (KIND == KIND_QMAP) {
-          tma_load_4d(s0, &maps.a[0], bar, 0, k0, t.m0 / 32, t.g);
-          tma_load_3d(s0 + a_part, &maps.x[0], bar, k0, t.g, t.n0);
-        } else {
-          tma_load_4d(s0, &maps.a[0], bar, 0, k0, t.m0 / 32, t.g);
-          for (int jb = 0; jb < nb; ++jb)
-            tma_load_4d(s0 + a_part + jb * b_tile, &maps.x[0], bar, k0, t.g, t.n0, jb);
-        }
+        if (!wait_bar(smem_u32(&empty[st]), ((i / NST) - 1) & 1, abort_flag, a.err, ERR_GEMM_EMPTY)) break;
+        issue_chunk(i);
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        // leave no copy in flight: wait (bounded) for the stages issued last
+        for (int i = max(0, issued - NST); i < issued; ++i)
+          wait_bar(smem_u32(&loaded[i % NST]), (i / NST) & 1, abort_flag, nullptr, 0, false);
       }
     }
   } else if (lane == 0) {
@@ -464,6 +521,27 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
     }
     mma_commit(smem_u32(done));
   }
+  if (KIND == KIND_OMAP && a.ks > 1) {
+    // every CTA's partial tile is complete: finish this CTA's columns from the
+    // partials of all ks CTAs (distributed shared memory), in rank order
+    __syncwarp();
+    cluster_sync_all();
+    if (warp < NPROD / 32) {
+      const int ld = ne + 1;
+      const bool bad = *abort_flag || (a.err && *a.err);
+      const uint32_t ps_addr = smem_u32(part_s);
+      for (int idx = col_lo * GM + tid; idx < col_hi * GM; idx += NPROD) {
+        const int bb = idx / GM, mm = idx % GM;
+        const int n = t.n0 + bb, m = t.m0 + mm;
+        float y = ywin_d[idx - col_lo * GM];
+        for (int rk = 0; rk < a.ks; ++rk) y += ld_shared_cluster(mapa_shared(ps_addr + 4u * idx, (uint32_t)rk));
+        if (m < t.Mv && n < t.Nv)
+          a.out[(int64_t)n * a.outs_b + (int64_t)t.g * a.Mtot + m] = bad ? NAN : y * wts[bb * ld + ne];
+      }
+    }
+    // no CTA leaves while a neighbour may still read its partial tile
+    cluster_sync_all();
+  }
   __syncthreads();
   if (warp == MMA_WARP) {
     tc_fence_after();
@@ -474,15 +552,21 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
 template <int KIND, int BN, int PREC>
 cudaError_t launch_one(const TcMaps& maps, TcGemmArgs a, int grid_y, int nb, size_t smem_budget, cudaStream_t st) {
   const int stage = (A_BYTES * (PREC == 3 ? 2 : 1)) + BN * 128 * nb * (PREC == 3 ? 2 : 1);
-  const int wts = KIND == KIND_OMAP ? BN * (nb + a.Sw + 1) * 4 : 0;
-  // stages: 2 to 6, as many as the budget allows
-  const size_t fixed = 1024 + 16 + wts + 8;
+  // output map: weights, partial maxima and the window term of the column slice
+  int misc = 0;
+  if (KIND == KIND_OMAP) {
+    const int ne = nb + a.Sw, cols_per = (BN + a.ks - 1) / a.ks;
+    misc = align8(BN * (ne + 1) * 4) + align16(BN * ne * 8) + (cols_per * GM * 4 <= YW_SMEM_MAX ? cols_per * GM * 4 : 0);
+  }
+  // stages: 2 to 6, as many as the budget allows (16 bytes for aligning the misc region)
+  const size_t fixed = 1024 + 16 + 16 + misc + 8;
   int nst = 2;
   while (nst < 6 && fixed + (size_t)(nst + 1) * (stage + 24) <= smem_budget) ++nst;
   a.nst = nst;
-  // the output map's epilogue tiles (window term, partial maxima) reuse the stages
-  if (KIND == KIND_OMAP && (size_t)BN * GM * 4 + (size_t)BN * (nb + a.Sw) * 8 > (size_t)nst * stage)
-    return cudaErrorNotSupported;
+  // with a cluster k-split, the partial tile reuses the stages
+  if (KIND == KIND_OMAP && a.ks > 1 && (size_t)BN * GM * 4 > (size_t)nst * stage) return cudaErrorNotSupported;
+  // a cluster k-split needs the window term of its slice in shared memory
+  if (KIND == KIND_OMAP && a.ks > 1 && ((BN + a.ks - 1) / a.ks) * GM * 4 > YW_SMEM_MAX) return cudaErrorNotSupported;
   size_t smem = fixed + (size_t)nst * stage + 8 * (3 * nst + 1);
   // keep the CTAs an SM can hold (228 KB of shared memory, 1 KB reserved per
   // CTA) within its 512 TMEM columns, so that no allocation ever waits
@@ -494,7 +578,24 @@ cudaError_t launch_one(const TcMaps& maps, TcGemmArgs a, int grid_y, int nb, siz
   if (smem > (size_t)SMEM_MAX) return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(tc_gemm<KIND, BN, PREC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.mtiles * a.ntiles, grid_y);
+  const int ksplit = KIND == KIND_OMAP ? a.ks : 1;
+  dim3 grid(a.mtiles * a.ntiles * ksplit, grid_y);
+  if (ksplit > 1) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(NTHR);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = ksplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, tc_gemm<KIND, BN, PREC>, maps, a);
+  }
   tc_gemm<KIND, BN, PREC><<<grid, NTHR, smem, st>>>(maps, a);
   return cudaGetLastError();
 }
@@ -593,7 +694,7 @@ cudaError_t launch_query_map_tc(const MapArgs& g, int* err, cudaStream_t st) {
   a.B = g.B; a.rows = g.rows; a.Mtot = g.N; a.K = g.K; a.mtiles = (g.N + GM - 1) / GM;
   a.Aw = g.W; a.X = g.X; a.xs_b = g.xs_b;
   a.rotate = g.rotate; a.pos = g.pos; a.d_h = g.d_h; a.base = g.base; a.qmul = g.qmul; a.qbf = g.qbf;
-  a.err = err; a.NB = 1; a.S = 1;
+  a.err = err; a.NB = 1; a.S = 1; a.ks = 1;
   TcMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   if (!map_codec_tmap(&maps.a[0], g.W, g.rows, g.K, g.N)) return cudaErrorNotSupported;
@@ -615,8 +716,15 @@ cudaError_t launch_output_map_tc(const MapArgs& g, cudaStream_t st) {
   a.part_ml = g.part_ml; a.win_ml = g.win_ml; a.win_y = g.win_y; a.Sw = g.Sw;
   a.out = g.out; a.outs_b = g.outs_b; a.err = const_cast<int*>(g.err);
   a.NB = g.S; a.S = 1;
-  int bn_cap = 256;
+  int bn_cap = 128;
   while (bn_cap > 32 && g.S * bn_cap > 256) bn_cap >>= 1;
+  // k-splits over a cluster so that small batches still fill the SMs
+  const int bn = std::min(pick_bn(g.B), bn_cap);
+  const int tiles = g.rows * ((g.B + bn - 1) / bn);
+  const int nk = (g.K + KCH - 1) / KCH;
+  // one CTA per SM (registers), and clusters do not tile every GPC's SMs:
+  // keep the whole grid to 128 CTAs so that it starts in one wave
+  a.ks = std::max(1, std::min(std::min(4, nk), 128 / std::max(tiles, 1)));
   TcMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   if (!map_codec_tmap(&maps.a[0], g.W, g.rows, g.K, g.N)) return cudaErrorNotSupported;
@@ -651,7 +759,7 @@ int writer_tc_splits(const WriterArgs& w, int num_sms) {
 cudaError_t launch_writer_tc(const WriterArgs& w, int* err, cudaStream_t st) {
   TcGemmArgs a;
   std::memset(&a, 0, sizeof(a));
-  a.w = w; a.err = err; a.S = w.S; a.NB = 1;
+  a.w = w; a.err = err; a.S = w.S; a.NB = 1; a.ks = 1;
   a.mtiles = (w.Nmax + GM - 1) / GM;
   TcMaps maps;
   std::memset(&maps, 0, sizeof(maps));

@@ -145,6 +145,7 @@ cudaError_t launch_output_map(const MapArgs& g, cudaStream_t st);
 struct TcGemmArgs {
   int B, rows, Mtot, K, mtiles, ntiles, S, NB, Sw;
   int nst;                 // shared-memory stages (set by the launcher)
+  int ks;                  // output map: k-splits over a cluster of ks CTAs (1: none)
   const float *Aw, *X;     // codec [group][K][Mtot]; activations (per kind)
   int64_t xs_b;
   int rotate, pos, d_h;    // query map epilogue
