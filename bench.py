@@ -473,7 +473,7 @@ def run_reference(args, cfg):
 # from ncu captures (profiles/absorb_split_tc_*.md), keyed by the sha256 prefix
 # of the kernel source it was taken on and the latent row width in bytes: a
 # changed kernel, or a row width never captured, reports no traffic.
-TC_TRAFFIC_PER_TOKEN = {("5163ad08b2a9e31d", 2048): 2122.7}
+TC_TRAFFIC_PER_TOKEN = {("5163ad08b2a9e31d", 2048): 2122.7, ("5163ad08b2a9e31d", 2304): 2408.5}
 
 
 def tc_traffic_per_token(row_bytes):

@@ -113,6 +113,8 @@ __global__ void __launch_bounds__(256) absorb_split_simt(AbsorbArgs a) {
   }
 }
 
+__device__ __forceinline__ bool warp0_of(unsigned tid) { return tid < 32; }
+
 // --------------------------------------------------------------- window --
 // Exact attention over the window ring (eq. 4, second term) as partial
 // softmax states.  One CTA per (token chunk, loop, sequence) covers every
@@ -160,11 +162,19 @@ __global__ void __launch_bounds__(256, MINB) window_part(WindowArgs w) {
   const int d0 = 4 * lane;
   const bool dv = d0 < w.d_h;
   const int j0 = chunk * w.cpt, j1 = min(w.n_win, j0 + w.cpt);
-  // the lane's two pairs (2 lane, 2 lane + 1) share their angles across heads
+  // the pairs' angles are the same for every head: warp 0 computes them once
+  __shared__ float2 rot[64];
+  if (w.rotate && warp0_of(threadIdx.x))
+    for (int p = threadIdx.x; p < w.d_h / 2; p += 32) {
+      float c, sn;
+      rope_cs(p, w.d_h, w.d_h, w.base, (double)w.pos, &c, &sn);
+      rot[p] = make_float2(c, sn);
+    }
+  __syncthreads();
   float c0 = 1.f, s0 = 0.f, c1 = 1.f, s1 = 0.f;
   if (w.rotate && dv) {
-    rope_cs(2 * lane, w.d_h, w.d_h, w.base, (double)w.pos, &c0, &s0);
-    rope_cs(2 * lane + 1, w.d_h, w.d_h, w.base, (double)w.pos, &c1, &s1);
+    c0 = rot[2 * lane].x; s0 = rot[2 * lane].y;
+    c1 = rot[2 * lane + 1].x; s1 = rot[2 * lane + 1].y;
   }
   const int64_t seq = (int64_t)b * w.wins_b;
   for (int h = warp; h < w.H; h += 8) {
@@ -279,6 +289,15 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(const __grid_consta
   uint64_t* full = reinterpret_cast<uint64_t*>(wsm + WB_NST * 2 * half);
   const int j0 = chunk * w.cpt, j1 = min(w.n_win, j0 + w.cpt);
   const int nsub = (j1 - j0 + TS - 1) / TS;
+  // rotation of the query (R_pos in head space): the angles of the d_h / 2
+  // pairs are the same for every head, so warp 0 computes them once
+  __shared__ float2 rot[64];
+  if (w.rotate && warp0_of(threadIdx.x))
+    for (int p = threadIdx.x; p < w.d_h / 2; p += 32) {
+      float c, sn;
+      rope_cs(p, w.d_h, w.d_h, w.base, (double)w.pos, &c, &sn);
+      rot[p] = make_float2(c, sn);
+    }
   if (threadIdx.x == 0) {
     for (int i = 0; i < WB_NST; ++i) ptx::mbar_init(ptx::smem_u32(&full[i]), 1);
     ptx::fence_mbar_init();
@@ -316,8 +335,8 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(const __grid_consta
   const int row = tt * w.H + h0 + warp;
   float c0 = 1.f, s0 = 0.f, c1 = 1.f, s1 = 0.f;
   if (w.rotate && dv) {
-    rope_cs(2 * lane, w.d_h, w.d_h, w.base, (double)w.pos, &c0, &s0);
-    rope_cs(2 * lane + 1, w.d_h, w.d_h, w.base, (double)w.pos, &c1, &s1);
+    c0 = rot[2 * lane].x; s0 = rot[2 * lane].y;
+    c1 = rot[2 * lane + 1].x; s1 = rot[2 * lane + 1].y;
   }
   float qv[4] = {0.f, 0.f, 0.f, 0.f}, acc[4] = {0.f, 0.f, 0.f, 0.f};
   if (dv) {
