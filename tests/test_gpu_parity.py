@@ -198,10 +198,11 @@ def test_writer_hla_layout_bit_exact(cuda_device, dtype):
     assert torch.equal(lat1.cpu(), exp1.to(dtype))
 
 
+@pytest.mark.parametrize("d_h", [16, 32])     # 16: SIMT writer; 32: tensor-core writer (tensor-map view)
 @pytest.mark.parametrize("mode", [L.LLA_WRITE_PERHEAD, L.LLA_WRITE_FOLDED])
-def test_writer_lla_layout_bit_exact(cuda_device, mode):
-    g = _gen(4 + mode)
-    B, n, pos0, Ncap, T, H, d_h = 2, 5, 3, 12, 3, 3, 16
+def test_writer_lla_layout_bit_exact(cuda_device, mode, d_h):
+    g = _gen(4 + mode + d_h)
+    B, n, pos0, Ncap, T, H = 2, 5, 3, 12, 3, 3
     r = 16 if mode == L.LLA_WRITE_PERHEAD else 24
     rV = r if mode == L.LLA_WRITE_PERHEAD else 40
     k = _int_tensor(g, (B, n, T, H, d_h), -2, 2)
@@ -283,6 +284,7 @@ LLA_CASES = [
     (2, 2, 96, 96, 8, 2, 3, 77, 5, 6),
     (1, 1, 64, 64, 1, 0, 1, 1, 0, 1),        # N = 1
     (3, 2, 64, 32, 2, 0, 2, 129, 3, 4),      # r < d_h, ragged tile
+    (1, 2, 128, 128, 2, 0, 2, 300, 2, 3),    # largest tensor-core layout (d_h = r = 128), ragged tile
 ]
 
 
