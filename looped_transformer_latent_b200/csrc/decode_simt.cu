@@ -4,6 +4,7 @@
 // B_t^T map back to head space.  Scores are kept in base-2 units: every query
 // is pre-multiplied by scale * log2(e) so the softmax uses exp2.
 #include <algorithm>
+#include <cmath>
 
 #include "kernels.cuh"
 #include "tc_ptx.cuh"
@@ -113,8 +114,6 @@ __global__ void __launch_bounds__(256) absorb_split_simt(AbsorbArgs a) {
   }
 }
 
-__device__ __forceinline__ bool warp0_of(unsigned tid) { return tid < 32; }
-
 // --------------------------------------------------------------- window --
 // Exact attention over the window ring (eq. 4, second term) as partial
 // softmax states.  One CTA per (token chunk, loop, sequence) covers every
@@ -162,19 +161,11 @@ __global__ void __launch_bounds__(256, MINB) window_part(WindowArgs w) {
   const int d0 = 4 * lane;
   const bool dv = d0 < w.d_h;
   const int j0 = chunk * w.cpt, j1 = min(w.n_win, j0 + w.cpt);
-  // the pairs' angles are the same for every head: warp 0 computes them once
-  __shared__ float2 rot[64];
-  if (w.rotate && warp0_of(threadIdx.x))
-    for (int p = threadIdx.x; p < w.d_h / 2; p += 32) {
-      float c, sn;
-      rope_cs(p, w.d_h, w.d_h, w.base, (double)w.pos, &c, &sn);
-      rot[p] = make_float2(c, sn);
-    }
-  __syncthreads();
+  // the pairs' angles are the same for every head (computed once per call)
   float c0 = 1.f, s0 = 0.f, c1 = 1.f, s1 = 0.f;
   if (w.rotate && dv) {
-    c0 = rot[2 * lane].x; s0 = rot[2 * lane].y;
-    c1 = rot[2 * lane + 1].x; s1 = rot[2 * lane + 1].y;
+    c0 = w.rot[2 * lane].x; s0 = w.rot[2 * lane].y;
+    c1 = w.rot[2 * lane + 1].x; s1 = w.rot[2 * lane + 1].y;
   }
   const int64_t seq = (int64_t)b * w.wins_b;
   for (int h = warp; h < w.H; h += 8) {
@@ -289,20 +280,9 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(const __grid_consta
   uint64_t* full = reinterpret_cast<uint64_t*>(wsm + WB_NST * 2 * half);
   const int j0 = chunk * w.cpt, j1 = min(w.n_win, j0 + w.cpt);
   const int nsub = (j1 - j0 + TS - 1) / TS;
-  // rotation of the query (R_pos in head space): the angles of the d_h / 2
-  // pairs are the same for every head, so warp 0 computes them once
-  __shared__ float2 rot[64];
-  if (w.rotate && warp0_of(threadIdx.x))
-    for (int p = threadIdx.x; p < w.d_h / 2; p += 32) {
-      float c, sn;
-      rope_cs(p, w.d_h, w.d_h, w.base, (double)w.pos, &c, &sn);
-      rot[p] = make_float2(c, sn);
-    }
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < WB_NST; ++i) ptx::mbar_init(ptx::smem_u32(&full[i]), 1);
-    ptx::fence_mbar_init();
-  }
-  __syncthreads();
+  // the copy thread (warp 1, lane 0) sets up the barriers and issues the
+  // first stages before the block barrier
+  const bool copier = threadIdx.x == 32;
   const char* kbase = reinterpret_cast<const char*>(w.wk) + ((int64_t)b * w.wins_b) * ES;
   const char* vbase = reinterpret_cast<const char*>(w.wv) + ((int64_t)b * w.wins_b) * ES;
   auto issue = [&](int i) {        // sub-chunk i into stage i % WB_NST (thread 0)
@@ -327,16 +307,20 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(const __grid_consta
       }
     }
   };
-  if (threadIdx.x == 0)
+  if (copier) {
+    for (int i = 0; i < WB_NST; ++i) ptx::mbar_init(ptx::smem_u32(&full[i]), 1);
+    ptx::fence_mbar_init();
     for (int i = 0; i < WB_NST && i < nsub; ++i) issue(i);
+  }
+  __syncthreads();
 
   const int d0 = 4 * lane;
   const bool dv = warp < nh && d0 < w.d_h;
   const int row = tt * w.H + h0 + warp;
   float c0 = 1.f, s0 = 0.f, c1 = 1.f, s1 = 0.f;
   if (w.rotate && dv) {
-    c0 = rot[2 * lane].x; s0 = rot[2 * lane].y;
-    c1 = rot[2 * lane + 1].x; s1 = rot[2 * lane + 1].y;
+    c0 = w.rot[2 * lane].x; s0 = w.rot[2 * lane].y;
+    c1 = w.rot[2 * lane + 1].x; s1 = w.rot[2 * lane + 1].y;
   }
   float qv[4] = {0.f, 0.f, 0.f, 0.f}, acc[4] = {0.f, 0.f, 0.f, 0.f};
   if (dv) {
@@ -409,10 +393,10 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(const __grid_consta
     }
     m = mn;
     __syncthreads();   // every warp is done with this stage
-    if (threadIdx.x == 0 && i + WB_NST < nsub) issue(i + WB_NST);
+    if (copier && i + WB_NST < nsub) issue(i + WB_NST);
   }
   if (failed_at >= 0) {
-    if (threadIdx.x == 0) {
+    if (copier) {
       if (w.err) atomicExch(w.err, ERR_WINDOW_TIMEOUT);
       // leave no copy in flight: wait (bounded) for the stages still owed
       for (int i = failed_at; i < nsub && i < failed_at + WB_NST; ++i) {
@@ -626,8 +610,17 @@ int window_chunks(int B, int nt, int H, int n_win, int dtype, int d_h, int num_s
   return (n_win + c - 1) / c;
 }
 
-cudaError_t launch_window(const WindowArgs& w, cudaStream_t st) {
-  if (w.n_win <= 0 || w.B == 0) return cudaSuccess;
+cudaError_t launch_window(const WindowArgs& w_in, cudaStream_t st) {
+  if (w_in.n_win <= 0 || w_in.B == 0) return cudaSuccess;
+  WindowArgs w = w_in;
+  // R_pos of the query in head space: pair p at angle pos * base^(-2p / d_h)
+  for (int p = 0; p < 64; ++p) {
+    w.rot[p] = make_float2(1.f, 0.f);
+    if (w.rotate && p < w.d_h / 2) {
+      const double ang = (double)w.pos * std::pow(w.base, -2.0 * (double)p / (double)w.d_h);
+      w.rot[p] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+    }
+  }
   const int nt = w.rows / w.H;
   if (w.HG > 0) {
     const int es = w.dtype == LLA_BF16 ? 2 : 4;

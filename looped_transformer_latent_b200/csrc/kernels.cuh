@@ -100,6 +100,7 @@ struct WindowArgs {
   float qmul;
   int rotate, pos;
   double base;
+  float2 rot[64];          // cos, sin of pair p at pos (set by launch_window when rotate)
   float *win_ml, *win_y;   // [Sw][B][rows][2], [Sw][B][rows][d_h]
   int* err;                // optional: set to ERR_WINDOW_TIMEOUT if a copy never lands
 };
