@@ -33,7 +33,18 @@
  *             launched and outputs are untouched.  LLA_ERR_CUDA reports a
  *             failed launch (cudaGetLastError) or device query.  Errors raised
  *             by kernels already running surface on the caller's next CUDA
- *             synchronisation, as usual.  No call aborts or traps.
+ *             synchronisation, as usual.  No call aborts or traps.  Every wait
+ *             inside the kernels (copy completion, tensor-core completion) is
+ *             bounded at about two seconds; a kernel that gives up records the
+ *             reason in the workspace and the call's outputs are written as NaN
+ *             (its status was already returned when it was enqueued).
+ * Precision.  Accumulation is fp32 throughout.  bf16 latents are read on the
+ *             tensor cores (query operand rounded to bf16 for the score MMA,
+ *             probabilities to bf16 for the accumulate MMA, tf32 maps); bf16
+ *             writer rows use 3xTF32 products (fp32-accurate) before one
+ *             round-to-nearest-even; the LLA reconstruction splits each fp32
+ *             codec into bf16 hi + lo parts (~2^-17).  fp32 latents and rows
+ *             take fp32 SIMT kernels.
  * Rotary.     R_pos rotates pair p = (x[2p], x[2p+1]) of a length-d vector by
  *             +pos * base^(-2 f(p) / d_h), with f(p) = floor(p * d_h / d):
  *             textbook interleaved RoPE at d = d_h, and m = d / d_h consecutive
