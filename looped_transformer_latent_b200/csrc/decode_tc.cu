@@ -97,6 +97,15 @@ __host__ __device__ __forceinline__ int first_cta(int64_t x, int64_t U, int G) {
   return (int)(((x + 1) * G + U - 1) / U - 1);
 }
 
+// Walks a CTA's flat tiles in order, tracking the sequence and the tile
+// within it (no division in the per-tile loops).
+struct TileCursor {
+  int b, tt, NT;
+  __device__ __forceinline__ void next() {
+    if (++tt == NT) { tt = 0; ++b; }
+  }
+};
+
 struct Layout {
   int nkb, nvb, ngrp, R;
   __host__ __device__ int q_off() const { return 0; }
@@ -148,9 +157,9 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
     u1 = (int64_t)blockIdx.y * NT + min(NT, (s + 1) * tpt);
   }
   const int ntot = (int)(u1 - u0);
-  // flat tile n of this CTA -> sequence and tile within the sequence
-  auto seq_of = [&](int n) { return (int)((u0 + n) / NT); };
-  auto tile_in = [&](int n, int b) { return (int)(u0 + n - (int64_t)b * NT); };
+  // the first tile: sequence b_start, tile t_start within it
+  const int b_start = (int)(u0 / NT);
+  const int t_start = (int)(u0 - (int64_t)b_start * NT);
   const int nkb = L.nkb, nvb = L.nvb, ngrp = L.ngrp;
   const int rows = a.rows, rows_pad = a.rows_pad;
 
@@ -201,14 +210,16 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       uint32_t i = 0;
       bool ok = true;
       const uint32_t ring_addr = smem_u32(ring), full_addr = smem_u32(full), empty_addr = smem_u32(empty);
+      TileCursor cur[2] = {{b_start, t_start, NT}, {b_start, t_start, NT}};   // K tiles, V tiles
       for (int n = 0; n < ntot + LAG && ok; ++n) {
         for (int g = 0; g < 2 && ok; ++g) {
           const int tile = g == 0 ? n : n - LAG;
           if (tile < 0 || tile >= ntot) continue;
           const int nb = g == 0 ? nkb : nvb;
           const int c0 = g == 0 ? 0 : nkb;
-          const int b = seq_of(tile);
-          const int y = tile_in(tile, b) * TOK;
+          const int b = cur[g].b;
+          const int y = cur[g].tt * TOK;
+          cur[g].next();
           for (int c = 0; c < nb; c += 2, ++i) {
             if ((int)(i & 1) != pid) continue;
             const int cnt = nb - c >= 2 ? 2 : 1;
@@ -240,7 +251,7 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       int k = 0, jstop = nq;
       bool ok = true;
       for (int n = 0; n < ntot && ok; ++k) {
-        const int b = seq_of(n);
+        const int b = b_start + k;
         for (int j = 0; j < nq; ++j) {
           if (k > 0 && !wait_bar(smem_u32(&q_free[j]), (k - 1) & 1, abort_flag, a.err, ERR_TIMEOUT_QFREE)) {
             ok = false;
@@ -253,7 +264,7 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
                     smem_u32(&q_full[j]));
         }
         if (!ok) break;
-        n = (int)min((int64_t)ntot, ((int64_t)b + 1) * NT - u0);
+        n += k == 0 ? NT - t_start : NT;   // the next segment starts a sequence
       }
       if (!ok) {
         // drain: pieces j < jstop were last loaded for segment k, the others
@@ -280,9 +291,11 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       int slot = 0;
       uint32_t phase = 0;
       int kS = -1, kO = -1;   // segment of the newest score tile / accumulate tile
+      TileCursor cs{b_start, t_start, NT}, co{b_start, t_start, NT};
       for (int n = 0; n < ntot + LAG && ok; ++n) {
         if (n < ntot) {
-          const int b = seq_of(n), tt = tile_in(n, b);
+          const int tt = cs.tt;
+          cs.next();
           const bool first = n == 0 || tt == 0, last = n == ntot - 1 || tt == NT - 1;
           if (first) ++kS;
           const int buf = n % NBUF;
@@ -311,7 +324,8 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
         }
         if (n >= LAG) {
           const int m = n - LAG, buf = m % NBUF;
-          const bool first_o = m == 0 || tile_in(m, seq_of(m)) == 0;
+          const bool first_o = m == 0 || co.tt == 0;
+          co.next();
           if (first_o) {
             // a new segment's accumulators: wait until the last one was read out
             ++kO;
@@ -357,8 +371,10 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
     const bool active = owner && r < rows;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     float m_run = -INFINITY, l_run = 0.f;
+    TileCursor cur{b_start, t_start, NT};
     for (int n = 0; n < ntot; ++n) {
-      const int b = seq_of(n), tt = tile_in(n, b);
+      const int b = cur.b, tt = cur.tt;
+      cur.next();
       const bool first = n == 0 || tt == 0, last = n == ntot - 1 || tt == NT - 1;
       const int buf = n % NBUF;
       if (tid == 0) lead[0] = wait_bar(smem_u32(&s_full[buf]), (n / NBUF) & 1, abort_flag, a.err, ERR_TIMEOUT_S);
