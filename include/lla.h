@@ -213,13 +213,7 @@ int lla_decode_attn(const lla_decode_params *p, void *ws, size_t ws_bytes,
  * Bm = (U^V)^T, rotate_query = 0 and a post-rotary q.
  * One call serves one latent (e.g. the loop-1 latent c^(1) with r_k = r_v =
  * r_1, or the main latent with loops 2..T) and the loops t0..t0+nt-1 that
- * share it: every (loop, head) pair is one query row reading the same tile.
- * Schedule: the latent range is cut into partials that the output map merges,
- * either a fixed split per sequence or, when the batch needs several waves of
- * one CTA per SM, equal ranges of (sequence, 64-token tile) per SM.  The
- * environment variable LLA_ABSORB_SCHEDULE=split|stream forces one of the two
- * (for tests and measurement); the workspace size follows the schedule, so
- * query it under the same setting. */
+ * share it: every (loop, head) pair is one query row reading the same tile. */
 typedef struct {
   int32_t B, H, d_h;
   int32_t T, t0, nt;       /* loops in the model; this call serves t0..t0+nt-1 */

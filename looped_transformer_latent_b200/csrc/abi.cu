@@ -163,7 +163,7 @@ int check_lla(const lla_decode_params& p) {
 
 // Workspace layout of the absorbed read.
 struct HlaPlan {
-  int rows, n_lat, win_start, n_win, S, tps, use_tc, rows_pad, Sw, cpt, HG, stream, NT, G;
+  int rows, n_lat, win_start, n_win, S, tps, use_tc, rows_pad, Sw, cpt, HG;
   size_t o_qlat, o_pml, o_py, o_wml, o_wy, o_qbf, o_err, bytes;
 };
 
@@ -177,11 +177,11 @@ HlaPlan plan_hla(const hla_decode_params& p) {
   pl.n_win = i - pl.win_start + 1;
   pl.use_tc = pl.n_lat > 0 && absorb_tc_supported(p.lat_dtype, p.r_k, p.r_v, pl.rows);
   pl.rows_pad = pl.use_tc ? absorb_tc_rows_pad(pl.rows) : pl.rows;
-  pl.stream = 0; pl.NT = 0; pl.G = 0;
   if (pl.use_tc) {
-    // tensor-core read over 64-token tiles: split or stream schedule
-    const AbsorbTcPlan tp = absorb_tc_plan(p.B, pl.n_lat, kNumSms);
-    pl.S = tp.S; pl.tps = tp.tps; pl.stream = tp.stream; pl.NT = tp.NT; pl.G = tp.G;
+    // tensor-core read: one CTA per (split, sequence), 64-token tiles
+    const int S = absorb_tc_splits(p.B, pl.n_lat, kNumSms);
+    pl.tps = (int)(((pl.n_lat + S - 1) / S + 63) / 64 * 64);
+    pl.S = (pl.n_lat + pl.tps - 1) / pl.tps;
   } else if (pl.n_lat > 0) {
     const long ctas = (long)p.B * ((pl.rows + 15) / 16);
     long S = (kTargetCtas + ctas - 1) / ctas;
@@ -341,7 +341,6 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
   a.win_ml = reinterpret_cast<float*>(w + pl.o_wml);
   a.win_y = reinterpret_cast<float*>(w + pl.o_wy);
   a.S = pl.S; a.tps = pl.tps; a.Sw = pl.Sw; a.cpt = pl.cpt;
-  a.stream = pl.stream; a.NT = pl.NT; a.G = pl.G;
   a.use_tc = pl.use_tc; a.rows_pad = pl.rows_pad;
   a.qbf = reinterpret_cast<__nv_bfloat16*>(w + pl.o_qbf);
   a.err = reinterpret_cast<int*>(w + pl.o_err);

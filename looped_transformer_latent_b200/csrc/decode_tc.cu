@@ -5,18 +5,8 @@
 // work is two dense contractions shared by up to 64 rows:
 //   S[row, j]  = q~[row, :] . c~^K_j                (scores, base-2 units)
 //   O^T[v, row] += sum_j c^V_j[v] P[row, j]          (latent-space accumulate)
-// Work is cut into 64-token tiles, numbered flat as u = b * NT + tile over
-// (sequence b, tile of its latent range).  Each CTA streams one contiguous
-// range of u:
-//   * split schedule: CTA (s, b) covers tiles [s * tps / 64, (s + 1) * tps / 64)
-//     of sequence b, one segment, and writes partial slot s;
-//   * stream schedule: G CTAs (one per SM) cover equal ranges of the flat
-//     index, so a range may end one sequence and start others.  Each
-//     (CTA, sequence) segment writes slot  c - (first CTA of the sequence);
-//     the first CTA of a sequence marks its unused slots empty (max = -inf),
-//     which the merges skip.  No CTA waits on another.
-// Per tile:
-//   * two TMA producer warps stream 64 x 64 bf16 blocks (128-byte swizzled,
+// One CTA handles one (split, sequence).  Per 64-token tile:
+//   * a TMA producer warp streams 64 x 64 bf16 blocks (128-byte swizzled,
 //     8 KB) of the latent through a ring of shared-memory slots;
 //   * an MMA warp issues S = Q~ C^K^T as M=64 x N=64 tcgen05 MMAs into one of
 //     three TMEM score buffers and, two tiles behind, O^T += C^V^T P^T as
@@ -27,19 +17,10 @@
 //     warp, the M=64 TMEM layout), read their 64 scores with tcgen05.ld, keep
 //     a running max that is only raised when it grows by more than 8 (2^8 in
 //     probability, safe in fp32/bf16) so the TMEM accumulator is rarely
-//     rescaled, and write P (bf16) to shared memory for the second MMA.  At
-//     a segment's last tile they write its (max, sum, O) partial and release
-//     the accumulators to the next segment;
-//   * a loader warp brings each segment's Q~ (bf16) into shared memory in
-//     16 KB pieces: a piece of the next segment is copied as soon as the
-//     current segment's last score MMA that reads that piece completes, so
-//     the switch to a new sequence overlaps the latent stream.
+//     rescaled, and write P (bf16) to shared memory for the second MMA.
 // Latent rows past the valid range are zero-filled by TMA and masked.  Every
 // mbarrier wait is bounded; on timeout the CTA records an error code in the
 // workspace (the merge then emits NaN), drains its copies and frees TMEM.
-#include <cstdlib>
-#include <cstring>
-
 #include <cuda.h>
 
 #include "kernels.cuh"
@@ -53,7 +34,7 @@ using namespace ptx;
 constexpr int TOK = 64;              // tokens per tile
 constexpr int BLK = 8192;            // one chunk: 64 tokens x 64 elements (128 bytes)
 constexpr int SLOT = 2 * BLK;        // ring slot: up to two chunks per TMA copy
-constexpr int NTHREADS = 256;        // warps 0-3 softmax, 4 and 6 TMA, 5 MMA, 7 Q~ loader
+constexpr int NTHREADS = 224;        // warps 0-3 softmax, 4 and 6 TMA, 5 MMA
 constexpr int SMEM_LIMIT = 232448;   // 227 KB per block (opt-in)
 constexpr int MAX_RING = 24;
 constexpr int MISC_BYTES = 512;
@@ -62,11 +43,9 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int NBUF = 3;              // score buffers (TMEM) and P buffers (smem)
 constexpr int LAG = NBUF - 1;        // O(n) is issued after S(n + LAG)
 constexpr uint32_t O_COL = 64 * NBUF;  // score buffers use columns [0, O_COL)
-constexpr int QB = 6;                // Q~ pieces of two chunks (r_k <= 768)
-constexpr int MAX_STREAM_SLOTS = 8;  // partial slots per sequence under the stream schedule
 
 enum : int { ERR_TIMEOUT_EMPTY = 1, ERR_TIMEOUT_FULL = 2, ERR_TIMEOUT_Q = 3, ERR_TIMEOUT_S = 4,
-             ERR_TIMEOUT_P = 5, ERR_TIMEOUT_O = 6, ERR_TIMEOUT_QFREE = 7, ERR_TIMEOUT_OFREE = 8 };
+             ERR_TIMEOUT_P = 5, ERR_TIMEOUT_O = 6 };
 
 // Bounded wait.  Gives up when the CTA's abort flag is raised (if honoured) or
 // after WAIT_CYCLES, raising the flag and recording `code`.
@@ -90,29 +69,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Stream schedule: CTA c of G covers flat tiles [c U / G, (c + 1) U / G).
-// first_cta(x) is the CTA whose range holds flat tile x (the largest c with
-// floor(c U / G) <= x).  Shared by the kernel and the host planner.
-__host__ __device__ __forceinline__ int first_cta(int64_t x, int64_t U, int G) {
-  return (int)(((x + 1) * G + U - 1) / U - 1);
-}
-
-// Walks a CTA's flat tiles in order, tracking the sequence and the tile
-// within it (no division in the per-tile loops).
-struct TileCursor {
-  int b, tt, NT;
-  __device__ __forceinline__ void next() {
-    if (++tt == NT) { tt = 0; ++b; }
-  }
-};
-
 struct Layout {
   int nkb, nvb, ngrp, R;
   __host__ __device__ int q_off() const { return 0; }
   __host__ __device__ int p_off() const { return nkb * BLK; }
   __host__ __device__ int ring_off() const { return p_off() + NBUF * BLK; }
   __host__ __device__ int bar_off() const { return ring_off() + R * SLOT; }
-  __host__ __device__ int nbars() const { return 2 * R + 2 * QB + 1 + 4 * NBUF + 1; }
+  __host__ __device__ int nbars() const { return 2 * R + 2 + 4 * NBUF; }
   __host__ __device__ int misc_off() const { return bar_off() + 8 * nbars(); }
   __host__ __device__ int bytes() const { return misc_off() + MISC_BYTES; }
 };
@@ -130,10 +93,8 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L.bar_off());
   uint64_t* full = bars;
   uint64_t* empty = bars + R;
-  uint64_t* q_full = bars + 2 * R;    // [QB] Q~ piece landed (one phase per segment)
-  uint64_t* q_free = q_full + QB;     // [QB] last score MMA of a segment on the piece done
-  uint64_t* o_free = q_free + QB;     // O accumulators read out at a segment's end
-  uint64_t* s_full = o_free + 1;      // [NBUF]
+  uint64_t* q_full = bars + 2 * R;
+  uint64_t* s_full = q_full + 1;      // [NBUF]
   uint64_t* s_free = s_full + NBUF;   // [NBUF]
   uint64_t* p_full = s_free + NBUF;   // [NBUF]
   uint64_t* o_done = p_full + NBUF;   // [NBUF]
@@ -145,21 +106,10 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
   float* alpha_s = reinterpret_cast<float*>(misc + 64);               // [64]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int NT = a.NT;
-  const int64_t U = (int64_t)a.B * NT;
-  int64_t u0, u1;
-  if (a.stream) {
-    u0 = (int64_t)blockIdx.x * U / a.G;
-    u1 = ((int64_t)blockIdx.x + 1) * U / a.G;
-  } else {
-    const int tpt = a.tps / TOK, s = blockIdx.x;
-    u0 = (int64_t)blockIdx.y * NT + (int64_t)s * tpt;
-    u1 = (int64_t)blockIdx.y * NT + min(NT, (s + 1) * tpt);
-  }
-  const int ntot = (int)(u1 - u0);
-  // the first tile: sequence b_start, tile t_start within it
-  const int b_start = (int)(u0 / NT);
-  const int t_start = (int)(u0 - (int64_t)b_start * NT);
+  const int s = blockIdx.x, b = blockIdx.y;
+  const int tok0 = s * a.tps;
+  const int tok1 = min(a.n_lat, tok0 + a.tps);
+  const int ntiles = (tok1 - tok0 + TOK - 1) / TOK;
   const int nkb = L.nkb, nvb = L.nvb, ngrp = L.ngrp;
   const int rows = a.rows, rows_pad = a.rows_pad;
 
@@ -168,11 +118,7 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       mbar_init(smem_u32(&full[i]), 1);
       mbar_init(smem_u32(&empty[i]), 1);
     }
-    for (int j = 0; j < QB; ++j) {
-      mbar_init(smem_u32(&q_full[j]), 1);
-      mbar_init(smem_u32(&q_free[j]), 1);
-    }
-    mbar_init(smem_u32(o_free), 128);
+    mbar_init(smem_u32(q_full), 1);
     for (int i = 0; i < NBUF; ++i) {
       mbar_init(smem_u32(&s_full[i]), 1);
       mbar_init(smem_u32(&s_free[i]), 128);
@@ -205,21 +151,23 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
     // for an odd last chunk).  Copy i goes to ring slot i mod R.
     if (lane == 0) {
       const int pid = warp == 4 ? 0 : 1;
+      const uint32_t qb = smem_u32(q_full);
+      if (pid == 0) {
+        mbar_arrive_tx(qb, nkb * BLK);
+        bulk_load(smem_u32(q_s), a.qbf + (size_t)b * nkb * (BLK / 2), nkb * BLK, qb);
+      }
       int slot = pid;
       uint32_t phase = 0, mine = 0;
       uint32_t i = 0;
       bool ok = true;
       const uint32_t ring_addr = smem_u32(ring), full_addr = smem_u32(full), empty_addr = smem_u32(empty);
-      TileCursor cur[2] = {{b_start, t_start, NT}, {b_start, t_start, NT}};   // K tiles, V tiles
-      for (int n = 0; n < ntot + LAG && ok; ++n) {
+      for (int n = 0; n < ntiles + LAG && ok; ++n) {
         for (int g = 0; g < 2 && ok; ++g) {
           const int tile = g == 0 ? n : n - LAG;
-          if (tile < 0 || tile >= ntot) continue;
+          if (tile < 0 || tile >= ntiles) continue;
           const int nb = g == 0 ? nkb : nvb;
           const int c0 = g == 0 ? 0 : nkb;
-          const int b = cur[g].b;
-          const int y = cur[g].tt * TOK;
-          cur[g].next();
+          const int y = tok0 + tile * TOK;
           for (int c = 0; c < nb; c += 2, ++i) {
             if ((int)(i & 1) != pid) continue;
             const int cnt = nb - c >= 2 ? 2 : 1;
@@ -235,43 +183,11 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       }
       if (!ok) {
         // drain: every copy this producer issued must land before the CTA exits
+        if (pid == 0) wait_bar(qb, 0, abort_flag, nullptr, 0, false);
         for (uint32_t k = 0; k < mine; ++k) {
           const uint32_t gi = pid + 2 * k;            // global copy index
           if (gi + R < i) continue;                   // long since consumed
           wait_bar(full_addr + 8 * (gi % R), (gi / R) & 1, abort_flag, nullptr, 0, false);
-        }
-      }
-    }
-  } else if (warp == 7) {
-    // ------------------------------------------------------------ Q~ loader --
-    // Segment k's Q~ goes to the same buffer in pieces of two chunks; piece j
-    // of segment k > 0 waits for q_free[j] of segment k - 1.
-    if (lane == 0) {
-      const int nq = (nkb + 1) / 2;
-      int k = 0, jstop = nq;
-      bool ok = true;
-      for (int n = 0; n < ntot && ok; ++k) {
-        const int b = b_start + k;
-        for (int j = 0; j < nq; ++j) {
-          if (k > 0 && !wait_bar(smem_u32(&q_free[j]), (k - 1) & 1, abort_flag, a.err, ERR_TIMEOUT_QFREE)) {
-            ok = false;
-            jstop = j;
-            break;
-          }
-          const int cnt = min(2, nkb - 2 * j);
-          mbar_arrive_tx(smem_u32(&q_full[j]), cnt * BLK);
-          bulk_load(smem_u32(q_s + 2 * j * BLK), a.qbf + ((size_t)b * nkb + 2 * j) * (BLK / 2), cnt * BLK,
-                    smem_u32(&q_full[j]));
-        }
-        if (!ok) break;
-        n += k == 0 ? NT - t_start : NT;   // the next segment starts a sequence
-      }
-      if (!ok) {
-        // drain: pieces j < jstop were last loaded for segment k, the others
-        // for segment k - 1
-        for (int j = 0; j < nq; ++j) {
-          const int kl = j < jstop ? k : k - 1;
-          if (kl >= 0) wait_bar(smem_u32(&q_full[j]), kl & 1, abort_flag, nullptr, 0, false);
         }
       }
     }
@@ -287,24 +203,17 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       const uint64_t k_desc = smem_desc_sw128(smem_u32(ring), 16, 1024);
       const uint64_t v_desc = smem_desc_sw128(smem_u32(ring), BLK, 1024);
       const uint64_t p_desc = smem_desc_sw128(smem_u32(p_s), 16, 1024);
-      bool ok = true;
+      bool ok = wait_bar(smem_u32(q_full), 0, abort_flag, a.err, ERR_TIMEOUT_Q);
       int slot = 0;
       uint32_t phase = 0;
-      int kS = -1, kO = -1;   // segment of the newest score tile / accumulate tile
-      TileCursor cs{b_start, t_start, NT}, co{b_start, t_start, NT};
-      for (int n = 0; n < ntot + LAG && ok; ++n) {
-        if (n < ntot) {
-          const int tt = cs.tt;
-          cs.next();
-          const bool first = n == 0 || tt == 0, last = n == ntot - 1 || tt == NT - 1;
-          if (first) ++kS;
+      for (int n = 0; n < ntiles + LAG && ok; ++n) {
+        if (n < ntiles) {
           const int buf = n % NBUF;
           if (n >= NBUF && !wait_bar(smem_u32(&s_free[buf]), ((n - NBUF) / NBUF) & 1, abort_flag, a.err, ERR_TIMEOUT_S)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + buf * 64;
           for (int kb = 0; kb < nkb && ok; kb += 2) {
             const int cnt = nkb - kb >= 2 ? 2 : 1;
-            if (first && !wait_bar(smem_u32(&q_full[kb >> 1]), kS & 1, abort_flag, a.err, ERR_TIMEOUT_Q)) { ok = false; break; }
             if (!wait_bar(full_addr + 8 * slot, phase, abort_flag, a.err, ERR_TIMEOUT_FULL)) { ok = false; break; }
             tc_fence_after();
             for (int j = 0; j < cnt; ++j) {
@@ -315,8 +224,6 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
                 mma_bf16(d, ad + 2 * k16, bd + 2 * k16, idS, ((kb + j) | k16) != 0);
             }
             mma_commit(empty_addr + 8 * slot);
-            // the segment's last read of this Q~ piece: the loader may refill it
-            if (last) mma_commit(smem_u32(&q_free[kb >> 1]));
             if (++slot == R) { slot = 0; phase ^= 1; }
           }
           if (!ok) break;
@@ -324,13 +231,6 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
         }
         if (n >= LAG) {
           const int m = n - LAG, buf = m % NBUF;
-          const bool first_o = m == 0 || co.tt == 0;
-          co.next();
-          if (first_o) {
-            // a new segment's accumulators: wait until the last one was read out
-            ++kO;
-            if (kO > 0 && !wait_bar(smem_u32(o_free), (kO - 1) & 1, abort_flag, a.err, ERR_TIMEOUT_OFREE)) { ok = false; break; }
-          }
           if (!wait_bar(smem_u32(&p_full[buf]), (m / NBUF) & 1, abort_flag, a.err, ERR_TIMEOUT_P)) { ok = false; break; }
           tc_fence_after();
           const uint64_t bd = p_desc + (uint64_t)((buf * BLK) >> 4);
@@ -348,9 +248,8 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
               const uint64_t ad = v_desc + (uint64_t)((slot * SLOT) >> 4);
 #pragma unroll
               for (int k16 = 0; k16 < 4; ++k16)
-                mma_bf16(dO, ad + 128 * k16, bd + 2 * k16, idO, (!first_o || k16 > 0) ? 1u : 0u);
+                mma_bf16(dO, ad + 128 * k16, bd + 2 * k16, idO, (m > 0 || k16 > 0) ? 1u : 0u);
             }
-            (void)cnt;
             mma_commit(empty_addr + 8 * slot);
             if (++slot == R) { slot = 0; phase ^= 1; }
           }
@@ -371,15 +270,12 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
     const bool active = owner && r < rows;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     float m_run = -INFINITY, l_run = 0.f;
-    TileCursor cur{b_start, t_start, NT};
-    for (int n = 0; n < ntot; ++n) {
-      const int b = cur.b, tt = cur.tt;
-      cur.next();
-      const bool first = n == 0 || tt == 0, last = n == ntot - 1 || tt == NT - 1;
+    bool ok = true;
+    for (int n = 0; n < ntiles; ++n) {
       const int buf = n % NBUF;
       if (tid == 0) lead[0] = wait_bar(smem_u32(&s_full[buf]), (n / NBUF) & 1, abort_flag, a.err, ERR_TIMEOUT_S);
       named_sync(1, 128);
-      if (!lead[0]) break;
+      if (!lead[0]) { ok = false; break; }
       tc_fence_after();
       float sc[64];
 #pragma unroll
@@ -387,7 +283,7 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(smem_u32(&s_free[buf]));
-      const int nvalid = min(TOK, a.n_lat - tt * TOK);
+      const int nvalid = min(TOK, tok1 - (tok0 + n * TOK));
       if (nvalid < TOK) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
@@ -404,9 +300,8 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       bool need = false;
       float alpha = 1.f;
       if (active) {
-        if (first) {
+        if (n == 0) {
           m_run = tmax;
-          l_run = 0.f;
         } else if (tmax > m_run + 8.f) {
           alpha = ex2(m_run - tmax);
           m_run = tmax;
@@ -426,11 +321,11 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       l_run = l_run * alpha + psum;
       if (named_any(1, 128, need)) {
-        // rescale the TMEM accumulators once O(n-1) (same segment) has landed
+        // rescale the TMEM accumulators once O(n-1) has landed
         if (owner) alpha_s[r] = alpha;
         if (tid == 0) lead[1] = wait_bar(smem_u32(&o_done[(n - 1) % NBUF]), ((n - 1) / NBUF) & 1, abort_flag, a.err, ERR_TIMEOUT_O);
         named_sync(1, 128);
-        if (!lead[1]) break;
+        if (!lead[1]) { ok = false; break; }
         tc_fence_after();
         for (int g = 0; g < ngrp; ++g) {
           for (int cc = 0; cc < rows_pad; cc += 16) {
@@ -450,7 +345,7 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
         // P buffer `buf` is free once O(n-NBUF) has completed
         if (tid == 0) lead[2] = wait_bar(smem_u32(&o_done[buf]), ((n - NBUF) / NBUF) & 1, abort_flag, a.err, ERR_TIMEOUT_O);
         named_sync(1, 128);
-        if (!lead[2]) break;
+        if (!lead[2]) { ok = false; break; }
       }
       if (owner && r < rows_pad) {
         uint8_t* prow = p_s + buf * BLK + r * 128;
@@ -461,31 +356,20 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       }
       fence_proxy_async_smem();
       mbar_arrive(smem_u32(&p_full[buf]));
-      if (!last) continue;
-      // ---- segment end: write its partial, then free the accumulators ----
-      if (tid == 0) lead[3] = wait_bar(smem_u32(&o_done[buf]), (n / NBUF) & 1, abort_flag, a.err, ERR_TIMEOUT_O);
+    }
+    if (ok) {
+      if (tid == 0) lead[3] = wait_bar(smem_u32(&o_done[(ntiles - 1) % NBUF]), ((ntiles - 1) / NBUF) & 1, abort_flag, a.err, ERR_TIMEOUT_O);
       named_sync(1, 128);
-      if (!lead[3]) break;
+      ok = lead[3] != 0;
+    }
+    if (ok) {
       tc_fence_after();
-      const int64_t seq0 = (int64_t)b * NT;
-      const int c_first = a.stream ? first_cta(seq0, U, a.G) : 0;
-      const int slot = a.stream ? (int)blockIdx.x - c_first : (int)blockIdx.x;
-      const int64_t bstride = (int64_t)a.B * rows;
       if (active) {
-        float* ml = a.part_ml + ((int64_t)slot * bstride + (int64_t)b * rows + r) * 2;
+        float* ml = a.part_ml + (((int64_t)s * a.B + b) * rows + r) * 2;
         ml[0] = m_run;
         ml[1] = l_run;
-        if (a.stream && seq0 >= u0) {
-          // this CTA holds the sequence's first segment: mark its unused slots
-          const int nseg = first_cta(seq0 + NT - 1, U, a.G) - c_first + 1;
-          for (int s2 = nseg; s2 < a.S; ++s2) {
-            float* e = a.part_ml + ((int64_t)s2 * bstride + (int64_t)b * rows + r) * 2;
-            e[0] = -INFINITY;
-            e[1] = 0.f;
-          }
-        }
       }
-      float* py = a.part_y + ((int64_t)slot * bstride + (int64_t)b * rows) * (int64_t)a.r_v;
+      float* py = a.part_y + ((int64_t)s * a.B + b) * rows * (int64_t)a.r_v;
       for (int g = 0; g < ngrp; ++g) {
         const int vv = g * 128 + 32 * warp + lane;   // M=128 layout: TMEM lane = value index
         for (int cc = 0; cc < rows_pad; cc += 16) {
@@ -499,8 +383,6 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(smem_u32(o_free));
     }
   }
 
@@ -531,15 +413,27 @@ EncodeTiledFn encode_fn() {
 int ring_slots(int r_k) {
   // 1 KB alignment slack + Q~ + P buffers + fixed barriers + misc; each ring
   // slot costs two chunks plus its two mbarriers
-  const int fixed = 1024 + (r_k / 64) * BLK + NBUF * BLK + 8 * (2 * QB + 2 + 4 * NBUF) + MISC_BYTES;
+  const int fixed = 1024 + (r_k / 64) * BLK + NBUF * BLK + 8 * (2 + 4 * NBUF) + MISC_BYTES;
   const int R = (SMEM_LIMIT - fixed) / (SLOT + 16);
   return R > MAX_RING ? MAX_RING : R;
 }
 
-// Split schedule: the split count with the smallest modelled time, in tile
-// periods: waves of one CTA per SM, each CTA streaming ceil(tiles / S) tiles
-// plus a fixed start-up cost of two tiles, plus the partials' cost.
-int split_count(int B, int tiles, int num_sms, double* t_best) {
+}  // namespace
+
+int absorb_tc_rows_pad(int rows) { return (rows + 15) / 16 * 16; }
+
+bool absorb_tc_supported(int lat_dtype, int r_k, int r_v, int rows) {
+  if (lat_dtype != LLA_BF16 || r_k % 64 || r_v % 64 || r_k < 64 || r_v < 64 || r_k > 768) return false;
+  if (rows < 1 || rows > 64 || ring_slots(r_k) < 4) return false;
+  // TMEM: two 64-column score buffers plus ceil(r_v/128) column groups of rows_pad
+  const int ngrp = (r_v / 64 + 1) / 2;
+  return O_COL + (uint32_t)(ngrp * absorb_tc_rows_pad(rows)) <= TMEM_COLS;
+}
+
+int absorb_tc_splits(int B, int n_lat, int num_sms) {
+  // pick the split count with the smallest modelled time: waves of one CTA per
+  // SM, each CTA streaming ceil(tiles / S) tiles plus a fixed start-up cost
+  const int tiles = (n_lat + TOK - 1) / TOK;
   int best = 1;
   double best_t = 1e300;
   for (int S = 1; S <= 16 && S <= tiles; ++S) {
@@ -548,64 +442,7 @@ int split_count(int B, int tiles, int num_sms, double* t_best) {
     const double t = (double)waves * ((tiles + S - 1) / S + 2.0) + 0.02 * S * tiles;
     if (t < best_t - 1e-9) { best_t = t; best = S; }
   }
-  if (t_best) *t_best = best_t;
   return best;
-}
-
-// Stream schedule: the most segments any sequence is cut into.
-int stream_slots(int B, int NT, int G) {
-  const int64_t U = (int64_t)B * NT;
-  int smax = 1;
-  for (int b = 0; b < B; ++b) {
-    const int64_t x = (int64_t)b * NT;
-    smax = std::max(smax, first_cta(x + NT - 1, U, G) - first_cta(x, U, G) + 1);
-  }
-  return smax;
-}
-
-}  // namespace
-
-int absorb_tc_rows_pad(int rows) { return (rows + 15) / 16 * 16; }
-
-bool absorb_tc_supported(int lat_dtype, int r_k, int r_v, int rows) {
-  if (lat_dtype != LLA_BF16 || r_k % 64 || r_v % 64 || r_k < 64 || r_v < 64 || r_k > 2 * 64 * QB) return false;
-  if (rows < 1 || rows > 64 || ring_slots(r_k) < 4) return false;
-  // TMEM: two 64-column score buffers plus ceil(r_v/128) column groups of rows_pad
-  const int ngrp = (r_v / 64 + 1) / 2;
-  return O_COL + (uint32_t)(ngrp * absorb_tc_rows_pad(rows)) <= TMEM_COLS;
-}
-
-AbsorbTcPlan absorb_tc_plan(int B, int n_lat, int num_sms) {
-  AbsorbTcPlan p;
-  p.NT = (n_lat + TOK - 1) / TOK;
-  double t_split = 0.0;
-  const int S = split_count(B, p.NT, num_sms, &t_split);
-  p.tps = ((n_lat + S - 1) / S + TOK - 1) / TOK * TOK;
-  p.S = (n_lat + p.tps - 1) / p.tps;
-  p.stream = 0;
-  p.G = 0;
-  // LLA_ABSORB_SCHEDULE=split|stream overrides the choice (stream only where
-  // every sequence fits the merge's slots)
-  const char* force = std::getenv("LLA_ABSORB_SCHEDULE");
-  const int want = !force ? -1 : std::strcmp(force, "stream") == 0 ? 1 : std::strcmp(force, "split") == 0 ? 0 : -1;
-  if (want == 0) return p;
-  const int64_t U = (int64_t)B * p.NT;
-  const int G = (int)std::min<int64_t>(num_sms, U);
-  const int S_stream = stream_slots(B, p.NT, G);
-  if (S_stream > MAX_STREAM_SLOTS) return p;
-  // equal ranges remove the last partial wave and all but one start-up per SM;
-  // a sequence switch costs about half a tile.  Chosen when the split grid
-  // needs more than one wave (a single wave leaves SMs to concurrent work).
-  const double per = (double)((U + G - 1) / G);
-  const double t_stream = per + 2.0 + 0.5 * (per / p.NT + 1.0) + 0.02 * p.NT * (double)(B + G) / B;
-  const bool multi_wave = (long)B * S > num_sms;
-  if (want == 1 || (multi_wave && t_stream < t_split)) {
-    p.stream = 1;
-    p.G = G;
-    p.S = S_stream;
-    p.tps = 0;
-  }
-  return p;
 }
 
 cudaError_t launch_absorb_split_tc(const AbsorbArgs& a, cudaStream_t st) {
@@ -636,7 +473,7 @@ cudaError_t launch_absorb_split_tc(const AbsorbArgs& a, cudaStream_t st) {
   const int smem = L.bytes() + 1024;
   cudaError_t e = cudaFuncSetAttribute(absorb_split_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid = a.stream ? dim3(a.G, 1) : dim3(a.S, a.B);
+  dim3 grid(a.S, a.B);
   absorb_split_tc<<<grid, NTHREADS, smem, st>>>(tmap2, tmap1, a, Rslots);
   return cudaGetLastError();
 }

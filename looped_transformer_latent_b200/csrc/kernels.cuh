@@ -57,9 +57,7 @@ struct AbsorbArgs {
   float *part_y;       // [S][B][rows][r_v]
   float *win_ml;       // [Sw][B][rows][2] per window chunk
   float *win_y;        // [Sw][B][rows][d_h]
-  int S, tps;          // partial slots per sequence; tokens per split (split schedule)
-  int stream, NT, G;   // tensor-core read: stream schedule flag, 64-token tiles per
-                       // sequence, CTAs of the stream schedule
+  int S, tps;          // splits of the latent range, tokens per split
   int Sw, cpt;         // window chunks, tokens per chunk
   // tensor-core path
   int use_tc;
@@ -177,11 +175,7 @@ cudaError_t launch_recon_split_tc(const ReconArgs& a, int* err, cudaStream_t st)
 
 bool absorb_tc_supported(int lat_dtype, int r_k, int r_v, int rows);
 int absorb_tc_rows_pad(int rows);
-// Schedule of the tensor-core read.  Split: S CTAs per sequence of tps tokens
-// each.  Stream: G CTAs over equal ranges of the B * NT tiles, S partial slots
-// per sequence (unused ones marked empty by the kernel).
-struct AbsorbTcPlan { int stream, S, tps, G, NT; };
-AbsorbTcPlan absorb_tc_plan(int B, int n_lat, int num_sms);
+int absorb_tc_splits(int B, int n_lat, int num_sms);
 cudaError_t launch_absorb_split_tc(const AbsorbArgs& a, cudaStream_t st);
 
 }  // namespace lla

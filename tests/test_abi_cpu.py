@@ -105,42 +105,6 @@ def test_hla_workspace_checks(lib):
     assert lib.hla_decode_workspace_bytes(ctypes.byref(_hla(N=0))) == 0
 
 
-def _stream_max_segments(B, NT, G):
-    # brute force: CTA c of G takes flat tiles [c U / G, (c + 1) U / G) of the
-    # U = B * NT tiles; count the CTAs that touch each sequence
-    U = B * NT
-    G = min(G, U)
-    owners = [set() for _ in range(B)]
-    for c in range(G):
-        for u in range(c * U // G, (c + 1) * U // G):
-            owners[u // NT].add(c)
-    return max(len(o) for o in owners)
-
-
-def test_read_schedule_slots(lib, monkeypatch):
-    # B = 37, 284 latent tokens (5 tiles of 64): the split planner picks 3
-    # splits; the stream schedule cuts some sequence into 4 segments, so the
-    # partial region grows by one slot of (max, sum) and r_v floats per row
-    B, N, W, H, nt, r_v = 37, 301, 16, 4, 3, 128
-    over = dict(B=B, N=N, W=W, H=H, nt=nt, q_stride_b=nt * H * 64, out_stride_b=nt * H * 64,
-                lat_stride_b=N * 256, win_stride_b=4 * 17 * H * 64)
-    monkeypatch.setenv("LLA_ABSORB_SCHEDULE", "split")
-    split = lib.hla_decode_workspace_bytes(ctypes.byref(_hla(**over)))
-    monkeypatch.setenv("LLA_ABSORB_SCHEDULE", "stream")
-    stream = lib.hla_decode_workspace_bytes(ctypes.byref(_hla(**over)))
-    rows = nt * H
-    rnd = lambda x: (x + 255) // 256 * 256
-    assert _stream_max_segments(B, 5, 148) == 4
-    assert stream - split == rnd(4 * B * rows * 8) - rnd(3 * B * rows * 8) + B * rows * r_v * 4
-    # 2 sequences of 10 tiles on 20 CTAs: 10 segments exceed the merge's 8
-    # slots, so the override falls back to the split schedule
-    over = dict(B=2, N=700, W=60, Wcap=61, win_stride_b=4 * 61 * 2 * 64, lat_stride_b=700 * 256)
-    assert _stream_max_segments(2, 10, 148) == 10
-    stream = lib.hla_decode_workspace_bytes(ctypes.byref(_hla(**over)))
-    monkeypatch.setenv("LLA_ABSORB_SCHEDULE", "split")
-    assert stream == lib.hla_decode_workspace_bytes(ctypes.byref(_hla(**over)))
-
-
 def test_empty_batch_is_a_no_op(lib):
     # B = 0 or nt = 0: nothing to do, null pointers allowed, no workspace
     p = _hla(B=0, lat=0, A=0, Bm=0, q=0, win_k=0, win_v=0, out=0)

@@ -131,44 +131,6 @@ def test_absorbed_read_bf16(cuda_device, case, rotate):
     assert err < TOL_BF16
 
 
-SCHEDULE_CASES = [
-    # B, N, W, H, nt, d_h, r_k, r_v, Wcap, schedule (None: the planner's choice)
-    (37, 301, 16, 4, 3, 64, 128, 128, 17, "stream"),  # CTAs of 1-2 tiles: up to 4 segments a sequence
-    (3, 500, 0, 16, 4, 128, 576, 576, 1, "stream"),   # one tile per CTA: 8 segments, every slot used
-    (160, 330, 8, 2, 2, 64, 128, 64, 9, None),         # planner picks stream; last tile holds one token
-    (150, 200, 0, 16, 4, 128, 576, 576, 1, None),      # LLA-2D-shaped rows, planner picks stream
-    (37, 301, 16, 4, 3, 64, 128, 128, 17, "split"),   # the split schedule on the first shape
-]
-
-
-@pytest.mark.parametrize("case", SCHEDULE_CASES)
-def test_absorbed_read_schedules(cuda_device, case, monkeypatch):
-    # the workspace starts as NaN bytes: a partial slot that the merge reads
-    # without the read having written it turns the output into NaN
-    B, N, W, H, nt, d_h, r_k, r_v, Wcap, sched = case
-    if sched:
-        monkeypatch.setenv("LLA_ABSORB_SCHEDULE", sched)
-    else:
-        monkeypatch.delenv("LLA_ABSORB_SCHEDULE", raising=False)
-    cs = _absorbed_case(2000 + B + N, B, N, W, H, nt, d_h, r_k, r_v, Wcap)
-    ref = _absorbed_oracle(cs, N, W, r_k, r_v, d_h, True)
-    dev = cuda_device
-    args = dict(lat=cs["lat"].to(dev), A=cs["A"].to(dev), Bm=cs["Bm"].to(dev), q=cs["q"].to(dev),
-                win_k=cs["wk"].to(dev), win_v=cs["wv"].to(dev),
-                out=torch.full(tuple(cs["q"].shape), float("nan"), device=dev),
-                N=N, W=W, t0=cs["t0"], rotate_query=True, rope_base=BASE)
-    need = L.hla_decode_workspace_bytes(**args)
-    assert need > 0
-    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=dev)
-    L.hla_decode_attn(workspace=ws, **args)
-    torch.cuda.synchronize()
-    got = f64(args["out"])
-    err = rel_l2(got, ref)
-    print(f"absorbed schedule {case}: rel L2 {err:.2e}")
-    assert np.all(np.isfinite(got))
-    assert err < TOL_BF16
-
-
 def test_absorbed_read_fp32_latents(cuda_device):
     B, N, W, H, nt, d_h, r_k, r_v, Wcap = 2, 333, 16, 4, 2, 64, 128, 64, 20
     cs = _absorbed_case(77, B, N, W, H, nt, d_h, r_k, r_v, Wcap, lat_dtype=torch.float32)
