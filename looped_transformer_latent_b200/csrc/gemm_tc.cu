@@ -400,13 +400,8 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] = 0.f;
           }
-          // a zero weight is an empty partial slot (or one that underflows):
-          // skipped, since an empty slot's values were never written
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float wt = wts[(16 * c + i) * ld + jb];
-            acc[i] = wt != 0.f ? fmaf(wt, v[i], acc[i]) : acc[i];
-          }
+          for (int i = 0; i < 16; ++i) acc[i] = fmaf(wts[(16 * c + i) * ld + jb], v[i], acc[i]);
         }
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = acc[i];

@@ -100,11 +100,8 @@ __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
           v = g.X[(int64_t)b * g.xs_b + (int64_t)row * g.xs_row + k];
         } else {
           const int64_t br = (int64_t)b * g.rows + row;
-          for (int s = 0; s < g.S; ++s) {
-            // zero weight: an empty slot (never written) or an underflow
-            const float w = wsplit[xb][s];
-            if (w != 0.f) v = fmaf(w, g.part_y[((int64_t)s * g.B * g.rows + br) * g.K + k], v);
-          }
+          for (int s = 0; s < g.S; ++s)
+            v = fmaf(wsplit[xb][s], g.part_y[((int64_t)s * g.B * g.rows + br) * g.K + k], v);
         }
       }
       xr[u] = v;
