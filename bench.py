@@ -206,26 +206,29 @@ class HlaStep(Step):
         L = self.L
         c = cfg
         B, N, T, H, d_h, D = c.B, c.N, c.T, c.H, c.d_h, c.D
-        codec = {k: v.to(dev) for k, v in synth.hla_codec(c, seed).items()}
+        self.codec_host = synth.hla_codec(c, seed)
+        codec = {k: v.to(dev) for k, v in self.codec_host.items()}
+        self.seed = seed
         g = torch.Generator(device=dev)
         g.manual_seed(seed + 7)
         lat0 = torch.empty(B, N, c.r_k + c.r_v, dtype=torch.bfloat16, device=dev)
         lat10 = torch.empty(B, N, 2 * c.r_1, dtype=torch.bfloat16, device=dev)
         # prefill: the writer fills layer 0 from synthetic hidden states; the
         # other layers get copies (the bytes every layer reads are its own)
-        chunk = max(1, (1 << 28) // (N * T * D))
+        chunk = self.prefill_chunk = max(1, (1 << 28) // (N * T * D))
         for b0 in range(0, B, chunk):
             nb = min(chunk, B - b0)
-            h = synth.hla_hidden(codec["P"], nb * (N - 1), seed + b0, D, device=dev).reshape(nb, N - 1, T, D)
+            h = self._prefill_hidden_chunk(b0, nb)
             L.lla_write_latents(L.LLA_WRITE_HLA, x=h, E_main=codec["E_main"], E_1=codec["E_1"],
                                 out0=lat0[b0:b0 + nb], out1=lat10[b0:b0 + nb], r_k=c.r_k, d_h=d_h,
                                 pos0=0, rope_base=c.base)
             del h
         lats = _clone_layers(lat0, c.L)
         lat1s = _clone_layers(lat10, c.L)
-        self.ins, self.outs = [], []
+        self.ins, self.outs, self.layers = [], [], []
         for layer in range(c.L):
             lay = {k: codec[k].clone() for k in ("E_main", "E_1", "A", "A_1", "Bm", "B_1")}
+            self.layers.append(lay)
             lay["lat"], lay["lat1"] = lats[layer], lat1s[layer]
             Wcap = c.W + 1
             lay["wk"] = torch.randn(B, T, Wcap, H, d_h, generator=g, device=dev).to(torch.bfloat16)
@@ -261,6 +264,18 @@ class HlaStep(Step):
             self.ws_side = torch.empty_like(self.ws)
             self.fork = [torch.cuda.Event() for _ in range(c.L)]
             self.join = [torch.cuda.Event() for _ in range(c.L)]
+
+    def _prefill_hidden_chunk(self, b0, nb):
+        c = self.cfg
+        return synth.hla_hidden(self.codec_host["P"], nb * (c.N - 1), self.seed + b0, c.D,
+                                device=self.dev).reshape(nb, c.N - 1, c.T, c.D)
+
+    def prefill_hidden(self, b):
+        """Host copy of the hidden states [N-1, T, D] the prefill wrote for
+        sequence b (regenerated from the same seeded generator)."""
+        b0 = b // self.prefill_chunk * self.prefill_chunk
+        nb = min(self.prefill_chunk, self.cfg.B - b0)
+        return self._prefill_hidden_chunk(b0, nb)[b - b0].cpu()
 
     def run(self, events=None):
         if self.side is None:
@@ -300,24 +315,25 @@ class Lla2dStep(Step):
         L = self.L
         c = cfg
         B, N, T, H, d_h = c.B, c.N, c.T, c.H, c.d_h
-        codec = {k: v.to(dev) for k, v in synth.lla_folded_codec(c, seed).items()}
+        self.codec_host = synth.lla_folded_codec(c, seed)
+        codec = {k: v.to(dev) for k, v in self.codec_host.items()}
+        self.seed = seed
         g = torch.Generator(device=dev)
         g.manual_seed(seed + 7)
         lat0 = torch.empty(B, N, c.r_k + c.r_v, dtype=torch.bfloat16, device=dev)
-        chunk = max(1, (1 << 28) // (N * T * H * d_h * 2))
+        chunk = self.prefill_chunk = max(1, (1 << 28) // (N * T * H * d_h * 2))
         for b0 in range(0, B, chunk):
             nb = min(chunk, B - b0)
-            k, v = synth.lla_kv(codec["P"], nb * (N - 1), d_h, seed + b0, device=dev)
-            k = k.reshape(nb, N - 1, T, H, d_h)
-            v = v.reshape(nb, N - 1, T, H, d_h)
+            k, v = self._prefill_kv_chunk(b0, nb)
             L.lla_write_latents(L.LLA_WRITE_FOLDED, x=k, xv=v, E_K=codec["E_K"], E_V=codec["E_V"],
                                 out0=lat0[b0:b0 + nb], pos0=0)
             del k, v
         lats = [lat0] + [lat0.clone() for _ in range(self.NBUF - 1)]
-        self.ins, self.outs = [], []
+        self.ins, self.outs, self.layers = [], [], []
         for layer in range(c.L):
             lay = {"UK": codec["U_K"].clone(), "UVt": codec["U_V"].transpose(2, 3).contiguous(),
                    "EK": codec["E_K"].clone(), "EV": codec["E_V"].clone(), "lat": lats[layer % self.NBUF]}
+            self.layers.append(lay)
             k_new, v_new = synth.lla_kv(codec["P"], B, d_h, seed + 1000 + layer, device=dev)
             lay["k"] = k_new.reshape(B, 1, T, H, d_h)
             lay["v"] = v_new.reshape(B, 1, T, H, d_h)
@@ -334,6 +350,21 @@ class Lla2dStep(Step):
             self.calls.append(("write", dict(mode=L.LLA_WRITE_FOLDED, x=lay["k"], xv=lay["v"], E_K=lay["EK"],
                                              E_V=lay["EV"], out0=lay["lat"], pos0=self.i), None))
         self._workspace()
+
+
+    def _prefill_kv_chunk(self, b0, nb):
+        c = self.cfg
+        k, v = synth.lla_kv(self.codec_host["P"], nb * (c.N - 1), c.d_h, self.seed + b0, device=self.dev)
+        shape = (nb, c.N - 1, c.T, c.H, c.d_h)
+        return k.reshape(shape), v.reshape(shape)
+
+    def prefill_kv(self, b):
+        """Host copies of the keys and values [N-1, T, H, d_h] the prefill
+        wrote for sequence b (regenerated from the same seeded generator)."""
+        b0 = b // self.prefill_chunk * self.prefill_chunk
+        nb = min(self.prefill_chunk, self.cfg.B - b0)
+        k, v = self._prefill_kv_chunk(b0, nb)
+        return k[b - b0].cpu(), v[b - b0].cpu()
 
 
 class LlaStep(Step):
@@ -454,16 +485,31 @@ def _slice_name(cfg):
     return "(sequence, head) slices of the single layer" if cfg.kind == "lla" else "(sequence, layer) slices"
 
 
-def cpu_baseline(cfg, budget_s=12.0):
+def cpu_baseline(cfg, budget_s=12.0, budget_1thread_s=6.0):
+    """The oracle on the host cores: all BLAS threads for about budget_s, then
+    one thread for about budget_1thread_s (value_1thread)."""
     total, n, threads, per_token = 0.0, 0, 1, 1
     while total < budget_s and n < 512:
         dt, threads, per_token = oracle_sample(cfg, seed=5 + n)
         total += dt
         n += 1
     tok_s = n / (per_token * total)   # a decoded token needs per_token slices
-    return {"value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n} {_slice_name(cfg)} of the {cfg.name} step (fp64 numpy), {total:.1f} s; "
-                      f"tokens/s = slices / ({per_token} slices per token x time)"}
+    out = {"value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "sample": f"{n} {_slice_name(cfg)} of the {cfg.name} step (fp64 numpy), {total:.1f} s; "
+                     f"tokens/s = slices / ({per_token} slices per token x time)"}
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        return out
+    t1, n1 = 0.0, 0
+    with threadpool_limits(limits=1):
+        while t1 < budget_1thread_s and n1 < 64:
+            dt, _, per_token = oracle_sample(cfg, seed=1005 + n1)
+            t1 += dt
+            n1 += 1
+    out["value_1thread"] = n1 / (per_token * t1)
+    out["sample_1thread"] = f"{n1} {_slice_name(cfg)} on one thread, {t1:.1f} s"
+    return out
 
 
 # ---------------------------------------------------------------- main --
@@ -503,20 +549,31 @@ def run_reference(args, cfg):
 
 
 # DRAM traffic (read + write) per latent token of the tensor-core latent read,
-# from ncu captures (profiles/absorb_split_tc_*.md), keyed by the sha256 prefix
-# of the kernel source it was taken on and the latent row width in bytes: a
-# changed kernel, or a row width never captured, reports no traffic.
-TC_TRAFFIC_PER_TOKEN = {("5163ad08b2a9e31d", 2048): 2122.7, ("5163ad08b2a9e31d", 2304): 2408.5}
+# from ncu captures of dram__bytes_read.sum + dram__bytes_write.sum, keyed by
+# the sha256 prefix of the kernel source it was taken on (comments and blank
+# lines removed, so only code changes count) and the latent row width in
+# bytes: a changed kernel, or a row width never captured, reports no traffic
+# (null) until it is captured again.
+TC_TRAFFIC_PER_TOKEN = {("bb2f3005e9069e90", 2048): 2122.7, ("bb2f3005e9069e90", 2304): 2408.5}
+
+
+def source_key(path):
+    """sha256 prefix of a source file with comments and blank lines removed."""
+    import hashlib
+    import re
+    try:
+        src = open(path).read()
+    except OSError:
+        return None
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    src = "\n".join(ln.strip() for ln in src.splitlines() if ln.strip())
+    return hashlib.sha256(src.encode()).hexdigest()[:16]
 
 
 def tc_traffic_per_token(row_bytes):
-    import hashlib
-    src = os.path.join(ROOT, "looped_transformer_latent_b200", "csrc", "decode_tc.cu")
-    try:
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    except OSError:
-        return None
-    return TC_TRAFFIC_PER_TOKEN.get((h, row_bytes))
+    key = source_key(os.path.join(ROOT, "looped_transformer_latent_b200", "csrc", "decode_tc.cu"))
+    return TC_TRAFFIC_PER_TOKEN.get((key, row_bytes))
 
 
 def reduce_max(dist, value, device):
@@ -534,7 +591,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="ouro_hla_4k", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--config", default="ouro_lla2d_768", choices=sorted(synth.CONFIGS))
     ap.add_argument("--mode", default="m1", choices=["m1", "m2"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

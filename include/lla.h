@@ -16,10 +16,15 @@
  * Conventions shared by every entry point
  * ----------------------------------------
  * Pointers.   Every tensor pointer is a DEVICE pointer owned by the caller.
- *             The library never allocates, frees or retains memory.  Scratch
- *             space is the caller's `ws` buffer of at least the size that the
- *             matching *_workspace_bytes() returns, 256-byte aligned.  Its
- *             contents need not be initialised and are garbage afterwards.
+ *             The library never allocates, frees or retains memory, with one
+ *             exception: hla_decode_attn_noalloc uses a static device array
+ *             held on each device that calls it (see that entry point).
+ *             Scratch space is otherwise the caller's `ws` buffer of at least
+ *             the size that the matching *_workspace_bytes() returns,
+ *             256-byte aligned.  Its contents need not be initialised and are
+ *             garbage afterwards.  Split plans, and so workspace sizes, follow
+ *             the current device's multiprocessor count: query a size with the
+ *             same device current as the call that uses it.
  * Layouts.    Row-major.  Sizes are in elements; strides are int64 element
  *             strides of the outermost (batch, head, token) axes only -- the
  *             inner axes named in each comment are dense.
@@ -27,11 +32,17 @@
  *             NULL = legacy default stream) and returns; it never synchronises.
  *             Inputs must stay valid until that work has run.  Two calls may
  *             share a workspace only if they are ordered on the GPU.
- * Threads.    No global mutable state: calls from several host threads are safe.
+ * Threads.    Calls from several host threads are safe, each with its own
+ *             workspace.  The exception is hla_decode_attn_noalloc: all of its
+ *             calls share one scratch array, so calls whose work may overlap
+ *             on the GPU race (see that entry point).
  * Errors.     Every function returns an lla_status.  Arguments are validated on
- *             the host before anything is launched; on any error nothing is
- *             launched and outputs are untouched.  LLA_ERR_CUDA reports a
- *             failed launch (cudaGetLastError) or device query.  Errors raised
+ *             the host before anything is launched: on a validation error
+ *             (LLA_ERR_NULL, _SHAPE, _DTYPE, _ALIGN, _WORKSPACE, _UNSUPPORTED)
+ *             nothing is launched and outputs are untouched.  LLA_ERR_CUDA
+ *             reports a failed launch (cudaGetLastError) or device query; it
+ *             can follow work the call had already enqueued, so the outputs of
+ *             such a call must be ignored.  Errors raised
  *             by kernels already running surface on the caller's next CUDA
  *             synchronisation, as usual.  No call aborts or traps.  Every wait
  *             inside the kernels (copy completion, tensor-core completion) is

@@ -1,5 +1,6 @@
 // C ABI entry points: host-side validation, workspace planning and launch
 // orchestration.  Nothing is launched unless every check passes.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -9,9 +10,32 @@ namespace lla {
 namespace {
 
 constexpr int kAbiVersion = 1;
-constexpr int kNumSms = 148;            // B200
-constexpr int kTargetCtas = 4 * kNumSms;  // SIMT split heuristics aim at ~4 CTAs per SM
+constexpr int kDefaultSms = 148;        // B200; used only when no device can be queried
+constexpr int kMaxDevices = 64;
 constexpr size_t kAlign = 256;
+
+// Streaming multiprocessors of the current device, queried once per device.
+// Split and wave plans (and so workspace sizes) follow it: query a workspace
+// size with the same device current as the call that uses it.  Without a
+// usable device (a host-only process sizing buffers) the B200's count is
+// assumed; any launch then fails with LLA_ERR_CUDA anyway.
+int num_sms() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return kDefaultSms;
+  }
+  const int known = cache[dev].load(std::memory_order_relaxed);
+  if (known > 0) return known;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    return kDefaultSms;
+  }
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline size_t elem_size(int dt) { return dt == LLA_BF16 ? 2 : 4; }
@@ -97,7 +121,8 @@ WriterArgs writer_args(const lla_write_params& p) {
   a.Nmax += a.Nmax % 2;
   // tensor cores (3xTF32, fp32-accurate) when the rows are stored as bf16
   a.use_tc = p.out_dtype == LLA_BF16 && writer_tc_ok(a);
-  a.S = a.use_tc ? writer_tc_splits(a, kNumSms) : writer_pick_splits(a, kNumSms);
+  const int sms = num_sms();
+  a.S = a.use_tc ? writer_tc_splits(a, sms) : writer_pick_splits(a, sms);
   return a;
 }
 
@@ -169,6 +194,8 @@ struct HlaPlan {
 
 HlaPlan plan_hla(const hla_decode_params& p) {
   HlaPlan pl;
+  const int sms = num_sms();
+  const long target_ctas = 4L * sms;   // SIMT split heuristic: about four CTAs per SM
   // SIMT split: one CTA per (split, sequence, 16 rows)
   pl.rows = p.nt * p.H;
   const int i = p.N - 1;
@@ -179,12 +206,12 @@ HlaPlan plan_hla(const hla_decode_params& p) {
   pl.rows_pad = pl.use_tc ? absorb_tc_rows_pad(pl.rows) : pl.rows;
   if (pl.use_tc) {
     // tensor-core read: one CTA per (split, sequence), 64-token tiles
-    const int S = absorb_tc_splits(p.B, pl.n_lat, kNumSms);
+    const int S = absorb_tc_splits(p.B, pl.n_lat, sms);
     pl.tps = (int)(((pl.n_lat + S - 1) / S + 63) / 64 * 64);
     pl.S = (pl.n_lat + pl.tps - 1) / pl.tps;
   } else if (pl.n_lat > 0) {
     const long ctas = (long)p.B * ((pl.rows + 15) / 16);
-    long S = (kTargetCtas + ctas - 1) / ctas;
+    long S = (target_ctas + ctas - 1) / ctas;
     const long tiles = (pl.n_lat + 15) / 16;
     S = std::max(1L, std::min(std::min(S, tiles), (long)map_max_splits()));
     pl.tps = (int)(((pl.n_lat + S - 1) / S + 15) / 16 * 16);
@@ -192,7 +219,7 @@ HlaPlan plan_hla(const hla_decode_params& p) {
   } else {
     pl.S = 0; pl.tps = 0;
   }
-  pl.Sw = window_chunks(p.B, p.nt, p.H, pl.n_win, p.win_dtype, p.d_h, kNumSms, &pl.cpt, &pl.HG);
+  pl.Sw = window_chunks(p.B, p.nt, p.H, pl.n_win, p.win_dtype, p.d_h, sms, &pl.cpt, &pl.HG);
   const size_t br = (size_t)p.B * pl.rows;
   Carve c;
   pl.o_qbf = c.take(pl.use_tc ? (size_t)p.B * 64 * p.r_k * 2 : 0);
@@ -208,6 +235,8 @@ HlaPlan plan_hla(const hla_decode_params& p) {
 
 HlaPlan plan_lla(const lla_decode_params& p) {
   HlaPlan pl;
+  const int sms = num_sms();
+  const long target_ctas = 4L * sms;
   pl.rows = p.nt * p.H;
   const int i = p.N - 1;
   pl.n_lat = std::max(0, i - p.W);
@@ -223,7 +252,7 @@ HlaPlan plan_lla(const lla_decode_params& p) {
     pl.tps = (pl.n_lat + 31) / 32 * 32;
   } else if (pl.n_lat > 0) {
     const long ctas = (long)p.B * pl.rows;
-    long S = (kTargetCtas + ctas - 1) / ctas;
+    long S = (target_ctas + ctas - 1) / ctas;
     const long tiles = (pl.n_lat + 31) / 32;
     S = std::max(1L, std::min(S, tiles));
     pl.tps = (int)(((pl.n_lat + S - 1) / S + 31) / 32 * 32);
@@ -231,7 +260,7 @@ HlaPlan plan_lla(const lla_decode_params& p) {
   } else {
     pl.S = 0; pl.tps = 0;
   }
-  pl.Sw = window_chunks(p.B, p.nt, p.H, pl.n_win, p.win_dtype, p.d_h, kNumSms, &pl.cpt, &pl.HG);
+  pl.Sw = window_chunks(p.B, p.nt, p.H, pl.n_win, p.win_dtype, p.d_h, sms, &pl.cpt, &pl.HG);
   const size_t br = (size_t)p.B * pl.rows;
   Carve c;
   pl.o_qlat = 0;

@@ -425,7 +425,8 @@ int absorb_tc_rows_pad(int rows) { return (rows + 15) / 16 * 16; }
 bool absorb_tc_supported(int lat_dtype, int r_k, int r_v, int rows) {
   if (lat_dtype != LLA_BF16 || r_k % 64 || r_v % 64 || r_k < 64 || r_v < 64 || r_k > 768) return false;
   if (rows < 1 || rows > 64 || ring_slots(r_k) < 4) return false;
-  // TMEM: two 64-column score buffers plus ceil(r_v/128) column groups of rows_pad
+  // TMEM: NBUF (three) 64-column score buffers, O_COL columns in all, plus
+  // ceil(r_v/128) column groups of rows_pad
   const int ngrp = (r_v / 64 + 1) / 2;
   return O_COL + (uint32_t)(ngrp * absorb_tc_rows_pad(rows)) <= TMEM_COLS;
 }

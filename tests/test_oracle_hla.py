@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 from scipy.special import softmax
 
-from oracle import codec, exact, hla, rope
+from oracle import codec, exact, hla, lla, rope
 
 BASE = 10000.0
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -295,5 +295,16 @@ def test_printed_cache_sizes():
     assert full == g["ouro_full_cache_kib_per_token"] * 1024
     assert lat == g["ouro_hla_cache_kib_per_token"] * 1024
     assert round(full / lat, 1) == g["ouro_hla_reduction"]
-    # LLA abstract: 32x on Huginn-3.5B; per-head rank r over T loops of d_h
-    assert 32 * 96 // 96 == g["huginn_lla_compression"]
+    # LLA abstract: 32x on Huginn-3.5B.  Count the numbers one token occupies
+    # through the oracle's own per-head writer at the Huginn-like shapes (32
+    # loops, 55 heads, d_h = 96, rank 96): its per-loop K and V in, the
+    # per-head K and V latent rows out.
+    T_h, H_h, dh_h, r_h = 32, 55, 96, 96
+    rng = np.random.default_rng(5)
+    k = rng.standard_normal((1, T_h, H_h, dh_h))
+    v = rng.standard_normal((1, T_h, H_h, dh_h))
+    EK = rng.standard_normal((T_h, H_h, r_h, dh_h))
+    EV = rng.standard_normal((T_h, H_h, r_h, dh_h))
+    cK, cV = lla.write_perhead(k, v, EK, EV)
+    assert cK.shape == (H_h, 1, r_h) and cV.shape == (H_h, 1, r_h)
+    assert (k.size + v.size) / (cK.size + cV.size) == g["huginn_lla_compression"]
