@@ -769,7 +769,7 @@ def main():
         tf = flops / 1e12 / (mean_ms / 1e3) if mean_ms > 0 else 0.0
         line["roofline"] = {"bound": "tensor", "achieved": tf, "peak": tflops, "unit": "TFLOP/s",
                             "frac": tf / tflops, "traffic": None,
-                            "kernel": "LLA reconstruct-on-read (recon_split_tc)",
+                            "kernel": "LLA reconstruct-on-read (recon_group_tc)",
                             "peak_source": src + " (dense bf16)", "per_launch_ms": mean_ms,
                             "flops_per_launch": flops, "latent_gbs": achieved,
                             "launches_per_step": len(main_ix),

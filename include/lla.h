@@ -53,9 +53,10 @@
  *             tensor cores (query operand rounded to bf16 for the score MMA,
  *             probabilities to bf16 for the accumulate MMA, tf32 maps); bf16
  *             writer rows use 3xTF32 products (fp32-accurate) before one
- *             round-to-nearest-even; the LLA reconstruction splits each fp32
- *             codec into bf16 hi + lo parts (~2^-17).  fp32 latents and rows
- *             take fp32 SIMT kernels.
+ *             round-to-nearest-even; the LLA reconstruction rounds each fp32
+ *             decoder to bf16 for its tensor-core product (about 2^-9
+ *             relative per entry; output error ~2e-3 relative).  fp32 latents
+ *             and rows take fp32 SIMT kernels.
  * Rotary.     R_pos rotates pair p = (x[2p], x[2p+1]) of a length-d vector by
  *             +pos * base^(-2 f(p) / d_h), with f(p) = floor(p * d_h / d):
  *             textbook interleaved RoPE at d = d_h, and m = d / d_h consecutive

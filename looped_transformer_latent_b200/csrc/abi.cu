@@ -451,7 +451,7 @@ int lla_decode_attn(const lla_decode_params* p, void* ws, size_t ws_bytes, lla_s
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
   if (e == cudaSuccess) e = mark(p->timing_events, 0, s);
   if (e == cudaSuccess && a.n_lat > 0) {
-    e = (pl.use_tc && recon_tc_supported(a)) ? launch_recon_split_tc(a, err, s) : cudaErrorNotSupported;
+    e = (pl.use_tc && recon_tc_supported(a)) ? launch_recon_tc(a, err, s, num_sms()) : cudaErrorNotSupported;
     if (e == cudaErrorNotSupported) e = launch_recon_split_simt(a, s);   // S = 1 covers every token as well
   }
   if (e == cudaSuccess) e = mark(p->timing_events, 1, s);

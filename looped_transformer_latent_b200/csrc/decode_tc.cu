@@ -6,13 +6,17 @@
 //   S[row, j]  = q~[row, :] . c~^K_j                (scores, base-2 units)
 //   O^T[v, row] += sum_j c^V_j[v] P[row, j]          (latent-space accumulate)
 // One CTA handles one (split, sequence).  Per 64-token tile:
-//   * a TMA producer warp streams 64 x 64 bf16 blocks (128-byte swizzled,
-//     8 KB) of the latent through a ring of shared-memory slots;
-//   * an MMA warp issues S = Q~ C^K^T as M=64 x N=64 tcgen05 MMAs into one of
-//     three TMEM score buffers and, two tiles behind, O^T += C^V^T P^T as
-//     M=128 x N=rows MMAs (two value chunks per MMA) into TMEM accumulators.  The two-tile lag gives the
-//     softmax of a tile two tile-periods to finish, so the MMA warp -- and
-//     with it the latent stream -- never waits on the softmax;
+//   * two TMA producer warps stream 64 x 64 bf16 blocks (128-byte swizzled,
+//     8 KB) of the latent through shared-memory rings, one for the key
+//     chunks and one for the value chunks;
+//   * one MMA warp issues S = Q~ C^K^T as M=64 x N=64 tcgen05 MMAs into one of
+//     three TMEM score buffers; a second issues O^T += C^V^T P^T as
+//     M=128 x N=rows MMAs (two value chunks per MMA) into TMEM accumulators
+//     once the softmax has written P.  A single issuing thread is bound by its
+//     own issue latency (a few hundred cycles per MMA, whatever its size), so
+//     the two chains need two issuers to keep the tensor pipe fed.  With three
+//     score buffers the score chain -- and with it the key stream -- runs up to
+//     two tiles ahead of the softmax;
 //   * four softmax warps own one query row per thread (lanes 0..15 of each
 //     warp, the M=64 TMEM layout), read their 64 scores with tcgen05.ld, keep
 //     a running max that is only raised when it grows by more than 8 (2^8 in
@@ -34,14 +38,13 @@ using namespace ptx;
 constexpr int TOK = 64;              // tokens per tile
 constexpr int BLK = 8192;            // one chunk: 64 tokens x 64 elements (128 bytes)
 constexpr int SLOT = 2 * BLK;        // ring slot: up to two chunks per TMA copy
-constexpr int NTHREADS = 224;        // warps 0-3 softmax, 4 and 6 TMA, 5 MMA
+constexpr int NTHREADS = 256;        // warps 0-3 softmax, 4 and 6 TMA, 5 and 7 MMA
 constexpr int SMEM_LIMIT = 232448;   // 227 KB per block (opt-in)
 constexpr int MAX_RING = 24;
 constexpr int MISC_BYTES = 512;
 constexpr long long WAIT_CYCLES = 1ll << 32;  // ~2 s at 2 GHz
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NBUF = 3;              // score buffers (TMEM) and P buffers (smem)
-constexpr int LAG = NBUF - 1;        // O(n) is issued after S(n + LAG)
 constexpr uint32_t O_COL = 64 * NBUF;  // score buffers use columns [0, O_COL)
 
 enum : int { ERR_TIMEOUT_EMPTY = 1, ERR_TIMEOUT_FULL = 2, ERR_TIMEOUT_Q = 3, ERR_TIMEOUT_S = 4,
@@ -75,7 +78,7 @@ struct Layout {
   __host__ __device__ int p_off() const { return nkb * BLK; }
   __host__ __device__ int ring_off() const { return p_off() + NBUF * BLK; }
   __host__ __device__ int bar_off() const { return ring_off() + R * SLOT; }
-  __host__ __device__ int nbars() const { return 2 * R + 2 + 4 * NBUF; }
+  __host__ __device__ int nbars() const { return 2 * R + 3 + 4 * NBUF; }
   __host__ __device__ int misc_off() const { return bar_off() + 8 * nbars(); }
   __host__ __device__ int bytes() const { return misc_off() + MISC_BYTES; }
 };
@@ -98,7 +101,7 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
   uint64_t* s_free = s_full + NBUF;   // [NBUF]
   uint64_t* p_full = s_free + NBUF;   // [NBUF]
   uint64_t* o_done = p_full + NBUF;   // [NBUF]
-  uint64_t* fin = o_done + NBUF;
+  uint64_t* fin = o_done + NBUF;      // [2] one per MMA issuer (abort path)
   uint8_t* misc = base + L.misc_off();
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
@@ -126,6 +129,7 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       mbar_init(smem_u32(&o_done[i]), 1);
     }
     mbar_init(smem_u32(fin), 1);
+    mbar_init(smem_u32(fin + 1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -142,58 +146,61 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // The ring is two rings: slots [0, RK) carry key chunks, read only by the
+  // score issuer, and slots [RK, R) value chunks, read only by the value
+  // issuer.  Each ring has one producer and one consumer that both walk it in
+  // order, so a consumer never waits on a phase more than one use ahead (the
+  // two MMA chains run at different paces; one shared ring could not keep
+  // that guarantee).
+  const int RK = R / 2, RV = R - RK;
   if (warp == 4 || warp == 6) {
     // ----------------------------------------------------------- producers --
-    // Two producer warps alternate over the copy sequence (one TMA copy costs
-    // a fixed issue time, so two issuers and two-chunk copies keep the latent
-    // stream near full bandwidth).  Sequence per step n: the K chunks of tile n,
-    // then the V chunks of tile n-LAG, each group in copies of two chunks (one
-    // for an odd last chunk).  Copy i goes to ring slot i mod R.
+    // Warp 4: Q~ (one bulk copy), then the key chunks of tiles 0, 1, ...;
+    // warp 6: the value chunks of tiles 0, 1, ...  Copies carry two 64-element
+    // chunks (one for an odd last chunk); copy i of a ring goes to its slot
+    // i mod (ring size).
     if (lane == 0) {
-      const int pid = warp == 4 ? 0 : 1;
+      const bool kring = warp == 4;
+      const int nslots = kring ? RK : RV, slot0 = kring ? 0 : RK;
+      const int nb = kring ? nkb : nvb, c0 = kring ? 0 : nkb;
       const uint32_t qb = smem_u32(q_full);
-      if (pid == 0) {
+      if (kring) {
         mbar_arrive_tx(qb, nkb * BLK);
         bulk_load(smem_u32(q_s), a.qbf + (size_t)b * nkb * (BLK / 2), nkb * BLK, qb);
       }
-      int slot = pid;
-      uint32_t phase = 0, mine = 0;
       uint32_t i = 0;
       bool ok = true;
       const uint32_t ring_addr = smem_u32(ring), full_addr = smem_u32(full), empty_addr = smem_u32(empty);
-      for (int n = 0; n < ntiles + LAG && ok; ++n) {
-        for (int g = 0; g < 2 && ok; ++g) {
-          const int tile = g == 0 ? n : n - LAG;
-          if (tile < 0 || tile >= ntiles) continue;
-          const int nb = g == 0 ? nkb : nvb;
-          const int c0 = g == 0 ? 0 : nkb;
-          const int y = tok0 + tile * TOK;
-          for (int c = 0; c < nb; c += 2, ++i) {
-            if ((int)(i & 1) != pid) continue;
-            const int cnt = nb - c >= 2 ? 2 : 1;
-            if (!wait_bar(empty_addr + 8 * slot, phase ^ 1, abort_flag, a.err, ERR_TIMEOUT_EMPTY)) { ok = false; break; }
-            mbar_arrive_tx(full_addr + 8 * slot, cnt * BLK);
-            tma_load_4d(ring_addr + slot * SLOT, cnt == 2 ? (const void*)&tmap2 : (const void*)&tmap1,
-                        full_addr + 8 * slot, 0, y, c0 + c, b);
-            ++mine;
-            slot += 2;
-            if (slot >= R) { slot -= R; phase ^= 1; }
+      for (int n = 0; n < ntiles && ok; ++n) {
+        const int y = tok0 + n * TOK;
+        for (int c = 0; c < nb; c += 2, ++i) {
+          const int cnt = nb - c >= 2 ? 2 : 1;
+          const uint32_t slot = slot0 + i % nslots;
+          if (!wait_bar(empty_addr + 8 * slot, ((i / nslots) & 1) ^ 1, abort_flag, a.err, ERR_TIMEOUT_EMPTY)) {
+            ok = false;
+            break;
           }
+          mbar_arrive_tx(full_addr + 8 * slot, cnt * BLK);
+          tma_load_4d(ring_addr + slot * SLOT, cnt == 2 ? (const void*)&tmap2 : (const void*)&tmap1,
+                      full_addr + 8 * slot, 0, y, c0 + c, b);
         }
       }
       if (!ok) {
         // drain: every copy this producer issued must land before the CTA exits
-        if (pid == 0) wait_bar(qb, 0, abort_flag, nullptr, 0, false);
-        for (uint32_t k = 0; k < mine; ++k) {
-          const uint32_t gi = pid + 2 * k;            // global copy index
-          if (gi + R < i) continue;                   // long since consumed
-          wait_bar(full_addr + 8 * (gi % R), (gi / R) & 1, abort_flag, nullptr, 0, false);
-        }
+        if (kring) wait_bar(qb, 0, abort_flag, nullptr, 0, false);
+        for (uint32_t k = (i > (uint32_t)nslots ? i - nslots : 0); k < i; ++k)
+          wait_bar(full_addr + 8 * (slot0 + k % nslots), (k / nslots) & 1, abort_flag, nullptr, 0, false);
       }
     }
-  } else if (warp == 5) {
-    // ---------------------------------------------------------- MMA issuer --
+  } else if (warp == 5 || warp == 7) {
+    // --------------------------------------------------------- MMA issuers --
+    // One tcgen05.mma chain per issuing thread runs at the thread's issue
+    // latency, not the tensor pipe's rate, so the two independent chains get
+    // one issuer each: warp 5 the scores S(n) = Q~ C^K^T from the key ring,
+    // warp 7 the value accumulation O(m) += C^V^T P^T from the value ring,
+    // each as soon as its inputs are ready.
     if (lane == 0) {
+      const bool scores = warp == 5;
       const uint32_t idS = idesc_bf16(64, 64, false, false);
       const uint32_t idO = idesc_bf16(128, rows_pad, true, false);
       const uint32_t full_addr = smem_u32(full), empty_addr = smem_u32(empty);
@@ -203,18 +210,18 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       const uint64_t k_desc = smem_desc_sw128(smem_u32(ring), 16, 1024);
       const uint64_t v_desc = smem_desc_sw128(smem_u32(ring), BLK, 1024);
       const uint64_t p_desc = smem_desc_sw128(smem_u32(p_s), 16, 1024);
-      bool ok = wait_bar(smem_u32(q_full), 0, abort_flag, a.err, ERR_TIMEOUT_Q);
-      int slot = 0;
-      uint32_t phase = 0;
-      for (int n = 0; n < ntiles + LAG && ok; ++n) {
-        if (n < ntiles) {
+      bool ok = !scores || wait_bar(smem_u32(q_full), 0, abort_flag, a.err, ERR_TIMEOUT_Q);
+      uint32_t i = 0;   // copy index within this issuer's ring
+      if (scores) {
+        for (int n = 0; n < ntiles && ok; ++n) {
           const int buf = n % NBUF;
           if (n >= NBUF && !wait_bar(smem_u32(&s_free[buf]), ((n - NBUF) / NBUF) & 1, abort_flag, a.err, ERR_TIMEOUT_S)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + buf * 64;
-          for (int kb = 0; kb < nkb && ok; kb += 2) {
+          for (int kb = 0; kb < nkb && ok; kb += 2, ++i) {
             const int cnt = nkb - kb >= 2 ? 2 : 1;
-            if (!wait_bar(full_addr + 8 * slot, phase, abort_flag, a.err, ERR_TIMEOUT_FULL)) { ok = false; break; }
+            const uint32_t slot = i % RK;
+            if (!wait_bar(full_addr + 8 * slot, (i / RK) & 1, abort_flag, a.err, ERR_TIMEOUT_FULL)) { ok = false; break; }
             tc_fence_after();
             for (int j = 0; j < cnt; ++j) {
               const uint64_t ad = q_desc + (uint64_t)(((kb + j) * BLK) >> 4);
@@ -224,19 +231,19 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
                 mma_bf16(d, ad + 2 * k16, bd + 2 * k16, idS, ((kb + j) | k16) != 0);
             }
             mma_commit(empty_addr + 8 * slot);
-            if (++slot == R) { slot = 0; phase ^= 1; }
           }
           if (!ok) break;
           mma_commit(smem_u32(&s_full[buf]));
         }
-        if (n >= LAG) {
-          const int m = n - LAG, buf = m % NBUF;
+      } else {
+        for (int m = 0; m < ntiles && ok; ++m) {
+          const int buf = m % NBUF;
           if (!wait_bar(smem_u32(&p_full[buf]), (m / NBUF) & 1, abort_flag, a.err, ERR_TIMEOUT_P)) { ok = false; break; }
           tc_fence_after();
           const uint64_t bd = p_desc + (uint64_t)((buf * BLK) >> 4);
-          for (int vb = 0; vb < nvb && ok; vb += 2) {
-            const int cnt = nvb - vb >= 2 ? 2 : 1;
-            if (!wait_bar(full_addr + 8 * slot, phase, abort_flag, a.err, ERR_TIMEOUT_FULL)) { ok = false; break; }
+          for (int vb = 0; vb < nvb && ok; vb += 2, ++i) {
+            const uint32_t slot = RK + i % RV;
+            if (!wait_bar(full_addr + 8 * slot, (i / RV) & 1, abort_flag, a.err, ERR_TIMEOUT_FULL)) { ok = false; break; }
             tc_fence_after();
             {
               // one M=128 MMA covers both chunks of the copy: the two 64-wide
@@ -251,16 +258,16 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
                 mma_bf16(dO, ad + 128 * k16, bd + 2 * k16, idO, (m > 0 || k16 > 0) ? 1u : 0u);
             }
             mma_commit(empty_addr + 8 * slot);
-            if (++slot == R) { slot = 0; phase ^= 1; }
           }
           if (!ok) break;
           mma_commit(smem_u32(&o_done[buf]));
         }
       }
       if (!ok) {
-        // let every MMA already issued finish before TMEM is released
-        mma_commit(smem_u32(fin));
-        wait_bar(smem_u32(fin), 0, abort_flag, nullptr, 0, false);
+        // let every MMA this thread issued finish before TMEM is released
+        const uint32_t f = smem_u32(fin) + (scores ? 0 : 8);
+        mma_commit(f);
+        wait_bar(f, 0, abort_flag, nullptr, 0, false);
       }
     }
   } else {
@@ -413,7 +420,7 @@ EncodeTiledFn encode_fn() {
 int ring_slots(int r_k) {
   // 1 KB alignment slack + Q~ + P buffers + fixed barriers + misc; each ring
   // slot costs two chunks plus its two mbarriers
-  const int fixed = 1024 + (r_k / 64) * BLK + NBUF * BLK + 8 * (2 + 4 * NBUF) + MISC_BYTES;
+  const int fixed = 1024 + (r_k / 64) * BLK + NBUF * BLK + 8 * (3 + 4 * NBUF) + MISC_BYTES;
   const int R = (SMEM_LIMIT - fixed) / (SLOT + 16);
   return R > MAX_RING ? MAX_RING : R;
 }
@@ -424,7 +431,7 @@ int absorb_tc_rows_pad(int rows) { return (rows + 15) / 16 * 16; }
 
 bool absorb_tc_supported(int lat_dtype, int r_k, int r_v, int rows) {
   if (lat_dtype != LLA_BF16 || r_k % 64 || r_v % 64 || r_k < 64 || r_v < 64 || r_k > 768) return false;
-  if (rows < 1 || rows > 64 || ring_slots(r_k) < 4) return false;
+  if (rows < 1 || rows > 64 || ring_slots(r_k) < 4) return false;   // two slots per ring at least
   // TMEM: NBUF (three) 64-column score buffers, O_COL columns in all, plus
   // ceil(r_v/128) column groups of rows_pad
   const int ngrp = (r_v / 64 + 1) / 2;

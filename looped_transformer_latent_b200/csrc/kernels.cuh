@@ -168,10 +168,11 @@ cudaError_t launch_absorb_split_simt(const AbsorbArgs& a, cudaStream_t st);
 cudaError_t launch_window(const WindowArgs& w, cudaStream_t st);
 cudaError_t launch_merge(const MergeArgs& m, cudaStream_t st);
 cudaError_t launch_recon_split_simt(const ReconArgs& a, cudaStream_t st);
-// tensor-core reconstruct-on-read (recon_tc.cu): one CTA per (loop, head,
-// sequence) over the whole latent range, i.e. a single split
+// tensor-core reconstruct-on-read (recon_tc.cu): one CTA per (group of loops,
+// head, chunk of sequences), each sequence's whole latent range in one CTA,
+// i.e. a single split
 bool recon_tc_supported(const ReconArgs& a);
-cudaError_t launch_recon_split_tc(const ReconArgs& a, int* err, cudaStream_t st);
+cudaError_t launch_recon_tc(const ReconArgs& a, int* err, cudaStream_t st, int num_sms);
 
 bool absorb_tc_supported(int lat_dtype, int r_k, int r_v, int rows);
 int absorb_tc_rows_pad(int rows);

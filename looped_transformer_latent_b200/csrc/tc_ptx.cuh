@@ -166,6 +166,13 @@ __device__ __forceinline__ bool named_any(uint32_t id, uint32_t nthreads, bool v
   return out != 0;
 }
 
+// Maximum of a float over the 32 lanes of a warp (one instruction on sm_100a).
+__device__ __forceinline__ float redux_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -195,6 +202,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_32b(uint32_t saddr, uint32_t
   d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)1 << 61;
+  return d;
+}
+
+// Same, for the 64-byte swizzle (layout type 4), K-major: rows of 64 bytes,
+// 8-row atoms of 512 bytes (the stride byte offset); the leading byte offset
+// is unused for a K-major swizzled operand whose K step fits one atom row.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(512 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;
   return d;
 }
 
