@@ -370,38 +370,62 @@ class Lla2dStep(Step):
 class LlaStep(Step):
     """LLA per-head reconstruct-on-read (Huginn-like): one layer, all T loops
     of every head read their head's latents in one call, plus the per-head
-    writer for the new token."""
+    writer.  With W = 0 the writer stores the new token's latent (read from the
+    next step on).  With W > 0 (served semantics: an exact ring of the last W
+    tokens and the current one) the writer is the streaming store of the token
+    leaving the window, N - 2 - W, whose latent this step's read already needs
+    (prefill wrote it too; the writer's rows do not depend on how many tokens a
+    call writes, so the store reproduces them bit for bit)."""
 
     def __init__(self, cfg, dev, mode, seed=777):
         super().__init__(cfg, dev, mode)
         L = self.L
         c = cfg
-        B, N, T, H, d_h, r = c.B, c.N, c.T, c.H, c.d_h, c.r_k
+        B, N, T, H, d_h, r, W = c.B, c.N, c.T, c.H, c.d_h, c.r_k, c.W
         codec = {k: v.to(dev) for k, v in synth.lla_perhead_codec(c, seed).items()}
         g = torch.Generator(device=dev)
         g.manual_seed(seed + 7)
+        Wc = W + 1
         cK = torch.empty(B, H, N, r, dtype=torch.bfloat16, device=dev)
         cV = torch.empty(B, H, N, r, dtype=torch.bfloat16, device=dev)
+        ring_k = torch.zeros(B, T, Wc, H, d_h, dtype=torch.bfloat16, device=dev)
+        ring_v = torch.zeros_like(ring_k)
+        evict = N - 2 - W
+        if W > 0:
+            self.ek = torch.empty(B, 1, T, H, d_h, device=dev)
+            self.ev = torch.empty(B, 1, T, H, d_h, device=dev)
         chunk = max(1, (1 << 28) // (N * T * H * d_h * 2))
         for b0 in range(0, B, chunk):
             nb = min(chunk, B - b0)
             k, v = synth.lla_kv(codec["P"], nb * (N - 1), d_h, seed + b0, device=dev)
-            L.lla_write_latents(L.LLA_WRITE_PERHEAD, x=k.reshape(nb, N - 1, T, H, d_h),
-                                xv=v.reshape(nb, N - 1, T, H, d_h), E_K=codec["E_K"], E_V=codec["E_V"],
+            k = k.reshape(nb, N - 1, T, H, d_h)
+            v = v.reshape(nb, N - 1, T, H, d_h)
+            L.lla_write_latents(L.LLA_WRITE_PERHEAD, x=k, xv=v, E_K=codec["E_K"], E_V=codec["E_V"],
                                 out0=cK[b0:b0 + nb], out1=cV[b0:b0 + nb], pos0=0)
+            for j in range(max(0, N - 1 - W), N - 1):   # exact tokens of the window before the new one
+                ring_k[b0:b0 + nb, :, j % Wc] = k[:, j].to(torch.bfloat16)
+                ring_v[b0:b0 + nb, :, j % Wc] = v[:, j].to(torch.bfloat16)
+            if W > 0:
+                self.ek[b0:b0 + nb, 0] = k[:, evict]
+                self.ev[b0:b0 + nb, 0] = v[:, evict]
             del k, v
         k_new, v_new = synth.lla_kv(codec["P"], B, d_h, seed + 99, device=dev)
         self.k = k_new.reshape(B, 1, T, H, d_h)
         self.v = v_new.reshape(B, 1, T, H, d_h)
-        wk = self.k.reshape(B, T, 1, H, d_h).to(torch.bfloat16)
-        wv = self.v.reshape(B, T, 1, H, d_h).to(torch.bfloat16)
+        ring_k[:, :, (N - 1) % Wc] = self.k[:, 0].to(torch.bfloat16)
+        ring_v[:, :, (N - 1) % Wc] = self.v[:, 0].to(torch.bfloat16)
         self.q = torch.randn(B, T, H, d_h, generator=g, device=dev)
         self.out = torch.empty(B, T, H, d_h, device=dev)
         self.ins, self.outs = [self.q, self.k, self.v], [self.out]
-        self.calls.append(("lla", dict(cK=cK, cV=cV, UK=codec["U_K"], UV=codec["U_V"], q=self.q, win_k=wk,
-                                       win_v=wv, out=self.out, N=N, W=0, t0=0), "main"))
-        self.calls.append(("write", dict(mode=L.LLA_WRITE_PERHEAD, x=self.k, xv=self.v, E_K=codec["E_K"],
-                                         E_V=codec["E_V"], out0=cK, out1=cV, pos0=self.i), None))
+        self.calls.append(("lla", dict(cK=cK, cV=cV, UK=codec["U_K"], UV=codec["U_V"], q=self.q, win_k=ring_k,
+                                       win_v=ring_v, out=self.out, N=N, W=W, t0=0), "main"))
+        if W > 0:
+            self.ins += [self.ek, self.ev]
+            wx, wv, wpos = self.ek, self.ev, evict
+        else:
+            wx, wv, wpos = self.k, self.v, self.i
+        self.calls.append(("write", dict(mode=L.LLA_WRITE_PERHEAD, x=wx, xv=wv, E_K=codec["E_K"],
+                                         E_V=codec["E_V"], out0=cK, out1=cV, pos0=wpos), None))
         self._workspace()
 
 
@@ -554,7 +578,7 @@ def run_reference(args, cfg):
 # lines removed, so only code changes count) and the latent row width in
 # bytes: a changed kernel, or a row width never captured, reports no traffic
 # (null) until it is captured again.
-TC_TRAFFIC_PER_TOKEN = {("bb2f3005e9069e90", 2048): 2122.7, ("bb2f3005e9069e90", 2304): 2408.5}
+TC_TRAFFIC_PER_TOKEN = {("21d0011aedbae00a", 2304): 2383.9}
 
 
 def source_key(path):

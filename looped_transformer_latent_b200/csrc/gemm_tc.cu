@@ -19,9 +19,11 @@
 // ties away) and, for PREC = 3, store the remainder x - tf32(x) as a second
 // tf32 tile.  PREC = 3 issues hi*hi + hi*lo + lo*hi ("3xTF32"), whose error is
 // that of fp32 arithmetic; PREC = 1 issues hi*hi (relative error about 2^-11
-// per product).  One thread of an MMA warp issues the MMAs into TMEM and
-// releases stages with tcgen05.commit; the converter warps then read the
-// accumulators back (tcgen05.ld) for the epilogue.  Waits are bounded: on a
+// per product).  Up to three MMA warps issue the MMAs into separate TMEM
+// accumulators (one thread issuing a dependent chain is bound by its issue
+// latency; see AccPlan) and release stages with tcgen05.commit; the converter
+// warps then read the accumulators back (tcgen05.ld), add them, and run the
+// epilogue.  Waits are bounded: on a
 // timeout the CTA records an error code (outputs become NaN downstream).
 #include <cuda.h>
 
@@ -41,9 +43,10 @@ constexpr int GM = 128;                 // M of every MMA (codec rows per tile)
 constexpr int KCH = 32;                 // k per chunk: 32 fp32 = one 128-byte row
 constexpr int A_BYTES = GM * KCH * 4;   // 16 KB
 constexpr int NPROD = 256;              // converter + epilogue threads (warps 0-7)
-constexpr int MMA_WARP = NPROD / 32;    // warp 8: TMEM allocation, MMA issue
-constexpr int TMA_WARP = MMA_WARP + 1;  // warp 9: tensor-map copies
-constexpr int NTHR = NPROD + 64;
+constexpr int MMA_WARP = NPROD / 32;    // warps 8..8+NISS-1: MMA issue (warp 8 also TMEM allocation)
+constexpr int NISS = 3;                 // MMA issuer warps
+constexpr int TMA_WARP = MMA_WARP + NISS;  // warp 11: tensor-map copies
+constexpr int NTHR = NPROD + 32 * (NISS + 1);
 constexpr int SMEM_MAX = 232448;
 constexpr int YW_SMEM_MAX = 65536;      // output map: window term of the column slice kept in smem up to this
 __host__ __device__ constexpr int align8(int x) { return (x + 7) & ~7; }
@@ -121,6 +124,27 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 __device__ __forceinline__ int64_t qbf_index(int b, int row, int k, int r_k) {
   const int kb = k >> 6, e = k & 63;
   return (int64_t)b * (r_k >> 6) * 4096 + kb * 4096 + row * 64 + ((((e >> 3) ^ (row & 7)) << 3) | (e & 7));
+}
+
+// Accumulators and issuers.  One thread issuing a chain of tcgen05.mma is
+// bound by its own issue latency, not the tensor pipe, so independent
+// accumulator chains are spread over NISS issuer warps:
+//   PREC = 3 (3xTF32):  one accumulator per product (hi*hi, lo*hi, hi*lo),
+//                       issuer p issues product p of every chunk;
+//   PREC = 1, nb >= 2:  one accumulator per operand block jb (output map:
+//                       one per latent split), issuer jb mod NISS;
+//   PREC = 1, nb = 1:   two accumulators taking alternate k-chunks, issuers
+//                       0 and 1; the epilogue adds them.
+// The epilogue sums the accumulators of a product in a fixed order.
+struct AccPlan {
+  int nacc;      // accumulators (BN columns each)
+  int per_st;    // issuers that read each stage
+  int active;    // issuers with work
+};
+__host__ __device__ inline AccPlan acc_plan(int prec, int nb) {
+  if (prec == 3) return {3, 3, 3};
+  if (nb >= 2) return {nb, nb < NISS ? nb : NISS, nb < NISS ? nb : NISS};
+  return {2, 1, 2};
 }
 
 // Per-tile geometry, resolved from blockIdx for each kind.
@@ -241,13 +265,14 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
     }
   };
   const int first = min(NST, nchunks);
+  const AccPlan ap = acc_plan(PREC, nb);
   if (warp == TMA_WARP && lane == 0) {
     for (int i = 0; i < NST; ++i) {
       mbar_init(smem_u32(&loaded[i]), 1);
       mbar_init(smem_u32(&full[i]), NPROD);
-      mbar_init(smem_u32(&empty[i]), 1);
+      mbar_init(smem_u32(&empty[i]), ap.per_st);
     }
-    mbar_init(smem_u32(done), 1);
+    mbar_init(smem_u32(done), ap.active);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&maps.a[0]);
@@ -255,7 +280,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
     for (int i = 0; i < first; ++i) issue_chunk(i);
   }
   uint32_t ncols = 32;
-  while (ncols < (uint32_t)(nb * BN)) ncols <<= 1;
+  while (ncols < (uint32_t)(ap.nacc * BN)) ncols <<= 1;
   if (warp == MMA_WARP) {
     tmem_alloc(smem_u32(tmem_slot), ncols);
     tmem_relinquish();
@@ -381,6 +406,19 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
     const int m = t.m0 + 32 * quarter + lane;   // this thread's TMEM lane = codec row
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
     const bool have = nchunks > 0;
+    // accumulators summed for one output column block (fixed order)
+    const int nsum = PREC == 3 ? 3 : (nb == 1 && nchunks > 1 ? 2 : 1);
+    auto load_sum = [&](uint32_t col, float* v) {
+      tmem_ld16(lane_addr + col, v);
+      tmem_wait_ld();
+      for (int q = 1; q < nsum; ++q) {
+        float w[16];
+        tmem_ld16(lane_addr + (uint32_t)(q * BN) + col, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] += w[i];
+      }
+    };
     float cq = 1.f, sq = 0.f;
     if (KIND == KIND_QMAP && a.rotate && m < t.Mv) rope_cs(m >> 1, a.Mtot, a.d_h, a.base, (double)a.pos, &cq, &sq);
     const bool bad = !ok || (KIND == KIND_OMAP && a.err && *a.err);
@@ -394,8 +432,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
         for (int i = 0; i < 16; ++i) acc[i] = 0.f;
         for (int jb = 0; jb < nb; ++jb) {
           if (have) {
-            tmem_ld16(lane_addr + jb * BN + 16 * c, v);
-            tmem_wait_ld();
+            load_sum(jb * BN + 16 * c, v);
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] = 0.f;
@@ -406,8 +443,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = acc[i];
       } else if (have) {
-        tmem_ld16(lane_addr + 16 * c, v);
-        tmem_wait_ld();
+        load_sum(16 * c, v);
       } else {
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = 0.f;
@@ -488,38 +524,47 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
       }
     }
   } else if (lane == 0) {
-    // ---- MMA issue -------------------------------------------------------------
+    // ---- MMA issue (warps MMA_WARP .. MMA_WARP + NISS - 1) ----------------------
+    const int me = warp - MMA_WARP;
     const bool a_mn = KIND != KIND_WRITER;
     constexpr uint32_t idesc = idesc_tf32(GM, BN, KIND != KIND_WRITER);
     const uint32_t a_step = a_mn ? (1024u >> 4) : (32u >> 4);   // 8 k: two 4-row groups, or 32 bytes
     const uint32_t b_step = 32u >> 4;
+    if (me < ap.active) {
 #pragma unroll 1
-    for (int i = 0; i < nchunks; ++i) {
-      const int st = i % NST;
-      if (!wait_bar(smem_u32(&full[st]), (i / NST) & 1, abort_flag, a.err, ERR_GEMM_FULL)) break;
-      tc_fence_after();
-      const uint32_t s0 = sbase + st * stage_bytes;
-      const uint64_t ahi = a_mn ? smem_desc_sw128_32b(s0, 4096, 512) : smem_desc_sw128(s0, 16, 1024);
-      const uint64_t alo = a_mn ? smem_desc_sw128_32b(s0 + A_BYTES, 4096, 512) : smem_desc_sw128(s0 + A_BYTES, 16, 1024);
-      for (int jb = 0; jb < nb; ++jb) {
-        const uint32_t bt = s0 + a_part + jb * b_tile;
-        const uint64_t bhi = smem_desc_sw128(bt, 16, 1024);
-        const uint64_t blo = smem_desc_sw128(bt + nb * b_tile, 16, 1024);
-        const uint32_t d = tmem + jb * BN;
+      for (int i = 0; i < nchunks; ++i) {
+        if (PREC == 1 && nb == 1 && (i & 1) != me) continue;   // alternate chunks
+        const int st = i % NST;
+        if (!wait_bar(smem_u32(&full[st]), (i / NST) & 1, abort_flag, a.err, ERR_GEMM_FULL)) break;
+        tc_fence_after();
+        const uint32_t s0 = sbase + st * stage_bytes;
+        const uint64_t ahi = a_mn ? smem_desc_sw128_32b(s0, 4096, 512) : smem_desc_sw128(s0, 16, 1024);
+        const uint64_t alo = a_mn ? smem_desc_sw128_32b(s0 + A_BYTES, 4096, 512) : smem_desc_sw128(s0 + A_BYTES, 16, 1024);
+        if (PREC == 3) {
+          // product me: 0 = hi*hi, 1 = lo*hi, 2 = hi*lo, into accumulator me
+          const uint32_t bt = s0 + a_part;
+          const uint64_t bhi = smem_desc_sw128(bt, 16, 1024);
+          const uint64_t blo = smem_desc_sw128(bt + nb * b_tile, 16, 1024);
+          const uint64_t ad = me == 1 ? alo : ahi, bd = me == 2 ? blo : bhi;
+          const uint32_t d = tmem + (uint32_t)(me * BN);
 #pragma unroll
-        for (int j = 0; j < KCH / 8; ++j) {
-          if (PREC == 3) {
-            mma_tf32(d, alo + j * a_step, bhi + j * b_step, idesc, (i > 0 || j > 0) ? 1u : 0u);
-            mma_tf32(d, ahi + j * a_step, blo + j * b_step, idesc, 1u);
-            mma_tf32(d, ahi + j * a_step, bhi + j * b_step, idesc, 1u);
-          } else {
-            mma_tf32(d, ahi + j * a_step, bhi + j * b_step, idesc, (i > 0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < KCH / 8; ++j)
+            mma_tf32(d, ad + j * a_step, bd + j * b_step, idesc, (i > 0 || j > 0) ? 1u : 0u);
+        } else {
+          for (int jb = nb == 1 ? 0 : me; jb < nb; jb += NISS) {
+            const uint32_t bt = s0 + a_part + jb * b_tile;
+            const uint64_t bhi = smem_desc_sw128(bt, 16, 1024);
+            const uint32_t d = tmem + (uint32_t)((nb == 1 ? me : jb) * BN);
+            const bool first = nb == 1 ? i < 2 : i == 0;
+#pragma unroll
+            for (int j = 0; j < KCH / 8; ++j)
+              mma_tf32(d, ahi + j * a_step, bhi + j * b_step, idesc, (!first || j > 0) ? 1u : 0u);
           }
         }
+        mma_commit(smem_u32(&empty[st]));
       }
-      mma_commit(smem_u32(&empty[st]));
+      mma_commit(smem_u32(done));
     }
-    mma_commit(smem_u32(done));
   }
   if (KIND == KIND_OMAP && a.ks > 1) {
     // every CTA's partial tile is complete: finish this CTA's columns from the
@@ -571,7 +616,7 @@ cudaError_t launch_one(const TcMaps& maps, TcGemmArgs a, int grid_y, int nb, siz
   // keep the CTAs an SM can hold (228 KB of shared memory, 1 KB reserved per
   // CTA) within its 512 TMEM columns, so that no allocation ever waits
   int ncols = 32;
-  while (ncols < nb * BN) ncols <<= 1;
+  while (ncols < acc_plan(PREC, nb).nacc * BN) ncols <<= 1;
   const int max_ctas = 512 / ncols;
   const size_t floor_smem = (size_t)233472 / (max_ctas + 1) - 1024 + 16;
   if (smem < floor_smem) smem = floor_smem;
@@ -744,16 +789,8 @@ bool writer_tc_ok(const WriterArgs& w) {
 }
 
 int writer_tc_splits(const WriterArgs& w, int num_sms) {
-  const int bn = std::min(pick_bn(w.M), 128);
-  int tiles = 0, nk_min = 1 << 30;
-  for (int z = 0; z < w.Z; ++z) {
-    const Slice s = slice_of(w, z);
-    tiles += ((s.N + GM - 1) / GM) * ((w.M + bn - 1) / bn);
-    nk_min = std::min(nk_min, (s.K_outer * s.d_in + KCH - 1) / KCH);
-  }
-  int S = num_sms / std::max(tiles, 1);        // one wave of CTAs (one per SM)
-  S = std::min(S, std::max(1, nk_min / 4));   // at least four chunks per split
-  return std::max(1, std::min(S, 64));
+  (void)num_sms;
+  return writer_depth_splits(w);
 }
 
 cudaError_t launch_writer_tc(const WriterArgs& w, int* err, cudaStream_t st) {

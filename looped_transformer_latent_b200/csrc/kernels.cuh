@@ -27,6 +27,11 @@ struct WriterArgs {
   int* err;    // tensor-core phase: set on a timed-out wait; the stores are then NaN
 };
 size_t writer_workspace_floats(const WriterArgs& a);
+// k-split count of the writer: a function of the reduction depth only (one
+// split per 16 chunks of 32, at most 64), never of the number of tokens, so a
+// token's stored row is bit-identical whether it is written in a prefill
+// batch or alone (the streaming store of a token leaving the exact window).
+int writer_depth_splits(const WriterArgs& a);
 int writer_pick_splits(const WriterArgs& a, int num_sms);
 cudaError_t launch_writer(const WriterArgs& a, cudaStream_t st);
 // tensor-core writer phase 1 (gemm_tc.cu)

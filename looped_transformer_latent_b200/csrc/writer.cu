@@ -145,20 +145,19 @@ size_t writer_workspace_floats(const WriterArgs& a) {
 
 static bool small_batch(const WriterArgs& a) { return a.M <= 32; }
 
+int writer_depth_splits(const WriterArgs& a) {
+  int nk_max = 1;
+  for (int z = 0; z < a.Z; ++z) {
+    const Slice s = slice_of(a, z);
+    nk_max = nk_max > ceil_div(s.K_outer * s.d_in, BK) ? nk_max : ceil_div(s.K_outer * s.d_in, BK);
+  }
+  const int S = ceil_div(nk_max, 16);
+  return S < 1 ? 1 : S > 64 ? 64 : S;
+}
+
 int writer_pick_splits(const WriterArgs& a, int num_sms) {
-  // about four CTAs per SM; never more splits than k-chunks
-  const int tm = small_batch(a) ? 32 : 64, tn = small_batch(a) ? 128 : 64;
-  const int tiles = ceil_div(a.Nmax, tn) * ceil_div(a.M, tm) * a.Z;
-  int K = 0;
-  if (a.mode == LLA_WRITE_HLA) K = a.D;  // smallest GEMM depth (loop-1)
-  else if (a.mode == LLA_WRITE_PERHEAD) K = a.T * a.d_h;
-  else K = a.T * a.H * a.d_h;
-  const int nk = ceil_div(K, BK);
-  int S = ceil_div(4 * num_sms, tiles > 0 ? tiles : 1);
-  if (S > nk) S = nk;
-  if (S > 96) S = 96;
-  if (S < 1) S = 1;
-  return S;
+  (void)num_sms;
+  return writer_depth_splits(a);
 }
 
 cudaError_t launch_writer(const WriterArgs& a_in, cudaStream_t st) {

@@ -27,6 +27,7 @@ Modules:
 * ``rope``     -- the rotary operator R at any even dimension, with the
                   frequency-aligned pairing of latent dimensions.
 * ``rounding`` -- IEEE round-to-nearest-even to bf16 / fp32 storage.
+* ``quant``    -- fp8 (e4m3) latent rows with per-token, per-part scales.
 * ``hla``      -- HLA latent writer (eq. 2) and absorbed read (eqs. 3-4), plus
                   the reconstruct-then-attend form used by invariants.
 * ``lla``      -- LLA per-head / LLA-2D writers, LLA reconstruct-on-read, and
@@ -47,4 +48,4 @@ with same-frequency pair combinations, a window covering the context is exact
 attention).  No function is "parity unpinned".
 """
 
-from . import rope, rounding, hla, lla, exact, codec  # noqa: F401
+from . import rope, rounding, quant, hla, lla, exact, codec  # noqa: F401

@@ -39,9 +39,17 @@ CONFIGS = {
     # Huginn-3.5B-like LLA per-head reconstruct-on-read, 32 loops, rank 96
     "huginn_lla_4k": ConfigShape("huginn_lla_4k", "lla", B=16, L=1, T=32, H=55, d_h=96, D=0,
                                  N=4096, W=0, r_k=96, r_v=96, r_1=0, lat_dtype="bf16"),
+    # the same under the served semantics: an exact window of the last 64 tokens
+    # (plus the current one), latents for older tokens only
+    "huginn_lla_4k_w64": ConfigShape("huginn_lla_4k_w64", "lla", B=16, L=1, T=32, H=55, d_h=96, D=0,
+                                     N=4096, W=64, r_k=96, r_v=96, r_1=0, lat_dtype="bf16"),
     # capacity regime: Ouro-shaped LLA-2D, batch 768, absorbed read, no window
     "ouro_lla2d_768": ConfigShape("ouro_lla2d_768", "lla2d", B=768, L=24, T=4, H=16, d_h=128, D=0,
                                   N=4096, W=0, r_k=576, r_v=576, r_1=0, lat_dtype="bf16"),
+    # the same at the printed 21.3x compression: 768 numbers per token and
+    # layer (r_K = r_V = 384) instead of the configured 1152
+    "ouro_lla2d_768_r384": ConfigShape("ouro_lla2d_768_r384", "lla2d", B=768, L=24, T=4, H=16, d_h=128,
+                                       D=0, N=4096, W=0, r_k=384, r_v=384, r_1=0, lat_dtype="bf16"),
     # long-context HLA, 16k, batch 64
     "ouro_hla_16k": ConfigShape("ouro_hla_16k", "hla", B=64, L=24, T=4, H=16, d_h=128, D=2048,
                                 N=16384, W=128, r_k=512, r_v=512, r_1=256, lat_dtype="bf16"),

@@ -91,16 +91,18 @@ def test_ouro_hla_16k_reads(cuda_device, group):
     print(f"ouro_hla_16k {group}: rel L2 (pooled, worst row) {errs}")
 
 
-def test_ouro_lla2d_768_absorbed_read(cuda_device):
-    c = synth.CONFIGS["ouro_lla2d_768"]
+@pytest.mark.parametrize("name", ["ouro_lla2d_768", "ouro_lla2d_768_r384"])
+def test_ouro_lla2d_768_absorbed_read(cuda_device, name):
+    c = synth.CONFIGS[name]
     errs = _absorbed_full(cuda_device, 13, c.B, c.N, 0, c.H, nt=c.T, t0=0, T=c.T, d_h=c.d_h, r_k=c.r_k,
                           r_v=c.r_v, rotate=False, samples=[0, 400, c.B - 1])
-    print(f"ouro_lla2d_768: rel L2 (pooled, worst row) {errs}")
+    print(f"{name}: rel L2 (pooled, worst row) {errs}")
 
 
-def test_huginn_lla_4k_reconstruct(cuda_device):
-    c = synth.CONFIGS["huginn_lla_4k"]
-    B, H, N, r, T, d_h = c.B, c.H, c.N, c.r_k, c.T, c.d_h
+@pytest.mark.parametrize("name", ["huginn_lla_4k", "huginn_lla_4k_w64"])
+def test_huginn_lla_4k_reconstruct(cuda_device, name):
+    c = synth.CONFIGS[name]
+    B, H, N, r, T, d_h, W = c.B, c.H, c.N, c.r_k, c.T, c.d_h, c.W
     g = torch.Generator().manual_seed(14)
     ndist = 2
     cK_d = torch.randn(ndist, H, N, r, generator=g).to(torch.bfloat16)
@@ -108,13 +110,13 @@ def test_huginn_lla_4k_reconstruct(cuda_device):
     UK = torch.randn(T, H, d_h, r, generator=g) / math.sqrt(r)
     UV = torch.randn(T, H, d_h, r, generator=g) / math.sqrt(r)
     q = torch.randn(B, T, H, d_h, generator=g)
-    wk_d = torch.randn(ndist, T, 1, H, d_h, generator=g).to(torch.bfloat16)
-    wv_d = torch.randn(ndist, T, 1, H, d_h, generator=g).to(torch.bfloat16)
+    wk_d = torch.randn(ndist, T, W + 1, H, d_h, generator=g).to(torch.bfloat16)
+    wv_d = torch.randn(ndist, T, W + 1, H, d_h, generator=g).to(torch.bfloat16)
     dev = cuda_device
     out = torch.full((B, T, H, d_h), float("nan"), device=dev)
     L.lla_decode_attn(cK=_tile_batch(cK_d, B, dev), cV=_tile_batch(cV_d, B, dev), UK=UK.to(dev),
                       UV=UV.to(dev), q=q.to(dev), win_k=_tile_batch(wk_d, B, dev),
-                      win_v=_tile_batch(wv_d, B, dev), out=out, N=N, W=0, t0=0)
+                      win_v=_tile_batch(wv_d, B, dev), out=out, N=N, W=W, t0=0)
     torch.cuda.synchronize()
     assert torch.isfinite(out).all()
     errs = []
@@ -122,9 +124,9 @@ def test_huginn_lla_4k_reconstruct(cuda_device):
         k = b % ndist
         ref = lla.decode_reconstruct(f64(cK_d[k][h:h + 1]), f64(cV_d[k][h:h + 1]), f64(UK[:, h:h + 1]),
                                      f64(UV[:, h:h + 1]), f64(q[b][:, h:h + 1]), f64(wk_d[k][:, :, h:h + 1]),
-                                     f64(wv_d[k][:, :, h:h + 1]), 0, N, 0)
+                                     f64(wv_d[k][:, :, h:h + 1]), 0, N, W)
         errs.append(assert_rows_close(out[b][:, h:h + 1], ref, TOL_BF16, f"sequence {b} head {h}"))
-    print(f"huginn_lla_4k: rel L2 (pooled, worst row) {errs}")
+    print(f"{name}: rel L2 (pooled, worst row) {errs}")
 
 
 def test_decode_step_writers_at_full_batch(cuda_device):

@@ -381,3 +381,60 @@ def test_lla2d_writer_then_absorbed_read(cuda_device):
                                        0, N, W, rK, rV))
     err = assert_rows_close(out, np.stack(ref), TOL_BF16, "lla2d end to end")
     print(f"lla2d end to end rel L2 (pooled, worst row) {err}")
+
+
+# ------------------------------------- streaming store = prefill rows --
+STREAM_CASES = [
+    # mode, dtype
+    (L.LLA_WRITE_PERHEAD, torch.bfloat16),
+    (L.LLA_WRITE_PERHEAD, torch.float32),
+    (L.LLA_WRITE_FOLDED, torch.bfloat16),
+    (L.LLA_WRITE_HLA, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("mode,dtype", STREAM_CASES)
+def test_streaming_store_matches_prefill_rows(cuda_device, mode, dtype):
+    """Served semantics (LLA abstract, streaming latent store): the latent of
+    a token written alone when it leaves the exact window -- one call with
+    n = 1 at pos0 = j -- must be bit-identical to the row the prefill writer
+    stored for it in a call over many tokens, since the read cannot tell which
+    of the two wrote it."""
+    g = _gen(90 + mode)
+    dev = cuda_device
+    B, n, T, H, d_h = 3, 200, 4, 5, 64
+    if mode == L.LLA_WRITE_HLA:
+        D, r_k, r_v, r_1 = 256, 128, 96, 64
+        h = torch.randn(B, n, T, D, generator=g)
+        E = torch.randn(T - 1, r_k + r_v, D, generator=g) / math.sqrt(D)
+        E1 = torch.randn(2 * r_1, D, generator=g) / math.sqrt(D)
+        kw = dict(E_main=E.to(dev), E_1=E1.to(dev), r_k=r_k, d_h=d_h, rope_base=BASE)
+        outs = lambda: (torch.zeros(B, n, r_k + r_v, dtype=dtype, device=dev),  # noqa: E731
+                        torch.zeros(B, n, 2 * r_1, dtype=dtype, device=dev))
+        args = lambda j0, j1: dict(x=h[:, j0:j1].contiguous().to(dev))  # noqa: E731
+    else:
+        r = 96 if mode == L.LLA_WRITE_PERHEAD else 160
+        k = torch.randn(B, n, T, H, d_h, generator=g)
+        v = torch.randn(B, n, T, H, d_h, generator=g)
+        EK = torch.randn(T, H, r, d_h, generator=g) / math.sqrt(T * d_h)
+        EV = torch.randn(T, H, r, d_h, generator=g) / math.sqrt(T * d_h)
+        kw = dict(E_K=EK.to(dev), E_V=EV.to(dev))
+        if mode == L.LLA_WRITE_PERHEAD:
+            outs = lambda: (torch.zeros(B, H, n, r, dtype=dtype, device=dev),  # noqa: E731
+                            torch.zeros(B, H, n, r, dtype=dtype, device=dev))
+        else:
+            outs = lambda: (torch.zeros(B, n, 2 * r, dtype=dtype, device=dev), None)  # noqa: E731
+        args = lambda j0, j1: dict(x=k[:, j0:j1].contiguous().to(dev),  # noqa: E731
+                                   xv=v[:, j0:j1].contiguous().to(dev))
+    pre0, pre1 = outs()
+    L.lla_write_latents(mode, out0=pre0, out1=pre1, pos0=0, **args(0, n), **kw)
+    one0, one1 = outs()
+    picks = [0, 1, 77, n - 1]
+    for j in picks:
+        L.lla_write_latents(mode, out0=one0, out1=one1, pos0=j, **args(j, j + 1), **kw)
+    torch.cuda.synchronize()
+    tok = (lambda t, j: t[:, :, j]) if mode == L.LLA_WRITE_PERHEAD else (lambda t, j: t[:, j])
+    for j in picks:
+        assert torch.equal(tok(one0, j), tok(pre0, j)), f"row {j} differs"
+        if one1 is not None:
+            assert torch.equal(tok(one1, j), tok(pre1, j)), f"row {j} (second latent) differs"
