@@ -94,7 +94,19 @@ typedef enum {
   LLA_ERR_CUDA = 7         /* a CUDA runtime call or launch failed           */
 } lla_status;
 
-typedef enum { LLA_F32 = 0, LLA_BF16 = 1 } lla_dtype;
+/* Storage formats.  LLA_FP8_E4M3 is a latent-row format, not an element
+ * type: each token's row holds the e4m3 codes (OCP FP8 E4M3: bias 7, 3
+ * mantissa bits, largest finite 448) of its key part and of its value part,
+ * then the two parts' fp32 scales and 8 zero bytes:
+ *   [codes of c^K: r_k bytes | codes of c^V: r_v bytes | s^K | s^V | 0 x 8]
+ * so a row is r_k + r_v + 16 bytes and element (byte) strides apply.  A
+ * stored element's value is code * s of its part; s = (largest magnitude of
+ * the part) / 448, codes rounded to nearest-even and saturated (HLA summary,
+ * "Conclusion / Future directions": combining the latents with quantisation;
+ * per-token, per-part scales are this library's reading).  Written by
+ * lla_write_latents (HLA and FOLDED modes) and read by hla_decode_attn on the
+ * tensor cores (codes widened exactly to f16). */
+typedef enum { LLA_F32 = 0, LLA_BF16 = 1, LLA_FP8_E4M3 = 2 } lla_dtype;
 
 /* Version of this ABI; bumped whenever a struct below changes. */
 int lla_abi_version(void);
@@ -153,7 +165,9 @@ typedef struct {
    *   FOLDED:  out0 = [B, Ncap, r_k + r_v]; out1 unused.
    * Rows must start 16-byte aligned.                                       */
   void *out0, *out1;
-  int32_t out_dtype;       /* lla_dtype of both outputs                        */
+  int32_t out_dtype;       /* lla_dtype of both outputs; LLA_FP8_E4M3 rows
+                              (HLA and FOLDED only) are r_k + r_v + 16 bytes
+                              (HLA loop-1: 2 r_1 + 16) and strides in bytes   */
   int32_t Ncap;            /* cache rows per sequence; pos0 + n <= Ncap        */
   int64_t out_stride_b, out_stride_h, out_stride_n;
   int64_t out1_stride_b, out1_stride_n; /* HLA loop-1 latent                   */
@@ -231,7 +245,8 @@ typedef struct {
   int32_t T, t0, nt;       /* loops in the model; this call serves t0..t0+nt-1 */
   int32_t N, W;            /* context length (query at N-1), exact window      */
   int32_t r_k, r_v;        /* key and value ranks of this latent               */
-  const void *lat;         /* [B, >= N-1-W rows, r_k + r_v], lat_dtype         */
+  const void *lat;         /* [B, >= N-1-W rows, r_k + r_v], lat_dtype; for
+                              LLA_FP8_E4M3 rows of r_k + r_v + 16 bytes        */
   int32_t lat_dtype;
   int64_t lat_stride_b, lat_stride_n;
   const float *A;          /* [nt, H, d_h, r_k] fp32                           */
@@ -252,6 +267,15 @@ typedef struct {
    * stream capture), so a caller can time that kernel alone.  Nothing else
    * changes; no work is skipped. */
   void *timing_events;
+  /* Query positions served at once (0 or 1: the decode read of position
+   * N - 1).  With nq > 1 the call serves the last nq positions of the context,
+   * i_p = N - nq + p (a prefill chunk, or a block of the two-pass procedure's
+   * parallel second pass; HLA summary, "Methodology / Fine-tuning"): q and out
+   * are [B, nq, nt, H, d_h], row (p, t, h) attends to latent tokens
+   * j < i_p - W and to exact tokens max(0, i_p - W) <= j <= i_p of the ring
+   * (Wcap >= min(N, W + nq)), and every latent tile is shared by all
+   * nq * nt * H rows on the tensor cores (at most 64 rows; bf16 or fp8 rows). */
+  int32_t nq;
 } hla_decode_params;
 
 size_t hla_decode_workspace_bytes(const hla_decode_params *p);

@@ -17,7 +17,7 @@ Entry points (names as in the C ABI):
 import ctypes
 
 from . import _abi
-from ._abi import (LLA_BF16, LLA_F32, LLA_WRITE_FOLDED, LLA_WRITE_HLA,  # noqa: F401
+from ._abi import (LLA_BF16, LLA_F32, LLA_FP8_E4M3, LLA_WRITE_FOLDED, LLA_WRITE_HLA,  # noqa: F401
                    LLA_WRITE_PERHEAD, LibraryMissing)
 
 __all__ = [
@@ -61,7 +61,17 @@ def _dtype_code(t):
         return LLA_F32
     if t.dtype == torch.bfloat16:
         return LLA_BF16
-    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+    if t.dtype == torch.uint8:
+        return LLA_FP8_E4M3          # byte rows: e4m3 codes, then the two fp32 scales and 8 zero bytes
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32, bfloat16 or uint8 (fp8 rows)")
+
+
+FP8_ROW_EXTRA = 16   # bytes after the codes of an fp8 row: s^K, s^V (fp32), 8 zero bytes
+
+
+def _row_width(t):
+    """Elements of one latent row: the codes only, for fp8 byte rows."""
+    return t.shape[-1] - (FP8_ROW_EXTRA if t.dtype == _torch().uint8 else 0)
 
 
 def _ptr(t):
@@ -128,7 +138,7 @@ def _write_params(mode, x, xv, E_main, E_1, E_K, E_V, out0, out1, pos0, d_h, r_k
         B, n, T, D = x.shape
         _dense_inner(x, 1, "h")
         p.B, p.n, p.T, p.D, p.H, p.d_h = B, n, T, D, 1, d_h
-        p.r_k, p.r_v, p.r_1 = r_k, out0.shape[-1] - r_k, out1.shape[-1] // 2
+        p.r_k, p.r_v, p.r_1 = r_k, _row_width(out0) - r_k, _row_width(out1) // 2
         p.out_stride_b, p.out_stride_n = out0.stride(0), out0.stride(1)
         p.out1_stride_b, p.out1_stride_n = out1.stride(0), out1.stride(1)
         p.Ncap = min(out0.shape[1], out1.shape[1])
@@ -233,11 +243,18 @@ def _events(p, timing_events):
 def _hla_params(lat, A, Bm, q, win_k, win_v, out, N, W, t0, r_k, rotate_query, rope_base, scale,
                 timing_events=None):
     p = _abi.HlaDecodeParams()
-    B, nt, H, d_h = q.shape
-    _dense_inner(q, 3, "q")
-    _dense_inner(out, 3, "out")
-    if tuple(out.shape) != (B, nt, H, d_h):
+    if q.dim() == 5:                       # [B, nq, nt, H, d_h]: the last nq positions at once
+        B, nq, nt, H, d_h = q.shape
+        _dense_inner(q, 4, "q")
+        _dense_inner(out, 4, "out")
+    else:
+        B, nt, H, d_h = q.shape
+        nq = 1
+        _dense_inner(q, 3, "q")
+        _dense_inner(out, 3, "out")
+    if tuple(out.shape) != tuple(q.shape):
         raise ValueError("out must have q's shape")
+    p.nq = nq
     for t, nm in ((A, "A"), (Bm, "Bm")):
         if not t.is_contiguous() or t.dtype != _torch().float32:
             raise ValueError(f"{nm} must be a contiguous float32 tensor")
@@ -283,10 +300,11 @@ def _hla_kw(kw):
 def hla_decode_attn(*, workspace=None, stream=None, **kw):
     """Absorbed latent read (HLA eqs. 3-4, or LLA-D with rotate_query=False).
 
-    lat [B,Ncap,r_k+r_v] (key part stored as R~_j c^K_j), A [nt,H,d_h,r_k],
-    Bm [nt,H,r_v,d_h], q [B,nt,H,d_h], ring win_k/win_v [B,T,Wcap,H,d_h],
-    out [B,nt,H,d_h] float32; N = context length, W = exact window, t0 = first
-    loop served.
+    lat [B,Ncap,r_k+r_v] (key part stored as R~_j c^K_j; bf16, float32, or
+    uint8 fp8 rows of r_k+r_v+16 bytes), A [nt,H,d_h,r_k], Bm [nt,H,r_v,d_h],
+    q [B,nt,H,d_h] (or [B,nq,nt,H,d_h]: the last nq positions of the context
+    at once), ring win_k/win_v [B,T,Wcap,H,d_h], out shaped like q, float32;
+    N = context length, W = exact window, t0 = first loop served.
     """
     args = _hla_kw(kw)
     dev = _cuda(args["lat"], args["A"], args["Bm"], args["q"], args["win_k"], args["win_v"], args["out"])

@@ -21,6 +21,7 @@ LLA_ERR_CUDA = 7
 
 LLA_F32 = 0
 LLA_BF16 = 1
+LLA_FP8_E4M3 = 2
 
 LLA_WRITE_HLA = 0
 LLA_WRITE_PERHEAD = 1
@@ -91,6 +92,7 @@ class HlaDecodeParams(ctypes.Structure):
         ("out_stride_b", c_i64),
         ("scale", c_f32),
         ("timing_events", c_vp),
+        ("nq", c_i32),
     ]
 
 

@@ -17,7 +17,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblla.so")
 
-SOURCES = ["abi.cu", "writer.cu", "decode_simt.cu", "decode_tc.cu", "maps.cu", "gemm_tc.cu", "recon_tc.cu", "noalloc.cu"]
+SOURCES = ["abi.cu", "writer.cu", "decode_simt.cu", "decode_tc.cu", "decode_fp8.cu", "maps.cu", "gemm_tc.cu",
+           "recon_tc.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -9,7 +9,7 @@
 namespace lla {
 namespace {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 3;   // 2: LLA_FP8_E4M3 latent rows; 3: hla_decode_params.nq
 constexpr int kDefaultSms = 148;        // B200; used only when no device can be queried
 constexpr int kMaxDevices = 64;
 constexpr size_t kAlign = 256;
@@ -38,8 +38,10 @@ int num_sms() {
 }
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-inline size_t elem_size(int dt) { return dt == LLA_BF16 ? 2 : 4; }
-inline bool dtype_ok(int dt) { return dt == LLA_F32 || dt == LLA_BF16; }
+inline size_t elem_size(int dt) { return dt == LLA_BF16 ? 2 : dt == LLA_FP8_E4M3 ? 1 : 4; }
+inline bool dtype_ok(int dt) { return dt == LLA_F32 || dt == LLA_BF16; }          // element types
+inline bool lat_dtype_ok(int dt) { return dtype_ok(dt) || dt == LLA_FP8_E4M3; }   // latent row formats
+constexpr int kFp8Extra = 16;   // fp8 rows: s^K, s^V (fp32) and 8 zero bytes after the codes
 inline size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Carve {
@@ -55,12 +57,14 @@ inline int ring_ok(int W, int N, int Wcap) {
 // --------------------------------------------------------------- writer --
 int check_write(const lla_write_params& p) {
   if (p.B < 0 || p.n < 0 || p.pos0 < 0 || p.Ncap < 0) return LLA_ERR_SHAPE;
-  if (!dtype_ok(p.out_dtype)) return LLA_ERR_DTYPE;
+  if (!lat_dtype_ok(p.out_dtype)) return LLA_ERR_DTYPE;
+  const bool fp8 = p.out_dtype == LLA_FP8_E4M3;
+  if (fp8 && p.mode == LLA_WRITE_PERHEAD) return LLA_ERR_UNSUPPORTED;   // fp8 rows feed the absorbed read
   if (p.mode != LLA_WRITE_HLA && p.mode != LLA_WRITE_PERHEAD && p.mode != LLA_WRITE_FOLDED)
     return LLA_ERR_UNSUPPORTED;
   if (p.T < 1 || p.H < 1 || p.d_h < 2) return LLA_ERR_SHAPE;
   if ((long)p.pos0 + p.n > p.Ncap) return LLA_ERR_SHAPE;
-  const int mult = p.out_dtype == LLA_BF16 ? 8 : 4;
+  const int mult = p.out_dtype == LLA_BF16 ? 8 : fp8 ? 16 : 4;
   if (p.mode == LLA_WRITE_HLA) {
     if (p.T < 2 || p.D < 16 || p.D % 16) return LLA_ERR_SHAPE;
     if (p.r_k < 2 || p.r_v < 1 || p.r_1 < 1) return LLA_ERR_SHAPE;
@@ -88,11 +92,13 @@ int check_write(const lla_write_params& p) {
   if (p.x_stride_b < 0 || p.x_stride_n < 0 || p.x_stride_t < 0) return LLA_ERR_SHAPE;
   const int64_t row = p.mode == LLA_WRITE_HLA ? (int64_t)p.D : (int64_t)p.H * p.d_h;
   if (p.x_stride_t < row) return LLA_ERR_SHAPE;
+  const int extra = fp8 ? kFp8Extra : 0;
+  if (fp8 && (p.r_k + p.r_v > 2048 || 2 * p.r_1 > 2048)) return LLA_ERR_UNSUPPORTED;
   if (p.mode == LLA_WRITE_HLA) {
-    if (p.out_stride_n < p.r_k + p.r_v || p.out1_stride_n < 2 * p.r_1) return LLA_ERR_SHAPE;
+    if (p.out_stride_n < p.r_k + p.r_v + extra || p.out1_stride_n < 2 * p.r_1 + extra) return LLA_ERR_SHAPE;
   } else if (p.mode == LLA_WRITE_PERHEAD) {
     if (p.out_stride_n < p.r_k) return LLA_ERR_SHAPE;
-  } else if (p.out_stride_n < p.r_k + p.r_v) {
+  } else if (p.out_stride_n < p.r_k + p.r_v + extra) {
     return LLA_ERR_SHAPE;
   }
   return LLA_OK;
@@ -119,8 +125,8 @@ WriterArgs writer_args(const lla_write_params& p) {
     a.Z = 2; a.Nmax = std::max(p.r_k, p.r_v);
   }
   a.Nmax += a.Nmax % 2;
-  // tensor cores (3xTF32, fp32-accurate) when the rows are stored as bf16
-  a.use_tc = p.out_dtype == LLA_BF16 && writer_tc_ok(a);
+  // tensor cores (3xTF32, fp32-accurate) when the rows are stored as bf16 or fp8
+  a.use_tc = p.out_dtype != LLA_F32 && writer_tc_ok(a);
   const int sms = num_sms();
   a.S = a.use_tc ? writer_tc_splits(a, sms) : writer_pick_splits(a, sms);
   return a;
@@ -128,30 +134,39 @@ WriterArgs writer_args(const lla_write_params& p) {
 
 // ------------------------------------------------------- decode checks --
 int check_hla(const hla_decode_params& p) {
-  if (p.B < 0 || p.nt < 0) return LLA_ERR_SHAPE;
-  if (!dtype_ok(p.lat_dtype) || !dtype_ok(p.win_dtype)) return LLA_ERR_DTYPE;
+  if (p.B < 0 || p.nt < 0 || p.nq < 0) return LLA_ERR_SHAPE;
+  const int nq = p.nq > 1 ? p.nq : 1;
+  if (!lat_dtype_ok(p.lat_dtype) || !dtype_ok(p.win_dtype)) return LLA_ERR_DTYPE;
   if (p.H < 1 || p.d_h < 4 || p.d_h % 4 || p.T < 1 || p.t0 < 0 || p.t0 + p.nt > p.T) return LLA_ERR_SHAPE;
   if (p.N < 1 || p.W < 0 || p.r_k < 2 || p.r_k % 2 || p.r_v < 1) return LLA_ERR_SHAPE;
+  const bool fp8 = p.lat_dtype == LLA_FP8_E4M3;
+  if (fp8 && !absorb_fp8_supported(p.r_k, p.r_v, p.nt * p.H)) return LLA_ERR_UNSUPPORTED;
   if (p.d_h > 128) return LLA_ERR_UNSUPPORTED;
   if (p.r_v > 1024 || p.r_k + p.r_v > 2048) return LLA_ERR_UNSUPPORTED;
-  if ((long)p.nt * p.H > 65535) return LLA_ERR_UNSUPPORTED;
-  if (!ring_ok(p.W, p.N, p.Wcap)) return LLA_ERR_SHAPE;
+  if ((long)nq * p.nt * p.H > 65535) return LLA_ERR_UNSUPPORTED;
+  if (p.N < nq) return LLA_ERR_SHAPE;
+  if (nq == 1 ? !ring_ok(p.W, p.N, p.Wcap) : (long)p.Wcap < std::min<long>(p.N, (long)p.W + nq)) return LLA_ERR_SHAPE;
   if (!std::isfinite(p.scale) || p.scale < 0.f) return LLA_ERR_SHAPE;
   if (p.B == 0 || p.nt == 0) return LLA_OK;
   const int n_lat = std::max(0, p.N - 1 - p.W);
   if (!p.A || !p.Bm || !p.q || !p.win_k || !p.win_v || !p.out) return LLA_ERR_NULL;
   if (n_lat > 0 && !p.lat) return LLA_ERR_NULL;
+  // several positions share the tensor-core read (bf16 or fp8 rows, <= 64 rows)
+  if (nq > 1 && n_lat > 0 &&
+      !(p.lat_dtype == LLA_FP8_E4M3 ? absorb_fp8_supported(p.r_k, p.r_v, nq * p.nt * p.H)
+                                    : absorb_tc_supported(p.lat_dtype, p.r_k, p.r_v, nq * p.nt * p.H)))
+    return LLA_ERR_UNSUPPORTED;
   const size_t es = elem_size(p.lat_dtype);
   if (n_lat > 0) {
     if (!aligned(p.lat, 16) || (p.lat_stride_b * es) % 16 || (p.lat_stride_n * es) % 16) return LLA_ERR_ALIGN;
     if (((size_t)(p.r_k + p.r_v) * es) % 16 || ((size_t)p.r_k * es) % 16) return LLA_ERR_ALIGN;
-    if (p.lat_stride_n < p.r_k + p.r_v || p.lat_stride_b < 0) return LLA_ERR_SHAPE;
+    if (p.lat_stride_n < p.r_k + p.r_v + (fp8 ? kFp8Extra : 0) || p.lat_stride_b < 0) return LLA_ERR_SHAPE;
   }
   if (!aligned(p.A, 16) || !aligned(p.Bm, 16) || p.r_k % 4) return LLA_ERR_ALIGN;
   if (!aligned(p.q, 4) || !aligned(p.out, 4)) return LLA_ERR_ALIGN;
   if (!aligned(p.win_k, 16) || !aligned(p.win_v, 16)) return LLA_ERR_ALIGN;
   if ((p.win_stride_b * elem_size(p.win_dtype)) % 16) return LLA_ERR_ALIGN;
-  const int64_t rowlen = (int64_t)p.nt * p.H * p.d_h;
+  const int64_t rowlen = (int64_t)nq * p.nt * p.H * p.d_h;
   if (p.q_stride_b < rowlen || p.out_stride_b < rowlen) return LLA_ERR_SHAPE;
   if (p.win_stride_b < (int64_t)p.T * p.Wcap * p.H * p.d_h) return LLA_ERR_SHAPE;
   return LLA_OK;
@@ -159,7 +174,8 @@ int check_hla(const hla_decode_params& p) {
 
 int check_lla(const lla_decode_params& p) {
   if (p.B < 0 || p.nt < 0) return LLA_ERR_SHAPE;
-  if (!dtype_ok(p.lat_dtype) || !dtype_ok(p.win_dtype)) return LLA_ERR_DTYPE;
+  if (!lat_dtype_ok(p.lat_dtype) || !dtype_ok(p.win_dtype)) return LLA_ERR_DTYPE;
+  if (p.lat_dtype == LLA_FP8_E4M3) return LLA_ERR_UNSUPPORTED;   // fp8 rows are read by the absorbed read
   if (p.H < 1 || p.d_h < 4 || p.d_h % 4 || p.T < 1 || p.t0 < 0 || p.t0 + p.nt > p.T) return LLA_ERR_SHAPE;
   if (p.N < 1 || p.W < 0 || p.r < 1) return LLA_ERR_SHAPE;
   if (p.d_h > 128 || p.r > 128) return LLA_ERR_UNSUPPORTED;
@@ -197,12 +213,13 @@ HlaPlan plan_hla(const hla_decode_params& p) {
   const int sms = num_sms();
   const long target_ctas = 4L * sms;   // SIMT split heuristic: about four CTAs per SM
   // SIMT split: one CTA per (split, sequence, 16 rows)
-  pl.rows = p.nt * p.H;
+  pl.rows = (p.nq > 1 ? p.nq : 1) * p.nt * p.H;
   const int i = p.N - 1;
   pl.n_lat = std::max(0, i - p.W);
   pl.win_start = pl.n_lat;
   pl.n_win = i - pl.win_start + 1;
-  pl.use_tc = pl.n_lat > 0 && absorb_tc_supported(p.lat_dtype, p.r_k, p.r_v, pl.rows);
+  pl.use_tc = pl.n_lat > 0 && (p.lat_dtype == LLA_FP8_E4M3 ? absorb_fp8_supported(p.r_k, p.r_v, pl.rows)
+                                                             : absorb_tc_supported(p.lat_dtype, p.r_k, p.r_v, pl.rows));
   pl.rows_pad = pl.use_tc ? absorb_tc_rows_pad(pl.rows) : pl.rows;
   if (pl.use_tc) {
     // tensor-core read: one CTA per (split, sequence), 64-token tiles
@@ -373,38 +390,50 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
   a.use_tc = pl.use_tc; a.rows_pad = pl.rows_pad;
   a.qbf = reinterpret_cast<__nv_bfloat16*>(w + pl.o_qbf);
   a.err = reinterpret_cast<int*>(w + pl.o_err);
+  const int nq = p->nq > 1 ? p->nq : 1;
+  const int rows_q = p->nt * p->H;     // rows of one query position
+  a.nq = nq; a.rows_per_q = rows_q;
 
   MapArgs qm;
   std::memset(&qm, 0, sizeof(qm));
   qm.B = a.B; qm.rows = a.rows; qm.K = a.d_h; qm.N = a.r_k; qm.d_h = a.d_h;
   qm.W = a.A; qm.X = a.q; qm.xs_b = a.qs_b; qm.xs_row = a.d_h;
-  qm.rotate = a.rotate; qm.pos = a.N - 1; qm.use_tc = a.use_tc; qm.base = a.base; qm.qmul = a.qmul;
+  qm.rotate = a.rotate; qm.pos = a.N - nq; qm.use_tc = a.use_tc; qm.base = a.base; qm.qmul = a.qmul;
+  if (nq > 1) { qm.ncodec = rows_q; qm.rows_per_q = rows_q; }   // position of row g: N - nq + g / rows_q
+  qm.q_f16 = a.lat_dtype == LLA_FP8_E4M3 && a.use_tc;   // no latent token: the operand is unused
   qm.qlat = a.qlat; qm.qbf = a.qbf;
   cudaError_t e = cudaSuccess;
   e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
   if (e == cudaSuccess) {
     // tensor-core map when the shapes allow a tensor-map view, else the SIMT map
     e = query_map_tc_ok(qm) ? launch_query_map_tc(qm, a.err, s) : cudaErrorNotSupported;
-    if (e == cudaErrorNotSupported) e = launch_query_map(qm, s);
+    // the SIMT map writes bf16 only; fp8 rows need the tensor-core map's f16 operand
+    if (e == cudaErrorNotSupported && !qm.q_f16) e = launch_query_map(qm, s);
   }
   if (e == cudaSuccess) e = mark(p->timing_events, 0, s);
   if (e == cudaSuccess && a.n_lat > 0)
-    e = a.use_tc ? launch_absorb_split_tc(a, s) : launch_absorb_split_simt(a, s);
+    e = a.lat_dtype == LLA_FP8_E4M3 ? launch_absorb_split_fp8(a, s)
+        : a.use_tc ? launch_absorb_split_tc(a, s) : launch_absorb_split_simt(a, s);
   if (e == cudaSuccess) e = mark(p->timing_events, 1, s);
-  if (e == cudaSuccess) {
+  // exact window: one launch per query position p (its own tokens and R_i)
+  for (int qp = 0; qp < nq && e == cudaSuccess; ++qp) {
+    const int ip = a.N - nq + qp;
     WindowArgs wa;
-    wa.B = a.B; wa.rows = a.rows; wa.H = a.H; wa.d_h = a.d_h; wa.t0 = a.t0; wa.Wcap = a.Wcap;
-    wa.win_start = a.win_start; wa.n_win = a.n_win; wa.Sw = a.Sw; wa.cpt = a.cpt; wa.HG = pl.HG;
+    wa.B = a.B; wa.rows = rows_q; wa.H = a.H; wa.d_h = a.d_h; wa.t0 = a.t0; wa.Wcap = a.Wcap;
+    wa.win_start = std::max(0, ip - a.W); wa.n_win = ip - wa.win_start + 1;
+    wa.Sw = a.Sw; wa.cpt = a.cpt; wa.HG = pl.HG;
     wa.wk = a.wk; wa.wv = a.wv; wa.dtype = a.win_dtype; wa.wins_b = a.wins_b;
     wa.q = a.q; wa.q_sb = a.qs_b; wa.q_srow = a.d_h; wa.qmul = a.qmul;
-    wa.rotate = a.rotate; wa.pos = a.N - 1; wa.base = a.base;
+    wa.rotate = a.rotate; wa.pos = ip; wa.base = a.base;
     wa.win_ml = a.win_ml; wa.win_y = a.win_y; wa.err = a.err;
+    wa.rows_total = a.rows; wa.row0 = qp * rows_q;
     e = launch_window(wa, s);
   }
   if (e == cudaSuccess) {
     MapArgs om;
     std::memset(&om, 0, sizeof(om));
     om.B = a.B; om.rows = a.rows; om.K = a.r_v; om.N = a.d_h; om.d_h = a.d_h; om.W = a.Bm;
+    if (nq > 1) om.ncodec = rows_q;
     om.part_ml = a.part_ml; om.part_y = a.part_y; om.win_ml = a.win_ml; om.win_y = a.win_y; om.S = a.S;
     om.Sw = a.Sw;
     om.out = a.out; om.outs_b = a.outs_b; om.err = a.err;
@@ -463,6 +492,7 @@ int lla_decode_attn(const lla_decode_params* p, void* ws, size_t ws_bytes, lla_s
     wa.q = a.q; wa.q_sb = a.qs_b; wa.q_srow = a.d_h; wa.qmul = a.qmul;
     wa.rotate = 0; wa.pos = a.N - 1; wa.base = 0.0;
     wa.win_ml = a.win_ml; wa.win_y = a.win_y; wa.err = err;
+    wa.rows_total = a.rows; wa.row0 = 0;
     e = launch_window(wa, s);
   }
   if (e == cudaSuccess) {

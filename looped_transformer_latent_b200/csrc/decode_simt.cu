@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(256, MINB) window_part(WindowArgs w) {
   }
   const int64_t seq = (int64_t)b * w.wins_b;
   for (int h = warp; h < w.H; h += 8) {
-    const int row = tt * w.H + h;
+    const int row = w.row0 + tt * w.H + h;
     float qv[4] = {0.f, 0.f, 0.f, 0.f}, acc[4] = {0.f, 0.f, 0.f, 0.f};
     if (dv) {
       const float* q = w.q + (int64_t)b * w.q_sb + (int64_t)row * w.q_srow + d0;
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(256, MINB) window_part(WindowArgs w) {
       }
       m = mn;
     }
-    const int64_t o = ((int64_t)chunk * w.B + b) * w.rows + row;
+    const int64_t o = ((int64_t)chunk * w.B + b) * w.rows_total + row;
     if (lane == 0) {
       w.win_ml[o * 2] = m;
       w.win_ml[o * 2 + 1] = l;
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(const __grid_consta
 
   const int d0 = 4 * lane;
   const bool dv = warp < nh && d0 < w.d_h;
-  const int row = tt * w.H + h0 + warp;
+  const int row = w.row0 + tt * w.H + h0 + warp;
   float c0 = 1.f, s0 = 0.f, c1 = 1.f, s1 = 0.f;
   if (w.rotate && dv) {
     c0 = w.rot[2 * lane].x; s0 = w.rot[2 * lane].y;
@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(const __grid_consta
     return;
   }
   if (warp < nh) {
-    const int64_t o = ((int64_t)chunk * w.B + b) * w.rows + row;
+    const int64_t o = ((int64_t)chunk * w.B + b) * w.rows_total + row;
     if (lane == 0) {
       w.win_ml[o * 2] = m;
       w.win_ml[o * 2 + 1] = l;

@@ -275,6 +275,8 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
     const int r = 16 * warp + (lane & 15);
     const bool owner = lane < 16;
     const bool active = owner && r < rows;
+    // last latent token (exclusive) of this row's query position
+    const int rlim = a.nq > 1 ? a.n_lat - (a.nq - 1 - r / a.rows_per_q) : a.n_lat;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
@@ -290,7 +292,7 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(smem_u32(&s_free[buf]));
-      const int nvalid = min(TOK, tok1 - (tok0 + n * TOK));
+      const int nvalid = min(TOK, min(tok1, rlim) - (tok0 + n * TOK));
       if (nvalid < TOK) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
@@ -317,7 +319,8 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
       }
       uint32_t pk[32];
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      const float mneg = active ? -m_run : -INFINITY;   // inactive rows give p = 0
+      // inactive rows, and rows with no token yet, give p = 0
+      const float mneg = (active && m_run != -INFINITY) ? -m_run : -INFINITY;
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
         const float p0 = ex2(sc[c] + mneg);

@@ -26,6 +26,7 @@
 // epilogue.  Waits are bounded: on a
 // timeout the CTA records an error code (outputs become NaN downstream).
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include <algorithm>
 #include <cstring>
@@ -256,10 +257,10 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
       tma_load_4d(s0, &maps.a[ai], bar, d, t.m0, ha, ta);
       tma_load_4d(s0 + a_part, &maps.x[ai], bar, d, hx, tx, t.n0);
     } else if (KIND == KIND_QMAP) {
-      tma_load_4d(s0, &maps.a[0], bar, 0, k0, t.m0 / 32, t.g);
+      tma_load_4d(s0, &maps.a[0], bar, 0, k0, t.m0 / 32, t.g % a.ncodec);
       tma_load_3d(s0 + a_part, &maps.x[0], bar, k0, t.g, t.n0);
     } else {
-      tma_load_4d(s0, &maps.a[0], bar, 0, k0, t.m0 / 32, t.g);
+      tma_load_4d(s0, &maps.a[0], bar, 0, k0, t.m0 / 32, t.g % a.ncodec);
       for (int jb = 0; jb < nb; ++jb)
         tma_load_4d(s0 + a_part + jb * b_tile, &maps.x[0], bar, k0, t.g, t.n0, jb);
     }
@@ -420,7 +421,10 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
       }
     };
     float cq = 1.f, sq = 0.f;
-    if (KIND == KIND_QMAP && a.rotate && m < t.Mv) rope_cs(m >> 1, a.Mtot, a.d_h, a.base, (double)a.pos, &cq, &sq);
+    if (KIND == KIND_QMAP && a.rotate && m < t.Mv) {
+      const int pos = a.pos + (a.rows_per_q > 0 ? t.g / a.rows_per_q : 0);   // this row's query position
+      rope_cs(m >> 1, a.Mtot, a.d_h, a.base, (double)pos, &cq, &sq);
+    }
     const bool bad = !ok || (KIND == KIND_OMAP && a.err && *a.err);
 #pragma unroll 1
     for (int c = half * (BN / 32); c < (half + 1) * (BN / 32); ++c) {
@@ -459,7 +463,9 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
           if (!(m & 1) && m < t.Mv && n < t.Nv) {
             const float rx = bad ? NAN : (x * cq - y * sq) * a.qmul;
             const float ry = bad ? NAN : (x * sq + y * cq) * a.qmul;
-            *reinterpret_cast<__nv_bfloat162*>(a.qbf + qbf_index(n, t.g, m, a.Mtot)) = __floats2bfloat162_rn(rx, ry);
+            void* dst = a.qbf + qbf_index(n, t.g, m, a.Mtot);
+            if (a.qf16) *reinterpret_cast<__half2*>(dst) = __floats2half2_rn(rx, ry);
+            else *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(rx, ry);
           }
         }
       } else if (KIND == KIND_OMAP) {
@@ -739,10 +745,13 @@ cudaError_t launch_query_map_tc(const MapArgs& g, int* err, cudaStream_t st) {
   a.B = g.B; a.rows = g.rows; a.Mtot = g.N; a.K = g.K; a.mtiles = (g.N + GM - 1) / GM;
   a.Aw = g.W; a.X = g.X; a.xs_b = g.xs_b;
   a.rotate = g.rotate; a.pos = g.pos; a.d_h = g.d_h; a.base = g.base; a.qmul = g.qmul; a.qbf = g.qbf;
+  a.qf16 = g.q_f16;
+  a.ncodec = g.ncodec > 0 ? g.ncodec : g.rows;
+  a.rows_per_q = g.rows_per_q;
   a.err = err; a.NB = 1; a.S = 1; a.ks = 1;
   TcMaps maps;
   std::memset(&maps, 0, sizeof(maps));
-  if (!map_codec_tmap(&maps.a[0], g.W, g.rows, g.K, g.N)) return cudaErrorNotSupported;
+  if (!map_codec_tmap(&maps.a[0], g.W, a.ncodec, g.K, g.N)) return cudaErrorNotSupported;
   return launch_bn<KIND_QMAP, 1>(maps, a, g.B, 64, 1, 128, SMEM_MAX / 2 - 1024, qmap_x, st);
 }
 
@@ -761,6 +770,7 @@ cudaError_t launch_output_map_tc(const MapArgs& g, cudaStream_t st) {
   a.part_ml = g.part_ml; a.win_ml = g.win_ml; a.win_y = g.win_y; a.Sw = g.Sw;
   a.out = g.out; a.outs_b = g.outs_b; a.err = const_cast<int*>(g.err);
   a.NB = g.S; a.S = 1;
+  a.ncodec = g.ncodec > 0 ? g.ncodec : g.rows;
   int bn_cap = 128;
   while (bn_cap > 32 && g.S * bn_cap > 256) bn_cap >>= 1;
   // k-splits over a cluster so that small batches still fill the SMs
@@ -772,7 +782,7 @@ cudaError_t launch_output_map_tc(const MapArgs& g, cudaStream_t st) {
   a.ks = std::max(1, std::min(std::min(4, nk), 128 / std::max(tiles, 1)));
   TcMaps maps;
   std::memset(&maps, 0, sizeof(maps));
-  if (!map_codec_tmap(&maps.a[0], g.W, g.rows, g.K, g.N)) return cudaErrorNotSupported;
+  if (!map_codec_tmap(&maps.a[0], g.W, a.ncodec, g.K, g.N)) return cudaErrorNotSupported;
   return launch_bn<KIND_OMAP, 1>(maps, a, g.B, g.rows, g.S, bn_cap, SMEM_MAX, omap_x, st);
 }
 

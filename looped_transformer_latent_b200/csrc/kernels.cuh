@@ -67,6 +67,10 @@ struct AbsorbArgs {
   // tensor-core path
   int use_tc;
   int rows_pad;        // rows rounded up to 16 (N of the accumulate MMA)
+  // several query positions (the last nq of the context) in one call: rows
+  // are (position, loop, head); row r's latent tokens end at
+  // n_lat - (nq - 1 - r / rows_per_q); nq = 1 is the plain decode read
+  int nq, rows_per_q;
   __nv_bfloat16* qbf;  // [B][r_k/64][64 rows x 64] bf16 Q~, 128-byte swizzled, rows >= rows zero
   int* err;            // 0, or the code of a timed-out wait in the latent read
 };
@@ -106,7 +110,8 @@ struct WindowArgs {
   int rotate, pos;
   double base;
   float2 rot[64];          // cos, sin of pair p at pos (set by launch_window when rotate)
-  float *win_ml, *win_y;   // [Sw][B][rows][2], [Sw][B][rows][d_h]
+  float *win_ml, *win_y;   // [Sw][B][rows_total][2], [Sw][B][rows_total][d_h]
+  int rows_total, row0;    // this launch's rows are rows row0.. of rows_total (one query position)
   int* err;                // optional: set to ERR_WINDOW_TIMEOUT if a copy never lands
 };
 constexpr int ERR_WINDOW_TIMEOUT = 21;
@@ -131,6 +136,9 @@ struct MapArgs {
   const float* X;
   int64_t xs_b, xs_row;
   int rotate, pos, use_tc;
+  int q_f16;               // query operand in f16 (fp8 latent read) instead of bf16
+  int ncodec;              // codec groups: row g uses codec g mod ncodec (0: rows)
+  int rows_per_q;          // query map: row g is at position pos + g / rows_per_q (0: pos)
   double base;
   float qmul;
   float* qlat;
@@ -155,6 +163,9 @@ struct TcGemmArgs {
   const float *Aw, *X;     // codec [group][K][Mtot]; activations (per kind)
   int64_t xs_b;
   int rotate, pos, d_h;    // query map epilogue
+  int qf16;                // query operand written as f16 (same layout) instead of bf16
+  int ncodec;              // codec groups: group g uses codec g mod ncodec
+  int rows_per_q;          // query map: group g is at position pos + g / rows_per_q (0: pos)
   double base;
   float qmul;
   __nv_bfloat16* qbf;
@@ -180,6 +191,10 @@ bool recon_tc_supported(const ReconArgs& a);
 cudaError_t launch_recon_tc(const ReconArgs& a, int* err, cudaStream_t st, int num_sms);
 
 bool absorb_tc_supported(int lat_dtype, int r_k, int r_v, int rows);
+// fp8 latent rows (LLA_FP8_E4M3): the same read with the codes widened to f16
+// on chip and the per-token scales applied on the softmax side (decode_fp8.cu)
+bool absorb_fp8_supported(int r_k, int r_v, int rows);
+cudaError_t launch_absorb_split_fp8(const AbsorbArgs& a, cudaStream_t st);
 int absorb_tc_rows_pad(int rows);
 int absorb_tc_splits(int B, int n_lat, int num_sms);
 cudaError_t launch_absorb_split_tc(const AbsorbArgs& a, cudaStream_t st);

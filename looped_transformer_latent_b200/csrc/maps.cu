@@ -83,7 +83,8 @@ __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
   const int n0 = blockIdx.y * GN;
   const int tn = lane;             // column pair within the tile
   const int tb = warp * BPW;       // first of this thread's sequences
-  const float* Wr = g.W + (int64_t)row * g.K * g.N;
+  // several query positions share each (loop, head) codec
+  const float* Wr = g.W + (int64_t)(g.ncodec > 0 ? row % g.ncodec : row) * g.K * g.N;
   // loader coordinates
   const int xb = tid / (GK / LX), xk = (tid % (GK / LX)) * LX;   // X: GB sequences x 32 k
   constexpr int LW = GK * GN / GT;                  // codec loads per thread
@@ -147,7 +148,8 @@ __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
   if (n >= g.N) return;
   if (MODE == 0) {
     float c = 1.f, s = 0.f;
-    if (g.rotate) rope_cs(n / 2, g.N, g.d_h, g.base, (double)g.pos, &c, &s);
+    if (g.rotate)
+      rope_cs(n / 2, g.N, g.d_h, g.base, (double)(g.pos + (g.rows_per_q > 0 ? row / g.rows_per_q : 0)), &c, &s);
 #pragma unroll
     for (int j = 0; j < BPW; ++j) {
       const int bb = tb + j;

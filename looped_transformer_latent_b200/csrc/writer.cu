@@ -5,6 +5,8 @@
 // split-K SIMT fp32 GEMM writing partial sums to the workspace; phase 2 adds
 // the partials in a fixed order (deterministic), rotates key pairs by
 // R~_pos (HLA), rounds once to the storage type and stores the cache rows.
+#include <cuda_fp8.h>
+
 #include "writer_slice.cuh"
 
 namespace lla {
@@ -136,6 +138,81 @@ __global__ void writer_epilogue(WriterArgs a) {
   }
 }
 
+// Phase 2 for fp8 rows (e4m3 codes with per-token, per-part scales): one warp
+// per (target row, token).  HLA: target 0 is the main latent (slice 0), target
+// 1 the loop-1 latent (slice 1); FOLDED: target 0 takes its key part from
+// slice 0 and its value part from slice 1.  The warp sums the splits in order,
+// rotates the key pairs (HLA), keeps the row in shared memory, reduces the
+// largest magnitude of each part, and stores codes = e4m3(x / s) (nearest-even,
+// saturating) with s = amax / 448, then s^K, s^V and 8 zero bytes.
+constexpr int FP8_WARPS = 4;                 // static shared memory: 4 rows of up to 2048 floats
+constexpr int FP8_ROW_MAX = 2048;
+
+__device__ __forceinline__ float fp8_part_value(const WriterArgs& a, int tgt, int m, int n, int kw) {
+  // column n of target row tgt, before rotation
+  int z = tgt, nn = n;
+  if (a.mode == LLA_WRITE_FOLDED && n >= kw) { z = 1; nn = n - kw; }
+  float x = 0.f;
+  for (int sp = 0; sp < a.S; ++sp) x += a.part[((int64_t)(z * a.S + sp) * a.M + m) * a.Nmax + nn];
+  return x;
+}
+
+__global__ void __launch_bounds__(FP8_WARPS * 32) writer_epilogue_fp8(WriterArgs a) {
+  __shared__ float rowbuf[FP8_WARPS][FP8_ROW_MAX];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntgt = a.mode == LLA_WRITE_HLA ? 2 : 1;
+  const int64_t total = (int64_t)ntgt * a.M;
+  float* buf = rowbuf[warp];
+  for (int64_t idx = (int64_t)blockIdx.x * FP8_WARPS + warp; idx < total; idx += (int64_t)gridDim.x * FP8_WARPS) {
+    const int tgt = (int)(idx / a.M), m = (int)(idx % a.M);
+    int kw, vw;
+    if (a.mode == LLA_WRITE_HLA) {
+      kw = tgt == 0 ? a.r_k : a.r_1;
+      vw = tgt == 0 ? a.r_v : a.r_1;
+    } else {
+      kw = a.r_k;
+      vw = a.r_v;
+    }
+    const bool rot = a.mode == LLA_WRITE_HLA && a.rotate;
+    const int b = m / a.n_tok, j = m % a.n_tok;
+    const int pos = a.pos0 + j;
+    float amax_k = 0.f, amax_v = 0.f;
+    for (int p = lane; p < (kw + vw) / 2; p += 32) {
+      const int n = 2 * p;
+      float x = fp8_part_value(a, tgt, m, n, kw), y = fp8_part_value(a, tgt, m, n + 1, kw);
+      if (rot && n < kw) {
+        float c, sn;
+        rope_cs(p, kw, a.d_h, a.base, (double)pos, &c, &sn);
+        const float xr = x * c - y * sn, yr = x * sn + y * c;
+        x = xr; y = yr;
+      }
+      buf[n] = x;
+      buf[n + 1] = y;
+      const float mx = fmaxf(fabsf(x), fabsf(y));
+      if (n < kw) amax_k = fmaxf(amax_k, mx); else amax_v = fmaxf(amax_v, mx);
+    }
+    amax_k = warp_max(amax_k);
+    amax_v = warp_max(amax_v);
+    __syncwarp();
+    const bool bad = *a.err != 0;
+    const float sk = bad ? NAN : amax_k / 448.f, sv = bad ? NAN : amax_v / 448.f;
+    uint8_t* row;
+    if (tgt == 0) row = reinterpret_cast<uint8_t*>(a.out0) + (int64_t)b * a.os_b + (int64_t)pos * a.os_n;
+    else row = reinterpret_cast<uint8_t*>(a.out1) + (int64_t)b * a.o1s_b + (int64_t)pos * a.o1s_n;
+    for (int n = lane; n < kw + vw; n += 32) {
+      const float s = n < kw ? sk : sv;
+      const float q = s > 0.f ? buf[n] / s : 0.f;
+      const __nv_fp8_e4m3 code(q);   // nearest-even, saturating to +-448
+      row[n] = *reinterpret_cast<const uint8_t*>(&code);
+    }
+    if (lane < 4) {
+      const float sc[2] = {sk, sv};
+      reinterpret_cast<float*>(row + kw + vw)[lane] = lane < 2 ? sc[lane] : 0.f;
+    }
+    __syncwarp();
+  }
+}
+
 }  // namespace
 
 // Partial sums, then (16 bytes) the tensor-core error flag.
@@ -182,6 +259,13 @@ cudaError_t launch_writer(const WriterArgs& a_in, cudaStream_t st) {
     e0 = cudaGetLastError();
   }
   if (e0 != cudaSuccess) return e0;
+  if (a.dtype == LLA_FP8_E4M3) {
+    const int64_t rows = (int64_t)(a.mode == LLA_WRITE_HLA ? 2 : 1) * a.M;
+    int blocks = (int)((rows + FP8_WARPS - 1) / FP8_WARPS);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    writer_epilogue_fp8<<<blocks, FP8_WARPS * 32, 0, st>>>(a);
+    return cudaGetLastError();
+  }
   const int64_t total = (int64_t)a.Z * a.M * (a.Nmax / 2);
   int blocks = (int)((total + 255) / 256);
   if (blocks > 148 * 16) blocks = 148 * 16;

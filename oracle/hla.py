@@ -113,6 +113,23 @@ def decode(lat, A, Bm, q, win_k, win_v, t0, N, W, r_k, r_v, d_h, base,
     return out
 
 
+def decode_positions(lat, A, Bm, q, win_k, win_v, t0, N, W, r_k, r_v, d_h, base,
+                     rotate_query=True, scale=None):
+    """The read of the last nq positions of a context of N tokens at once.
+
+    Used for a prefill chunk, or for a block of the two-pass procedure's
+    parallel second pass (HLA summary, "Methodology / Fine-tuning"), where
+    every position's query exists together.  Position i_p = N - nq + p is read
+    exactly as a decode at i = i_p: latent tokens j < i_p - W, exact tokens
+    i_p - W .. i_p from the ring (eqs. 3-4 with N = i_p + 1).
+    q [nq, nt, H, d_h] -> o [nq, nt, H, d_h].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    nq = q.shape[0]
+    return np.stack([decode(lat, A, Bm, q[p], win_k, win_v, t0, N - nq + p + 1, W, r_k, r_v, d_h, base,
+                            rotate_query=rotate_query, scale=scale) for p in range(nq)])
+
+
 def decode_reconstruct(lat, A, Bm, q, win_k, win_v, t0, N, W, r_k, r_v, d_h,
                        base, rotate_query=True, scale=None):
     """The same read with keys and values rebuilt in head space first.

@@ -102,6 +102,24 @@ def row_bytes(codes, sK, sV):
     return out
 
 
+def from_row_bytes(rows, r_k, r_v):
+    """Values of stored fp8 rows given as bytes [n, r_k + r_v + 16] (uint8):
+    each code decoded from its e4m3 bit pattern, times its part's scale."""
+    rows = np.asarray(rows, dtype=np.uint8)
+    w = r_k + r_v
+    b = rows[:, :w].astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 7).astype(np.float64)
+    if np.any((e == 15) & (m == 7)):
+        raise ValueError("NaN code in a latent row")
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.ldexp(1.0, e - 7))
+    codes = sign * mag
+    sK = rows[:, w:w + 4].copy().view(np.float32)[:, 0]
+    sV = rows[:, w + 4:w + 8].copy().view(np.float32)[:, 0]
+    return dequantize_rows(codes, sK, sV, r_k)
+
+
 def to_storage_fp8(c, r_k, r_v):
     """Convenience: the values the read sees for exact rows c."""
     codes, sK, sV = quantize_rows(c, r_k, r_v)
@@ -109,4 +127,4 @@ def to_storage_fp8(c, r_k, r_v):
 
 
 __all__ = ["E4M3_MAX", "to_e4m3", "quantize_rows", "dequantize_rows", "e4m3_bits", "row_bytes",
-           "to_storage_fp8"]
+           "from_row_bytes", "to_storage_fp8"]

@@ -18,5 +18,5 @@ numpy default_rng), so the same seed gives the same bits on every machine.
 
 from .gen import (  # noqa: F401
     CONFIGS, ConfigShape, tiny_hla, hla_codec, hla_hidden, lla_perhead_codec,
-    lla_folded_codec, lla_kv, queries, window_ring, random_latents,
+    lla_folded_codec, lla_kv, queries, window_ring, random_latents, random_fp8_rows,
 )

@@ -246,3 +246,19 @@ def random_latents(B, n, width, seed, dtype=torch.bfloat16, std=1.0, device="cpu
     """Latent rows drawn directly ~ N(0, std^2) [B, n, width]."""
     x = torch.randn(B, n, width, generator=_gen(seed, device), device=device) * std
     return x.to(dtype)
+
+
+def random_fp8_rows(B, n, r_k, r_v, seed, device="cpu"):
+    """fp8 latent rows [B, n, r_k + r_v + 16] (uint8): e4m3 codes of N(0, 100^2)
+    draws clipped to +-448 (torch's float32 -> float8_e4m3fn conversion), then
+    per-token scales s^K, s^V ~ U(0.002, 0.02) as fp32 bytes, then 8 zero
+    bytes."""
+    g = _gen(seed)
+    w = r_k + r_v
+    x = (torch.randn(B, n, w, generator=g) * 100).clamp(-448, 448)
+    codes = x.to(torch.float8_e4m3fn).view(torch.uint8)
+    sc = (torch.rand(B, n, 2, generator=g) * 0.018 + 0.002).to(torch.float32)
+    rows = torch.zeros(B, n, w + 16, dtype=torch.uint8)
+    rows[:, :, :w] = codes
+    rows[:, :, w:w + 8] = sc.view(torch.uint8).reshape(B, n, 8)
+    return rows.to(device)

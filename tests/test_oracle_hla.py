@@ -308,3 +308,29 @@ def test_printed_cache_sizes():
     cK, cV = lla.write_perhead(k, v, EK, EV)
     assert cK.shape == (H_h, 1, r_h) and cV.shape == (H_h, 1, r_h)
     assert (k.size + v.size) / (cK.size + cV.size) == g["huginn_lla_compression"]
+
+
+def test_several_positions_with_full_window_are_causal_exact_attention():
+    """decode_positions with W >= N: every position p reads only the exact ring,
+    so each must equal textbook causal rotary attention over tokens 0..i_p with
+    i_p = N - nq + p (pins the positions, the ring slots j mod Wcap and the
+    per-position rotation against an independent formula)."""
+    rng = np.random.default_rng(21)
+    N, nq, T, H, d_h, W = 12, 4, 3, 2, 8, 20
+    Wcap = 13
+    k = rng.standard_normal((N, T, H, d_h))
+    v = rng.standard_normal((N, T, H, d_h))
+    q = rng.standard_normal((nq, 2, H, d_h))
+    ring_k = np.zeros((T, Wcap, H, d_h))
+    ring_v = np.zeros((T, Wcap, H, d_h))
+    for j in range(N):
+        ring_k[:, j % Wcap] = rope.rotate(k[j], j, d_h, BASE)
+        ring_v[:, j % Wcap] = v[j]
+    A = rng.standard_normal((2, H, d_h, 16))
+    Bm = rng.standard_normal((2, H, 16, d_h))
+    lat = rng.standard_normal((N, 32))
+    got = hla.decode_positions(lat, A, Bm, q, ring_k, ring_v, 1, N, W, 16, 16, d_h, BASE)
+    for p in range(nq):
+        i = N - nq + p
+        ref = exact.attention(q[p], k[:i + 1], v[:i + 1], 1, d_h, BASE)
+        np.testing.assert_allclose(got[p], ref, atol=1e-12)

@@ -64,3 +64,22 @@ def test_zero_part_and_row_bytes():
     assert not np.any(rb[:, 56:])
     # -8 / (8 / 448) = -448 exactly: code byte of -448 is 0xFE
     assert rb[1, 32] == 0xFE
+
+
+def test_row_bytes_decode_round_trip_and_library_codes():
+    """from_row_bytes inverts row_bytes, and decodes code bytes exactly as
+    torch's float8_e4m3fn does."""
+    rng = np.random.default_rng(8)
+    c = rng.standard_normal((20, 192)) * 3
+    codes, sK, sV = quant.quantize_rows(c, 128, 64)
+    rows = quant.row_bytes(codes, sK, sV)
+    assert np.array_equal(quant.from_row_bytes(rows, 128, 64), quant.dequantize_rows(codes, sK, sV, 128))
+    allb = np.arange(256, dtype=np.uint8)
+    allb = allb[(allb & 0x7F) != 0x7F]                          # drop the two NaN codes
+    lib = torch.from_numpy(allb.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    row = np.zeros((1, 256 + 16), dtype=np.uint8)
+    row[0, :allb.size] = allb
+    row[0, 256:260] = np.array([1.0], dtype=np.float32).view(np.uint8)
+    row[0, 260:264] = np.array([1.0], dtype=np.float32).view(np.uint8)
+    vals = quant.from_row_bytes(row, 128, 128)[0, :allb.size]
+    assert np.array_equal(vals, lib)
