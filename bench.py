@@ -130,10 +130,23 @@ class Step:
                 nb = max(nb, L.lla_write_workspace_bytes(mode, **{k: v for k, v in kw.items() if k != "mode"}))
         self.ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=self.dev)
 
-    def run(self, events=None):
+    def layer_io(self):
+        """(inputs, outputs) of each layer in order: every workload appends the
+        same number of calls, inputs and outputs per layer."""
+        n = self.cfg.L
+        ci, co = len(self.ins) // n, len(self.outs) // n
+        return [(self.ins[k * ci:(k + 1) * ci], self.outs[k * co:(k + 1) * co]) for k in range(n)]
+
+    def run(self, events=None, hook=None):
+        """Issue the step on the current stream.  hook(layer, "begin"/"end"),
+        if given, runs on the current stream before a layer's first call and
+        after its last one."""
         L = self.L
         ei = 0
-        for kind, kw, _ in self.calls:
+        per = len(self.calls) // self.cfg.L
+        for idx, (kind, kw, _) in enumerate(self.calls):
+            if hook is not None and idx % per == 0:
+                hook(idx // per, "begin")
             if kind in ("hla", "lla"):
                 ev = None
                 if events is not None:
@@ -144,6 +157,8 @@ class Step:
             else:
                 mode = kw["mode"]
                 L.lla_write_latents(mode, workspace=self.ws, **{k: v for k, v in kw.items() if k != "mode"})
+            if hook is not None and idx % per == per - 1:
+                hook(idx // per, "end")
 
     def read_tags(self):
         return [tag for kind, _, tag in self.calls if kind in ("hla", "lla")]
@@ -277,15 +292,17 @@ class HlaStep(Step):
         nb = min(self.prefill_chunk, self.cfg.B - b0)
         return self._prefill_hidden_chunk(b0, nb)[b - b0].cpu()
 
-    def run(self, events=None):
+    def run(self, events=None, hook=None):
         if self.side is None:
-            return super().run(events)
+            return super().run(events, hook)
         L = self.L
         main = torch.cuda.current_stream(self.dev)
         ei = 0
         for layer in range(self.cfg.L):
             (k1, kw1, _), (k2, kw2, _), (_, kww, _) = self.calls[3 * layer:3 * layer + 3]
             assert k1 == "hla" and k2 == "hla"
+            if hook is not None:
+                hook(layer, "begin")
             self.fork[layer].record(main)
             self.side.wait_event(self.fork[layer])
             L.hla_decode_attn(workspace=self.ws_side, stream=self.side,
@@ -297,6 +314,8 @@ class HlaStep(Step):
             L.hla_decode_attn(workspace=self.ws, stream=main,
                               timing_events=events[ei + 1] if events is not None else None, **kw2)
             main.wait_event(self.join[layer])
+            if hook is not None:
+                hook(layer, "end")
             ei += 2
 
 
@@ -600,6 +619,28 @@ def tc_traffic_per_token(row_bytes):
     return TC_TRAFFIC_PER_TOKEN.get((key, row_bytes))
 
 
+_DRIVER = None
+
+
+def memcpy_async(dst, src, stream):
+    """One cuMemcpyAsync of a dense tensor on `stream` (unified addressing:
+    either side may be pinned host memory); under stream capture it becomes a
+    copy node of the graph, with no host-allocator bookkeeping."""
+    global _DRIVER
+    if _DRIVER is None:
+        import ctypes
+        lib = ctypes.CDLL("libcuda.so.1")
+        lib.cuMemcpyAsync.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_size_t, ctypes.c_void_p]
+        lib.cuMemcpyAsync.restype = ctypes.c_int
+        _DRIVER = lib
+    n = src.numel() * src.element_size()
+    if not (dst.is_contiguous() and src.is_contiguous()) or dst.numel() * dst.element_size() != n:
+        raise ValueError("memcpy_async needs two dense tensors of the same size")
+    rc = _DRIVER.cuMemcpyAsync(dst.data_ptr(), src.data_ptr(), n, stream.cuda_stream)
+    if rc != 0:
+        raise RuntimeError(f"cuMemcpyAsync failed with CUresult {rc}")
+
+
 def reduce_max(dist, value, device):
     """Max of a per-rank float over all ranks (the value itself on one rank)."""
     if dist is None:
@@ -680,19 +721,52 @@ def main():
     if dist is not None:
         dist.barrier()
 
-    # end to end: pinned host inputs -> device, step, outputs -> host
-    ins, outs = step.io_tensors()
-    h_ins = [t.detach().cpu().pin_memory() for t in ins]
-    h_outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
-    h2d = sum(t.numel() * t.element_size() for t in h_ins)
-    d2h = sum(t.numel() * t.element_size() for t in h_outs)
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            for d, hsrc in zip(ins, h_ins):
-                d.copy_(hsrc, non_blocking=True)
-            graph.replay()
-            for hdst, d in zip(h_outs, outs):
-                hdst.copy_(d, non_blocking=True)
+    # end to end: every step copies its inputs from pinned host memory, runs,
+    # and copies its outputs back.  One graph holds all of it: layer l's
+    # inputs go up on a copy stream ahead of its compute, its outputs come
+    # down on another as soon as it finishes, so the copies overlap the
+    # compute of neighbouring layers.
+    layers = step.layer_io()
+    h_layers = [([t.detach().cpu().pin_memory() for t in li],
+                 [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in lo]) for li, lo in layers]
+    h2d = sum(t.numel() * t.element_size() for hi, _ in h_layers for t in hi)
+    d2h = sum(t.numel() * t.element_size() for _, ho in h_layers for t in ho)
+    cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in layers]
+    ev_done = [torch.cuda.Event() for _ in layers]
+    fork, fin = torch.cuda.Event(), torch.cuda.Event()
+
+    def io_hook(layer, phase):
+        cur = torch.cuda.current_stream(dev)
+        if phase == "begin":
+            cur.wait_event(ev_in[layer])
+            return
+        ev_done[layer].record(cur)
+        cout.wait_event(ev_done[layer])
+        for hdst, d in zip(h_layers[layer][1], layers[layer][1]):
+            memcpy_async(hdst, d, cout)
+
+    e2e_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(e2e_graph, stream=stream):
+        fork.record(stream)
+        cin.wait_event(fork)
+        cout.wait_event(fork)
+        for k, (li, _) in enumerate(layers):
+            for d, hsrc in zip(li, h_layers[k][0]):
+                memcpy_async(d, hsrc, cin)
+            ev_in[k].record(cin)
+        step.run(hook=io_hook)
+        fin.record(cout)
+        stream.wait_event(fin)
+    torch.cuda.synchronize()
+    e2e_graph.replay()
+    torch.cuda.synchronize()
+    h_all = [t for _, ho in h_layers for t in ho]
+    for h, e in zip(h_all, eager):      # the copied-back outputs are the eager step's
+        if not torch.equal(h, e.cpu()):
+            raise SystemExit("end-to-end step output differs from the eager step")
+    for _ in range(3):
+        e2e_graph.replay()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -701,11 +775,7 @@ def main():
     with torch.cuda.stream(stream):
         e0.record(stream)
         for _ in range(args.steps):
-            for d, hsrc in zip(ins, h_ins):
-                d.copy_(hsrc, non_blocking=True)
-            graph.replay()
-            for hdst, d in zip(h_outs, outs):
-                hdst.copy_(d, non_blocking=True)
+            e2e_graph.replay()
         e1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1) / args.steps
@@ -802,7 +872,7 @@ def main():
         line["cpu_baseline"] = cpu_baseline(cfg)
     if rank == 0:
         print(json.dumps(line))
-    del graph
+    del graph, e2e_graph
     if dist is not None:
         dist.destroy_process_group()
 
