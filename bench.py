@@ -174,7 +174,8 @@ class Step:
     def latent_bytes(self, kind, kw):
         c = self.cfg
         if kind == "hla":
-            return c.B * self.n_lat * kw["lat"].shape[-1] * 2
+            lat = kw["lat"]
+            return c.B * self.n_lat * lat.shape[-1] * lat.element_size()
         return c.B * c.H * self.n_lat * kw["cK"].shape[-1] * 2 * 2
 
     def read_latent_bytes(self):
@@ -339,7 +340,10 @@ class Lla2dStep(Step):
         self.seed = seed
         g = torch.Generator(device=dev)
         g.manual_seed(seed + 7)
-        lat0 = torch.empty(B, N, c.r_k + c.r_v, dtype=torch.bfloat16, device=dev)
+        if c.lat_dtype == "fp8":   # byte rows: codes, then s^K, s^V and 8 zero bytes
+            lat0 = torch.empty(B, N, c.r_k + c.r_v + 16, dtype=torch.uint8, device=dev)
+        else:
+            lat0 = torch.empty(B, N, c.r_k + c.r_v, dtype=torch.bfloat16, device=dev)
         chunk = self.prefill_chunk = max(1, (1 << 28) // (N * T * H * d_h * 2))
         for b0 in range(0, B, chunk):
             nb = min(chunk, B - b0)
@@ -496,9 +500,17 @@ def oracle_sample(cfg, seed=5):
         q = rng.standard_normal((c.T, c.H, c.d_h))
         k = rng.standard_normal((1, c.T, c.H, c.d_h))
         v = rng.standard_normal((1, c.T, c.H, c.d_h))
-        t = time.perf_counter()
-        lla.decode_absorbed(lat, UK, UV, q, k[0][:, None], v[0][:, None], 0, c.N, 0, c.r_k, c.r_v)
-        lla.write_folded(k, v, EK, EV)
+        if c.lat_dtype == "fp8":
+            from oracle import quant
+            rows = quant.row_bytes(*quant.quantize_rows(lat, c.r_k, c.r_v))
+            t = time.perf_counter()
+            lat = quant.from_row_bytes(rows, c.r_k, c.r_v)
+            lla.decode_absorbed(lat, UK, UV, q, k[0][:, None], v[0][:, None], 0, c.N, 0, c.r_k, c.r_v)
+            quant.quantize_rows(lla.write_folded(k, v, EK, EV), c.r_k, c.r_v)
+        else:
+            t = time.perf_counter()
+            lla.decode_absorbed(lat, UK, UV, q, k[0][:, None], v[0][:, None], 0, c.N, 0, c.r_k, c.r_v)
+            lla.write_folded(k, v, EK, EV)
         per_token = c.L
     else:
         cK = rng.standard_normal((1, n, c.r_k))
@@ -597,7 +609,7 @@ def run_reference(args, cfg):
 # lines removed, so only code changes count) and the latent row width in
 # bytes: a changed kernel, or a row width never captured, reports no traffic
 # (null) until it is captured again.
-TC_TRAFFIC_PER_TOKEN = {("21d0011aedbae00a", 2304): 2383.9}
+TC_TRAFFIC_PER_TOKEN = {("40779eafbad62733", 2304): 2376.1}
 
 
 def source_key(path):
@@ -801,7 +813,8 @@ def main():
         mean_ms = sum(spans) / max(1, len(spans))
         achieved = (nbytes / 1e9) / (sum(spans) / 1e3) if sum(spans) > 0 else 0.0
     all_gbs = (sum(lb) / 1e9) / (sum(split_ms) / 1e3) if sum(split_ms) > 0 else 0.0
-    per_tok = tc_traffic_per_token((cfg.r_k + cfg.r_v) * 2) if cfg.kind != "lla" else None
+    per_tok = (tc_traffic_per_token((cfg.r_k + cfg.r_v) * 2)
+               if cfg.kind != "lla" and cfg.lat_dtype == "bf16" else None)
     traffic = None
     if per_tok is not None and main_ix:
         traffic = per_tok * cfg.B * step.n_lat
@@ -821,7 +834,7 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "fp8-e4m3 latents, bf16/f16 tensor-core operands" if cfg.lat_dtype == "fp8" else "bf16",
         "data": "synthetic",
         "config": {"workload": cfg.name, "mode": args.mode, "batch_per_gpu": cfg.B, "context": cfg.N,
                    "layers": cfg.L, "loops": cfg.T, "heads": cfg.H, "d_h": cfg.d_h,
@@ -840,6 +853,8 @@ def main():
                      "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
                      "kernel": ("tensor-core latent read (absorb_split_tc), loop-1 and main launches of each "
                                 "layer running concurrently" if overlapped else
+                                "tensor-core latent read of fp8 rows (absorb_split_fp8), main-latent launches"
+                                if cfg.lat_dtype == "fp8" else
                                 "tensor-core latent read (absorb_split_tc), main-latent launches"),
                      "peak_source": src, "per_launch_ms": mean_ms,
                      "per_launch_ms_min_med_max": [srt[0], srt[len(srt) // 2], srt[-1]] if srt else None,

@@ -25,7 +25,7 @@ class ConfigShape:
     r_k: int
     r_v: int
     r_1: int
-    lat_dtype: str       # 'bf16' | 'f32'
+    lat_dtype: str       # 'bf16' | 'f32' | 'fp8' (e4m3 rows with per-token scales)
     base: float = 10000.0
 
 
@@ -50,6 +50,9 @@ CONFIGS = {
     # layer (r_K = r_V = 384) instead of the configured 1152
     "ouro_lla2d_768_r384": ConfigShape("ouro_lla2d_768_r384", "lla2d", B=768, L=24, T=4, H=16, d_h=128,
                                        D=0, N=4096, W=0, r_k=384, r_v=384, r_1=0, lat_dtype="bf16"),
+    # the gate workload with fp8 (e4m3) latent rows and per-token scales
+    "ouro_lla2d_768_fp8": ConfigShape("ouro_lla2d_768_fp8", "lla2d", B=768, L=24, T=4, H=16, d_h=128,
+                                      D=0, N=4096, W=0, r_k=576, r_v=576, r_1=0, lat_dtype="fp8"),
     # long-context HLA, 16k, batch 64
     "ouro_hla_16k": ConfigShape("ouro_hla_16k", "hla", B=64, L=24, T=4, H=16, d_h=128, D=2048,
                                 N=16384, W=128, r_k=512, r_v=512, r_1=256, lat_dtype="bf16"),

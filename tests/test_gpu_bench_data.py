@@ -22,7 +22,7 @@ import torch
 
 import bench
 import synth
-from oracle import hla, lla, rounding
+from oracle import hla, lla, quant, rounding
 from parity_check import assert_rows_close
 
 pytestmark = pytest.mark.gpu
@@ -83,3 +83,30 @@ def test_ouro_lla2d_768_bench_step_matches_oracle(cuda_device):
                                       f64(lay["wv"][b]), 0, c.N, 0, c.r_k, c.r_v)
             err = assert_rows_close(lay["out"][b], out, TOL_BF16, f"layer {layer} sequence {b}")
             print(f"ouro_lla2d_768 bench step, layer {layer} sequence {b}: rel L2 (pooled, worst row) {err}")
+
+
+def test_ouro_lla2d_768_fp8_bench_step_matches_oracle(cuda_device):
+    """The fp8-row variant of the gate step: the GPU writer quantises its rows
+    (e4m3 codes, per-token scales); the oracle quantises its own fp64 rows and
+    reads those.  The codes are compared byte for byte (a code may differ by
+    one step where the exact value sits on a rounding boundary, so 98 % equal
+    is required) and the outputs at the bf16 tolerance."""
+    c = synth.CONFIGS["ouro_lla2d_768_fp8"]
+    step = bench.Lla2dStep(c, cuda_device, "m1")
+    _run_eager(step, cuda_device)
+    cod = {k: v.double().numpy() for k, v in step.codec_host.items()}
+    n_lat, w = c.N - 1, c.r_k + c.r_v
+    for b in (0, 400, c.B - 1):
+        k, v = step.prefill_kv(b)
+        exact = lla.write_folded(k.double().numpy(), v.double().numpy(), cod["E_K"], cod["E_V"])
+        codes, sK, sV = quant.quantize_rows(exact, c.r_k, c.r_v)
+        got = step.layers[0]["lat"][b, :n_lat].cpu().numpy()
+        frac_eq = np.mean(got[:, :w] == quant.e4m3_bits(codes))
+        assert frac_eq > 0.98, f"sequence {b}: equal code fraction {frac_eq:.4f}"
+        rows = quant.dequantize_rows(codes, sK, sV, c.r_k)
+        for layer in (0, c.L - 1):
+            lay = step.layers[layer]
+            out = lla.decode_absorbed(rows, cod["U_K"], cod["U_V"], f64(lay["q"][b]), f64(lay["wk"][b]),
+                                      f64(lay["wv"][b]), 0, c.N, 0, c.r_k, c.r_v)
+            err = assert_rows_close(lay["out"][b], out, TOL_BF16, f"layer {layer} sequence {b}")
+            print(f"ouro_lla2d_768_fp8 bench step, layer {layer} sequence {b}: rel L2 (pooled, worst row) {err}")

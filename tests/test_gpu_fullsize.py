@@ -177,3 +177,33 @@ def test_decode_step_writers_at_full_batch(cuda_device):
         rk, rv = lla.write_perhead(f64(k[b]), f64(v[b]), f64(EK), f64(EV))
         assert_rows_close(cK[b, :, 3:], rk, 1e-2, "per-head K rows")
         assert_rows_close(cV[b, :, 3:], rv, 1e-2, "per-head V rows")
+
+
+def test_ouro_lla2d_768_fp8_read(cuda_device):
+    """The gate workload's shapes with fp8 rows (e4m3 codes, per-token scales)
+    at batch 768, sampled sequences against the oracle's read of the same rows."""
+    from oracle import quant
+    c = synth.CONFIGS["ouro_lla2d_768_fp8"]
+    B, N, H, T, d_h, r_k, r_v = c.B, c.N, c.H, c.T, c.d_h, c.r_k, c.r_v
+    g = torch.Generator().manual_seed(17)
+    ndist = 3
+    rows_d = synth.random_fp8_rows(ndist, N, r_k, r_v, 18)
+    A = torch.randn(T, H, d_h, r_k, generator=g) / math.sqrt(d_h)
+    Bm = torch.randn(T, H, r_v, d_h, generator=g) / math.sqrt(r_v)
+    q = torch.randn(B, T, H, d_h, generator=g)
+    wk_d = torch.randn(ndist, T, 1, H, d_h, generator=g).to(torch.bfloat16)
+    wv_d = torch.randn(ndist, T, 1, H, d_h, generator=g).to(torch.bfloat16)
+    dev = cuda_device
+    out = torch.full((B, T, H, d_h), float("nan"), device=dev)
+    L.hla_decode_attn(lat=_tile_batch(rows_d, B, dev), A=A.to(dev), Bm=Bm.to(dev), q=q.to(dev),
+                      win_k=_tile_batch(wk_d, B, dev), win_v=_tile_batch(wv_d, B, dev), out=out, N=N, W=0, t0=0,
+                      rotate_query=False)
+    torch.cuda.synchronize()
+    errs = []
+    for b in (0, 400, B - 1):
+        k = b % ndist
+        vals = quant.from_row_bytes(rows_d[k].numpy(), r_k, r_v)
+        ref = hla.decode(vals, f64(A), f64(Bm), f64(q[b]), f64(wk_d[k]), f64(wv_d[k]), 0, N, 0, r_k, r_v, d_h,
+                         BASE, rotate_query=False)
+        errs.append(assert_rows_close(out[b], ref, TOL_BF16, f"sequence {b}"))
+    print(f"ouro_lla2d_768_fp8: rel L2 (pooled, worst row) {errs}")
