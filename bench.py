@@ -129,6 +129,9 @@ class Step:
                 mode = kw["mode"]
                 nb = max(nb, L.lla_write_workspace_bytes(mode, **{k: v for k, v in kw.items() if k != "mode"}))
         self.ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=self.dev)
+        # the prefill ran on the constructing stream; the step may run on any
+        # other, so setup ends with everything it issued complete
+        torch.cuda.synchronize(self.dev)
 
     def layer_io(self):
         """(inputs, outputs) of each layer in order: every workload appends the

@@ -114,6 +114,13 @@ int lla_abi_version(void);
 /* Static description of a status code; never NULL. */
 const char *lla_status_str(int status);
 
+/* The cudaError_t value behind the most recent LLA_ERR_CUDA returned to the
+ * calling thread by any entry point (0 if none yet), and the CUDA runtime's
+ * name for it (static, never NULL).  Kept per thread; reading it clears
+ * nothing. */
+int lla_last_cuda_error(void);
+const char *lla_cuda_error_name(int cuda_error);
+
 /* ------------------------------------------------------------------------ */
 /* (a) Latent writer                                                          */
 /* ------------------------------------------------------------------------ */

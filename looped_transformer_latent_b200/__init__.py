@@ -17,7 +17,7 @@ Entry points (names as in the C ABI):
 import ctypes
 
 from . import _abi
-from ._abi import (LLA_BF16, LLA_F32, LLA_FP8_E4M3, LLA_WRITE_FOLDED, LLA_WRITE_HLA,  # noqa: F401
+from ._abi import (LLA_BF16, LLA_ERR_CUDA, LLA_F32, LLA_FP8_E4M3, LLA_WRITE_FOLDED, LLA_WRITE_HLA,  # noqa: F401
                    LLA_WRITE_PERHEAD, LibraryMissing)
 
 __all__ = [
@@ -34,7 +34,12 @@ class LLAError(RuntimeError):
 
     def __init__(self, status, where):
         self.status = status
-        super().__init__(f"{where}: status {status} ({lla_status_str(status)})")
+        msg = f"{where}: status {status} ({lla_status_str(status)})"
+        self.cuda_error = None
+        if status == LLA_ERR_CUDA:
+            self.cuda_error = lib().lla_last_cuda_error()
+            msg += f": {lib().lla_cuda_error_name(self.cuda_error).decode()} ({self.cuda_error})"
+        super().__init__(msg)
 
 
 def lib():

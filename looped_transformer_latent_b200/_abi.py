@@ -100,6 +100,8 @@ class HlaDecodeParams(ctypes.Structure):
 PROTOTYPES = {
     "lla_abi_version": (ctypes.c_int, []),
     "lla_status_str": (ctypes.c_char_p, [ctypes.c_int]),
+    "lla_last_cuda_error": (ctypes.c_int, []),
+    "lla_cuda_error_name": (ctypes.c_char_p, [ctypes.c_int]),
     "lla_write_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(WriteParams)]),
     "lla_write_latents": (ctypes.c_int, [ctypes.POINTER(WriteParams), c_vp, ctypes.c_size_t, c_vp]),
     "lla_decode_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(LlaDecodeParams)]),

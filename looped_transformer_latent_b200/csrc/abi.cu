@@ -296,7 +296,13 @@ int ws_ok(void* ws, size_t ws_bytes, size_t need) {
   return LLA_OK;
 }
 
-inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? LLA_OK : LLA_ERR_CUDA; }
+thread_local int g_last_cuda_error = 0;   // cudaError_t behind the calling thread's last LLA_ERR_CUDA
+
+inline int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return LLA_OK;
+  g_last_cuda_error = (int)e;
+  return LLA_ERR_CUDA;
+}
 
 // Optional measurement hook: record caller-owned event i (0 = before, 1 = after
 // the latent-read kernel) on the stream; captured as an external event node.
@@ -318,6 +324,10 @@ using namespace lla;
 extern "C" {
 
 int lla_abi_version(void) { return kAbiVersion; }
+
+int lla_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* lla_cuda_error_name(int cuda_error) { return cudaGetErrorName((cudaError_t)cuda_error); }
 
 const char* lla_status_str(int s) {
   switch (s) {

@@ -9,21 +9,34 @@
 //   S[row, j]  = s^K_j * (q~[row, :] . codes^K_j)
 //   O^T[v, row] += sum_j codes^V_j[v] * (P[row, j] * s^V_j)
 // so the tensor cores contract the codes and the scales are applied per token
-// on the softmax side.  Per 64-token tile:
-//   * two producer warps land the key and the value chunks (64 tokens x 64
-//     codes, 4 KB each) in fp8 landing rings, and one 1 KB box of the tile's
-//     scales;
-//   * two converter pairs widen the codes to f16 (exact: every e4m3 value is
-//     an f16 value) into 128-byte-swizzled slots, the layout the MMAs read;
-//   * two MMA warps issue S = Q~ codes^K^T (M=64 x N=64, f16 in, fp32 in
-//     TMEM) and O^T += codes^V^T P'^T (M=128 x N=rows) on independent chains;
-//   * four softmax warps scale the scores by s^K, run the online softmax and
-//     write P' = p * s^V in f16 for the value MMA (l sums p itself).
+// on the softmax side.
+//
+// Codes become f16 operands by bit placement on the integer pipe, not by the
+// conversion unit: an e4m3 byte s.eeee.mmm moved to the f16 bits
+// s.0eeee.mmm0000000 is the f16 number code * 2^-8 exactly (normal codes: the
+// exponent biases are 15 and 7; subnormal codes m * 2^-9 become the f16
+// subnormals m * 2^-17), so the scores take s^K * 2^8 and the value partials
+// are multiplied by 2^8 when written.
+//
+// Per 64-token tile, four rings carry the chunks (64 tokens x 64 codes): key
+// chunks of the first and second half of r_K (rings 0 and 1) and value chunks
+// of the first and second half of the 128-wide value groups (rings 2 and 3).
+// A ring slot holds two f16 chunk blocks (16 KB, 128-byte swizzle); the codes
+// land by TMA in its upper half and one converter warp per ring rewrites them
+// in place into the f16 blocks.  Each ring has its own MMA issuer warp, so the
+// four tcgen05 chains run concurrently (one thread's chain is bound by its own
+// issue latency):
+//   * two score chains S_a, S_b = Q~ codes^T over the two halves of r_K
+//     (M = 64 rows, N = 64 tokens, f16 in, fp32 in TMEM), summed by the
+//     softmax in a fixed order;
+//   * two value chains O^T += codes^V^T P'^T over their value groups
+//     (M = 128 value indices, N = rows);
+//   * four softmax warps scale the scores by s^K, run the online softmax
+//     (base 2, lazy rescale) and write P' = p * s^V in f16.
 // Every wait is bounded; on a timeout the CTA records an error code (the merge
 // then emits NaN), drains its copies and frees TMEM.
 #include <cuda.h>
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 
 #include "kernels.cuh"
 #include "tc_ptx.cuh"
@@ -37,22 +50,21 @@ using namespace ptx;
 constexpr int TOK = 64;
 constexpr int BLK = 8192;             // f16 chunk block: 64 tokens x 64 elements, 128-byte rows, swizzled
 constexpr int BLK8 = 4096;            // fp8 chunk block as landed: 64 tokens x 64 codes
-constexpr int LSLOT = 2 * BLK8;       // landing slot: one or two chunks
-constexpr int CSLOT = 2 * BLK;        // converted slot: one or two chunks
-constexpr int NL = 3;                 // landing slots per ring
-constexpr int NC = 2;                 // converted slots per ring
+constexpr int SLOT = 2 * BLK;         // ring slot: two f16 chunk blocks; codes land in the upper half
+constexpr int NRING = 4;              // key halves a/b, value halves a/b
 constexpr int NSB = 4;                // scale slots (one per tile)
 constexpr int SBYTES = TOK * 16;      // one tile's scales: 64 x (s^K, s^V, 8 pad bytes)
-constexpr int NBUF = 3;               // score buffers (TMEM) and P buffers (smem)
-constexpr int NTHREADS = 384;         // 0-3 softmax, 4/6 producers, 5/7 MMA, 8-9/10-11 converters
+constexpr int NBP = 2;                // P buffers (smem)
+constexpr int NTHREADS = 448;         // 0-3 softmax, 4/5 producers, 6/7 score MMA, 8/9 value MMA, 10-13 converters
 constexpr int SMEM_LIMIT = 232448;
 constexpr int MISC_BYTES = 512;
 constexpr long long WAIT_CYCLES = 1ll << 32;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t O_COL = 64 * NBUF;
+constexpr uint32_t O_COL = 128;       // S_a at column 0, S_b at 64, the value groups from 128
+constexpr float CODE_UNIT = 256.f;    // f16 operand = code * 2^-8
 
-enum : int { ERR8_LEMPTY = 51, ERR8_LFULL = 52, ERR8_CEMPTY = 53, ERR8_CFULL = 54, ERR8_Q = 55, ERR8_S = 56,
-             ERR8_P = 57, ERR8_O = 58, ERR8_SC = 59 };
+enum : int { ERR8_EMPTY = 51, ERR8_LFULL = 52, ERR8_CFULL = 54, ERR8_Q = 55, ERR8_S = 56, ERR8_P = 57,
+             ERR8_O = 58, ERR8_SC = 59 };
 
 __device__ __forceinline__ bool wait8(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err, int code,
                                       bool honour_abort = true) {
@@ -74,55 +86,76 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// four e4m3 codes (one 32-bit word, lowest byte first) -> four f16, exactly
-__device__ __forceinline__ uint2 widen4(uint32_t w) {
-  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
-  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
-  return make_uint2((uint32_t)lo.x | ((uint32_t)lo.y << 16), (uint32_t)hi.x | ((uint32_t)hi.y << 16));
+// byte permute; a selector nibble with bit 3 set fills its byte with the
+// sign bit of the selected byte
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// four e4m3 codes (one word, lowest byte first) -> four f16 equal to code * 2^-8.
+// For the pair (b0, b1) the bytes [b0 & 7F, sign(b0) fill, b1 & 7F, sign(b1)
+// fill] shifted left by 7 put each magnitude under the f16 exponent and
+// mantissa fields and each sign on bit 15 / 31; the sign fill that spills
+// into bits 16-22 (f16 mantissa bits no code sets) is cleared.
+__device__ __forceinline__ uint2 code4_to_f16(uint32_t w) {
+  const uint32_t m = w & 0x7F7F7F7Fu;
+  const uint32_t lo = (prmt(m, w, 0xD1C0u) << 7) & 0xFF80FFFFu;
+  const uint32_t hi = (prmt(m, w, 0xF3E2u) << 7) & 0xFF80FFFFu;
+  return make_uint2(lo, hi);
 }
 
 struct Layout8 {
-  int nkb, nvb;
+  int nkb, nvb, ns;
   __host__ __device__ int q_off() const { return 0; }
   __host__ __device__ int p_off() const { return nkb * BLK; }
-  __host__ __device__ int sc_off() const { return p_off() + NBUF * BLK; }
-  __host__ __device__ int lk_off() const { return sc_off() + NSB * SBYTES; }
-  __host__ __device__ int lv_off() const { return lk_off() + NL * LSLOT; }
-  __host__ __device__ int ck_off() const { return lv_off() + NL * LSLOT; }
-  __host__ __device__ int cv_off() const { return ck_off() + NC * CSLOT; }
-  __host__ __device__ int bar_off() const { return cv_off() + NC * CSLOT; }
-  __host__ __device__ int nbars() const { return 4 * NL + 4 * NC + 2 * NSB + 1 + 4 * NBUF + 2; }
+  __host__ __device__ int sc_off() const { return p_off() + NBP * BLK; }
+  __host__ __device__ int ring_off(int r) const { return sc_off() + NSB * SBYTES + r * ns * SLOT; }
+  __host__ __device__ int bar_off() const { return ring_off(NRING); }
+  __host__ __device__ int nbars() const { return 3 * NRING * ns + 2 * NSB + 1 + 3 + 2 * NBP + 4; }
   __host__ __device__ int misc_off() const { return bar_off() + 8 * nbars(); }
   __host__ __device__ int bytes() const { return misc_off() + MISC_BYTES; }
 };
 
+// Chunk range of ring r: key chunks [0, ka) and [ka, nkb); value chunks of the
+// groups [0, ga) and [ga, ngrp) (a group is two chunks, the last possibly one).
+struct Rings {
+  int nkb, nvb, ka, ngrp, ga;
+  __device__ int lo(int r) const { return r == 0 ? 0 : r == 1 ? ka : r == 2 ? 0 : 2 * ga; }
+  __device__ int hi(int r) const { return r == 0 ? ka : r == 1 ? nkb : r == 2 ? min(nvb, 2 * ga) : nvb; }
+};
+
+// 14 warps: four share an SM sub-partition's 16 K registers, so at most 128 per thread
 __global__ void __launch_bounds__(NTHREADS, 1)
 absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant__ CUtensorMap map1,
-                 const __grid_constant__ CUtensorMap mapsc, const AbsorbArgs a) {
+                 const __grid_constant__ CUtensorMap mapsc, const AbsorbArgs a, const int ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Layout8 L;
-  L.nkb = a.r_k / 64; L.nvb = a.r_v / 64;
+  L.nkb = a.r_k / 64; L.nvb = a.r_v / 64; L.ns = ns;
+  Rings R;
+  R.nkb = L.nkb; R.nvb = L.nvb;
+  R.ka = (L.nkb + 1) / 2;
+  R.ngrp = (L.nvb + 1) / 2;
+  R.ga = (R.ngrp + 1) / 2;
+  const bool two_s = R.ka < L.nkb;      // a second score chain (r_K >= 128)
+  const bool two_v = R.ga < R.ngrp;     // a second value chain (r_V > 128)
   uint8_t* q_s = base + L.q_off();
   uint8_t* p_s = base + L.p_off();
   uint8_t* sc_s = base + L.sc_off();
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L.bar_off());
-  uint64_t* lk_full = bars;               // [NL] key codes landed
-  uint64_t* lk_empty = lk_full + NL;      // [NL] key codes converted (64 arrivals)
-  uint64_t* lv_full = lk_empty + NL;
-  uint64_t* lv_empty = lv_full + NL;
-  uint64_t* ck_full = lv_empty + NL;      // [NC] f16 key chunks written (64 arrivals)
-  uint64_t* ck_empty = ck_full + NC;      // [NC] score MMAs reading them done
-  uint64_t* cv_full = ck_empty + NC;
-  uint64_t* cv_empty = cv_full + NC;
-  uint64_t* sc_full = cv_empty + NC;      // [NSB] a tile's scales landed
-  uint64_t* sc_free = sc_full + NSB;      // [NSB] softmax done with them (128 arrivals)
+  uint64_t* lfull = bars;                       // [ring][slot] codes landed (TMA)
+  uint64_t* cfull = lfull + NRING * ns;         // [ring][slot] f16 blocks written (converter)
+  uint64_t* rempty = cfull + NRING * ns;        // [ring][slot] MMAs reading the slot done
+  uint64_t* sc_full = rempty + NRING * ns;      // [NSB] a tile's scales landed
+  uint64_t* sc_free = sc_full + NSB;            // [NSB] softmax done with them (128 arrivals)
   uint64_t* q_full = sc_free + NSB;
-  uint64_t* s_full = q_full + 1;          // [NBUF]
-  uint64_t* s_free = s_full + NBUF;
-  uint64_t* p_full = s_free + NBUF;
-  uint64_t* o_done = p_full + NBUF;
-  uint64_t* fin = o_done + NBUF;          // [2] one per MMA issuer (abort path)
+  uint64_t* s_full = q_full + 1;                // [2] score chains a, b
+  uint64_t* s_free = s_full + 2;                // softmax has read S_a and S_b (128 arrivals)
+  uint64_t* p_full = s_free + 1;                // [NBP]
+  uint64_t* o_done = p_full + NBP;              // [NBP] the value chains are done with a tile
+  uint64_t* fin = o_done + NBP;                 // [4] one per MMA issuer (abort path)
   uint8_t* misc = base + L.misc_off();
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
@@ -134,39 +167,32 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
   const int tok0 = s * a.tps;
   const int tok1 = min(a.n_lat, tok0 + a.tps);
   const int ntiles = (tok1 - tok0 + TOK - 1) / TOK;
-  const int nkb = L.nkb, nvb = L.nvb, ngrp = (nvb + 1) / 2;
+  const int nkb = L.nkb, ngrp = R.ngrp;
   const int rows = a.rows, rows_pad = a.rows_pad;
 
   if (tid == 0) {
-    for (int i = 0; i < NL; ++i) {
-      mbar_init(smem_u32(&lk_full[i]), 1);
-      mbar_init(smem_u32(&lk_empty[i]), 64);
-      mbar_init(smem_u32(&lv_full[i]), 1);
-      mbar_init(smem_u32(&lv_empty[i]), 64);
-    }
-    for (int i = 0; i < NC; ++i) {
-      mbar_init(smem_u32(&ck_full[i]), 64);
-      mbar_init(smem_u32(&ck_empty[i]), 1);
-      mbar_init(smem_u32(&cv_full[i]), 64);
-      mbar_init(smem_u32(&cv_empty[i]), 1);
+    for (int i = 0; i < NRING * ns; ++i) {
+      mbar_init(smem_u32(&lfull[i]), 1);
+      mbar_init(smem_u32(&cfull[i]), 1);
+      mbar_init(smem_u32(&rempty[i]), 1);
     }
     for (int i = 0; i < NSB; ++i) {
       mbar_init(smem_u32(&sc_full[i]), 1);
       mbar_init(smem_u32(&sc_free[i]), 128);
     }
     mbar_init(smem_u32(q_full), 1);
-    for (int i = 0; i < NBUF; ++i) {
-      mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&s_free[i]), 128);
+    mbar_init(smem_u32(&s_full[0]), 1);
+    mbar_init(smem_u32(&s_full[1]), 1);
+    mbar_init(smem_u32(s_free), 128);
+    for (int i = 0; i < NBP; ++i) {
       mbar_init(smem_u32(&p_full[i]), 128);
-      mbar_init(smem_u32(&o_done[i]), 1);
+      mbar_init(smem_u32(&o_done[i]), two_v ? 2 : 1);
     }
-    mbar_init(smem_u32(fin), 1);
-    mbar_init(smem_u32(fin + 1), 1);
+    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&fin[i]), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 6) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
   }
@@ -180,40 +206,67 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4 || warp == 6) {
+  if (warp == 4 || warp == 5) {
     // ----------------------------------------------------------- producers --
-    // Warp 4: Q~ (one bulk copy), then per tile the scales and the key chunks;
-    // warp 6: the value chunks.  Copies carry two chunks (one for an odd last
-    // chunk); copy i of a ring goes to landing slot i mod NL.
+    // Warp 4: Q~ (one bulk copy), the tiles' scales and the key copies of
+    // rings 0 and 1; warp 5: the value copies of rings 2 and 3.  A copy is two
+    // chunks (one for an odd last chunk); copy i of a ring goes to slot i mod
+    // ns.  The thread polls its rings without blocking, so a ring whose slots
+    // are all in use never holds back the other's copies.
     if (lane == 0) {
       const bool kside = warp == 4;
-      const int nb = kside ? nkb : nvb, c0 = kside ? 0 : nkb;
-      uint8_t* ring = base + (kside ? L.lk_off() : L.lv_off());
-      const uint32_t full0 = smem_u32(kside ? lk_full : lv_full), empty0 = smem_u32(kside ? lk_empty : lv_empty);
+      const int r0 = kside ? 0 : 2, c0 = kside ? 0 : nkb;
       const uint32_t qb = smem_u32(q_full);
       if (kside) {
         mbar_arrive_tx(qb, nkb * BLK);
         bulk_load(smem_u32(q_s), a.qbf + (size_t)b * nkb * (BLK / 2), nkb * BLK, qb);
       }
-      uint32_t i = 0;
-      int nsc = 0;
+      uint32_t cnt[2] = {0, 0};
+      int tile[2] = {0, 0}, chunk[2] = {R.lo(r0), R.lo(r0 + 1)};
+      bool done[2] = {R.lo(r0) >= R.hi(r0), R.lo(r0 + 1) >= R.hi(r0 + 1)};
+      int nsc = kside ? 0 : ntiles;
       bool ok = true;
-      for (int n = 0; n < ntiles && ok; ++n) {
-        const int y = tok0 + n * TOK;
-        if (kside) {
-          const int ss = n % NSB;
-          if (!wait8(smem_u32(&sc_free[ss]), ((n / NSB) & 1) ^ 1, abort_flag, a.err, ERR8_SC)) { ok = false; break; }
-          mbar_arrive_tx(smem_u32(&sc_full[ss]), SBYTES);
-          tma_load_3d(smem_u32(sc_s + ss * SBYTES), &mapsc, smem_u32(&sc_full[ss]), 0, y, b);
-          nsc = n + 1;
+      long long t_last = clock64();
+      while (true) {
+        bool progress = false;
+        if (nsc < ntiles) {
+          const int ss = nsc % NSB;
+          if (mbar_test_wait(smem_u32(&sc_free[ss]), ((nsc / NSB) & 1) ^ 1)) {
+            mbar_arrive_tx(smem_u32(&sc_full[ss]), SBYTES);
+            tma_load_3d(smem_u32(sc_s + ss * SBYTES), &mapsc, smem_u32(&sc_full[ss]), 0, tok0 + nsc * TOK, b);
+            ++nsc;
+            progress = true;
+          }
         }
-        for (int c = 0; c < nb; c += 2, ++i) {
-          const int cnt = nb - c >= 2 ? 2 : 1;
-          const uint32_t slot = i % NL;
-          if (!wait8(empty0 + 8 * slot, ((i / NL) & 1) ^ 1, abort_flag, a.err, ERR8_LEMPTY)) { ok = false; break; }
-          mbar_arrive_tx(full0 + 8 * slot, cnt * BLK8);
-          tma_load_4d(smem_u32(ring + slot * LSLOT), cnt == 2 ? (const void*)&map2 : (const void*)&map1,
-                      full0 + 8 * slot, 0, y, c0 + c, b);
+        for (int k = 0; k < 2; ++k) {
+          if (done[k]) continue;
+          const int r = r0 + k;
+          const uint32_t slot = cnt[k] % ns, ph = cnt[k] / ns;
+          if (!mbar_test_wait(smem_u32(&rempty[r * ns + slot]), (ph & 1) ^ 1)) continue;
+          const int c = chunk[k], w = R.hi(r) - c >= 2 ? 2 : 1;
+          const uint32_t fb = smem_u32(&lfull[r * ns + slot]);
+          mbar_arrive_tx(fb, w * BLK8);
+          tma_load_4d(smem_u32(base + L.ring_off(r) + slot * SLOT + BLK),
+                      w == 2 ? (const void*)&map2 : (const void*)&map1, fb, 0, tok0 + tile[k] * TOK, c0 + c, b);
+          ++cnt[k];
+          chunk[k] = c + 2;
+          if (chunk[k] >= R.hi(r)) {
+            chunk[k] = R.lo(r);
+            if (++tile[k] == ntiles) done[k] = true;
+          }
+          progress = true;
+        }
+        if (done[0] && done[1] && nsc == ntiles) break;
+        if (progress) {
+          t_last = clock64();
+        } else if (*abort_flag) {
+          ok = false;
+          break;
+        } else if (clock64() - t_last > WAIT_CYCLES) {
+          *abort_flag = 1;
+          atomicExch(a.err, ERR8_EMPTY);
+          ok = false;
+          break;
         }
       }
       if (!ok) {
@@ -223,110 +276,118 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
           for (int n = max(0, nsc - NSB); n < nsc; ++n)
             wait8(smem_u32(&sc_full[n % NSB]), (n / NSB) & 1, abort_flag, nullptr, 0, false);
         }
-        for (uint32_t k = (i > (uint32_t)NL ? i - NL : 0); k < i; ++k)
-          wait8(full0 + 8 * (k % NL), (k / NL) & 1, abort_flag, nullptr, 0, false);
+        for (int k = 0; k < 2; ++k)
+          for (uint32_t i = (cnt[k] > (uint32_t)ns ? cnt[k] - ns : 0); i < cnt[k]; ++i)
+            wait8(smem_u32(&lfull[(r0 + k) * ns + i % ns]), (i / ns) & 1, abort_flag, nullptr, 0, false);
       }
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 10) {
     // ----------------------------------------------------------- converters --
-    // Warps 8-9 widen the key chunks, 10-11 the value chunks, copy by copy in
-    // the producers' order: 16 codes (one 16-byte piece of a landed token row)
-    // per task become two 16-byte f16 pieces of the swizzled slot.
-    const bool kside = warp < 10;
-    const int ct = tid - (kside ? 256 : 320);      // 0..63
-    const int nb = kside ? nkb : nvb;
-    const uint8_t* land = base + (kside ? L.lk_off() : L.lv_off());
-    uint8_t* conv = base + (kside ? L.ck_off() : L.cv_off());
-    const uint32_t lfull = smem_u32(kside ? lk_full : lv_full), lempty = smem_u32(kside ? lk_empty : lv_empty);
-    const uint32_t cfull = smem_u32(kside ? ck_full : cv_full), cempty = smem_u32(kside ? ck_empty : cv_empty);
-    uint32_t i = 0;
+    // Warp 10 + r rewrites ring r's landed codes into f16 blocks, copy by copy
+    // in the producer's order.  Per chunk each lane loads 8 x 16 codes (the
+    // warp reads the 4 KB block contiguously), the warp synchronises (the
+    // second chunk's f16 block overlaps its own codes), then each lane stores
+    // 8 x 32 bytes into the swizzled rows.
+    const int r = warp - 10;
+    uint8_t* ring = base + L.ring_off(r);
+    uint32_t cnt = 0;
     bool ok = true;
     for (int n = 0; n < ntiles && ok; ++n) {
-      for (int c = 0; c < nb && ok; c += 2, ++i) {
-        const int cnt = nb - c >= 2 ? 2 : 1;
-        const uint32_t ls = i % NL, cs = i % NC;
-        if (!wait8(lfull + 8 * ls, (i / NL) & 1, abort_flag, a.err, ERR8_LFULL) ||
-            !wait8(cempty + 8 * cs, ((i / NC) & 1) ^ 1, abort_flag, a.err, ERR8_CEMPTY)) {
-          ok = false;
-          break;
-        }
-        const uint8_t* src = land + ls * LSLOT;
-        uint8_t* dst = conv + cs * CSLOT;
-        for (int t = ct; t < cnt * 256; t += 64) {
-          const int j = t >> 8, row = (t >> 2) & 63, p = t & 3;
-          const uint4 w = *reinterpret_cast<const uint4*>(src + j * BLK8 + row * 64 + p * 16);
-          const uint2 h0 = widen4(w.x), h1 = widen4(w.y), h2 = widen4(w.z), h3 = widen4(w.w);
-          uint8_t* drow = dst + j * BLK + row * 128;
-          *reinterpret_cast<uint4*>(drow + (((2 * p) ^ (row & 7)) << 4)) = make_uint4(h0.x, h0.y, h1.x, h1.y);
-          *reinterpret_cast<uint4*>(drow + (((2 * p + 1) ^ (row & 7)) << 4)) = make_uint4(h2.x, h2.y, h3.x, h3.y);
+      for (int c = R.lo(r); c < R.hi(r); c += 2, ++cnt) {
+        const int w = R.hi(r) - c >= 2 ? 2 : 1;
+        const uint32_t slot = cnt % ns, ph = cnt / ns;
+        if (!wait8(smem_u32(&lfull[r * ns + slot]), ph & 1, abort_flag, a.err, ERR8_LFULL)) { ok = false; break; }
+        uint8_t* sl = ring + slot * SLOT;
+        for (int j = 0; j < w; ++j) {
+          const uint4* src = reinterpret_cast<const uint4*>(sl + BLK + j * BLK8);
+          uint4 cw[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) cw[k] = src[lane + 32 * k];
+          __syncwarp();
+          // 16-byte piece lane + 32k holds codes 16p..16p+15 of token row lane/4 + 8k
+          const int p = lane & 3, sw = (lane >> 2) & 7;
+          uint8_t* dst = sl + j * BLK + (lane >> 2) * 128;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint2 h0 = code4_to_f16(cw[k].x), h1 = code4_to_f16(cw[k].y);
+            const uint2 h2 = code4_to_f16(cw[k].z), h3 = code4_to_f16(cw[k].w);
+            uint8_t* drow = dst + k * 8 * 128;
+            *reinterpret_cast<uint4*>(drow + (((2 * p) ^ sw) << 4)) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+            *reinterpret_cast<uint4*>(drow + (((2 * p + 1) ^ sw) << 4)) = make_uint4(h2.x, h2.y, h3.x, h3.y);
+          }
+          __syncwarp();
         }
         fence_proxy_async_smem();
-        mbar_arrive(lempty + 8 * ls);
-        mbar_arrive(cfull + 8 * cs);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&cfull[r * ns + slot]));
       }
     }
-  } else if (warp == 5 || warp == 7) {
+  } else if (warp >= 6) {
     // --------------------------------------------------------- MMA issuers --
-    if (lane == 0) {
-      const bool scores = warp == 5;
+    // Warps 6/7: score chains a/b over rings 0/1; warps 8/9: value chains a/b
+    // over rings 2/3.
+    const int r = warp - 6;
+    const bool scores = r < 2;
+    const bool has_chain = scores ? (r == 0 || two_s) : (r == 2 || two_v);
+    if (lane == 0 && has_chain) {
       const uint32_t idS = idesc_f16(64, 64, false, false);
       const uint32_t idO = idesc_f16(128, rows_pad, true, false);
       const uint64_t q_desc = smem_desc_sw128(smem_u32(q_s), 16, 1024);
-      const uint64_t k_desc = smem_desc_sw128(smem_u32(base + L.ck_off()), 16, 1024);
-      const uint64_t v_desc = smem_desc_sw128(smem_u32(base + L.cv_off()), BLK, 1024);
+      const uint64_t k_desc = smem_desc_sw128(smem_u32(base + L.ring_off(r)), 16, 1024);
+      const uint64_t v_desc = smem_desc_sw128(smem_u32(base + L.ring_off(r)), BLK, 1024);
       const uint64_t p_desc = smem_desc_sw128(smem_u32(p_s), 16, 1024);
-      const uint32_t ckf = smem_u32(ck_full), cke = smem_u32(ck_empty);
-      const uint32_t cvf = smem_u32(cv_full), cve = smem_u32(cv_empty);
       bool ok = !scores || wait8(smem_u32(q_full), 0, abort_flag, a.err, ERR8_Q);
-      uint32_t i = 0;
+      uint32_t cnt = 0;
       if (scores) {
+        const uint32_t d = tmem + r * 64;
         for (int n = 0; n < ntiles && ok; ++n) {
-          const int buf = n % NBUF;
-          if (n >= NBUF && !wait8(smem_u32(&s_free[buf]), ((n - NBUF) / NBUF) & 1, abort_flag, a.err, ERR8_S)) { ok = false; break; }
+          if (n >= 1 && !wait8(smem_u32(s_free), (n - 1) & 1, abort_flag, a.err, ERR8_S)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t d = tmem + buf * 64;
-          for (int kb = 0; kb < nkb && ok; kb += 2, ++i) {
-            const int cnt = nkb - kb >= 2 ? 2 : 1;
-            const uint32_t slot = i % NC;
-            if (!wait8(ckf + 8 * slot, (i / NC) & 1, abort_flag, a.err, ERR8_CFULL)) { ok = false; break; }
+          uint32_t acc = 0;
+          for (int c = R.lo(r); c < R.hi(r) && ok; c += 2, ++cnt) {
+            const int w = R.hi(r) - c >= 2 ? 2 : 1;
+            const uint32_t slot = cnt % ns, ph = cnt / ns;
+            if (!wait8(smem_u32(&cfull[r * ns + slot]), ph & 1, abort_flag, a.err, ERR8_CFULL)) { ok = false; break; }
             tc_fence_after();
-            for (int j = 0; j < cnt; ++j) {
-              const uint64_t ad = q_desc + (uint64_t)(((kb + j) * BLK) >> 4);
-              const uint64_t bd = k_desc + (uint64_t)((slot * CSLOT + j * BLK) >> 4);
+            for (int j = 0; j < w; ++j) {
+              const uint64_t ad = q_desc + (uint64_t)(((c + j) * BLK) >> 4);
+              const uint64_t bd = k_desc + (uint64_t)((slot * SLOT + j * BLK) >> 4);
 #pragma unroll
-              for (int k16 = 0; k16 < 4; ++k16)
-                mma_bf16(d, ad + 2 * k16, bd + 2 * k16, idS, ((kb + j) | k16) != 0);
+              for (int k16 = 0; k16 < 4; ++k16) {
+                mma_bf16(d, ad + 2 * k16, bd + 2 * k16, idS, acc);
+                acc = 1;
+              }
             }
-            mma_commit(cke + 8 * slot);
+            mma_commit(smem_u32(&rempty[r * ns + slot]));
           }
           if (!ok) break;
-          mma_commit(smem_u32(&s_full[buf]));
+          mma_commit(smem_u32(&s_full[r]));
         }
       } else {
         for (int m = 0; m < ntiles && ok; ++m) {
-          const int buf = m % NBUF;
-          if (!wait8(smem_u32(&p_full[buf]), (m / NBUF) & 1, abort_flag, a.err, ERR8_P)) { ok = false; break; }
+          const int buf = m % NBP;
+          if (!wait8(smem_u32(&p_full[buf]), (m / NBP) & 1, abort_flag, a.err, ERR8_P)) { ok = false; break; }
           tc_fence_after();
           const uint64_t bd = p_desc + (uint64_t)((buf * BLK) >> 4);
-          for (int vb = 0; vb < nvb && ok; vb += 2, ++i) {
-            const uint32_t slot = i % NC;
-            if (!wait8(cvf + 8 * slot, (i / NC) & 1, abort_flag, a.err, ERR8_CFULL)) { ok = false; break; }
+          for (int c = R.lo(r); c < R.hi(r) && ok; c += 2, ++cnt) {
+            const uint32_t slot = cnt % ns, ph = cnt / ns;
+            if (!wait8(smem_u32(&cfull[r * ns + slot]), ph & 1, abort_flag, a.err, ERR8_CFULL)) { ok = false; break; }
             tc_fence_after();
             // one M=128 MMA covers both chunks of the slot (BLK apart); for a
-            // one-chunk copy rows 64..127 are value indices >= r_v, never read
-            const uint32_t dO = tmem + O_COL + (vb >> 1) * rows_pad;
-            const uint64_t ad = v_desc + (uint64_t)((slot * CSLOT) >> 4);
+            // one-chunk group rows 64..127 are value indices >= r_v, never read
+            const uint32_t dO = tmem + O_COL + (c >> 1) * rows_pad;
+            const uint64_t ad = v_desc + (uint64_t)((slot * SLOT) >> 4);
 #pragma unroll
             for (int k16 = 0; k16 < 4; ++k16)
               mma_bf16(dO, ad + 128 * k16, bd + 2 * k16, idO, (m > 0 || k16 > 0) ? 1u : 0u);
-            mma_commit(cve + 8 * slot);
+            mma_commit(smem_u32(&rempty[r * ns + slot]));
           }
           if (!ok) break;
           mma_commit(smem_u32(&o_done[buf]));
         }
       }
       if (!ok) {
-        const uint32_t f = smem_u32(fin) + (scores ? 0 : 8);
+        const uint32_t f = smem_u32(&fin[r]);
         mma_commit(f);
         wait8(f, 0, abort_flag, nullptr, 0, false);
       }
@@ -342,31 +403,37 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int n = 0; n < ntiles; ++n) {
-      const int buf = n % NBUF, ss = n % NSB;
+      const int buf = n % NBP, ss = n % NSB;
       if (tid == 0)
-        lead[0] = wait8(smem_u32(&s_full[buf]), (n / NBUF) & 1, abort_flag, a.err, ERR8_S) &&
+        lead[0] = wait8(smem_u32(&s_full[0]), n & 1, abort_flag, a.err, ERR8_S) &&
+                  (!two_s || wait8(smem_u32(&s_full[1]), n & 1, abort_flag, a.err, ERR8_S)) &&
                   wait8(smem_u32(&sc_full[ss]), (n / NSB) & 1, abort_flag, a.err, ERR8_SC);
       named_sync(1, 128);
       if (!lead[0]) { ok = false; break; }
       tc_fence_after();
       float sc[64];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld16(tmem + buf * 64 + q * 16 + lane_off, sc + q * 16);
+      for (int q = 0; q < 4; ++q) {
+        tmem_ld16(tmem + q * 16 + lane_off, sc + q * 16);
+        if (two_s) {
+          float t[16];
+          tmem_ld16(tmem + 64 + q * 16 + lane_off, t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) sc[q * 16 + j] += t[j];
+        }
+      }
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(smem_u32(&s_free[buf]));
+      mbar_arrive(smem_u32(s_free));
       const float* scl = reinterpret_cast<const float*>(sc_s + ss * SBYTES);   // [64][4]: s^K, s^V, pad
       const int nvalid = min(TOK, min(tok1, rlim) - (tok0 + n * TOK));
 #pragma unroll
-      for (int c = 0; c < 64; ++c) sc[c] = c < nvalid ? sc[c] * scl[4 * c] : -INFINITY;
-      float mx[16];
+      for (int c = 0; c < 64; ++c) sc[c] = c < nvalid ? sc[c] * (scl[4 * c] * CODE_UNIT) : -INFINITY;
+      float mx[4] = {sc[0], sc[1], sc[2], sc[3]};
 #pragma unroll
-      for (int c = 0; c < 16; ++c) mx[c] = fmaxf(fmaxf(sc[c], sc[c + 16]), fmaxf(sc[c + 32], sc[c + 48]));
-#pragma unroll
-      for (int w = 8; w > 0; w >>= 1)
-#pragma unroll
-        for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
-      const float tmax = mx[0];
+      for (int c = 4; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], sc[c]);
+      const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       bool need = false;
       float alpha = 1.f;
       if (active) {
@@ -378,24 +445,37 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
           need = true;
         }
       }
-      uint32_t pk[32];
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (n >= NBP) {
+        // P buffer `buf` is free once O(n-NBP) has completed
+        if (tid == 0) lead[2] = wait8(smem_u32(&o_done[buf]), ((n - NBP) / NBP) & 1, abort_flag, a.err, ERR8_O);
+        named_sync(1, 128);
+        if (!lead[2]) { ok = false; break; }
+      }
       // inactive rows, and rows with no token yet, give p = 0
       const float mneg = (active && m_run != -INFINITY) ? -m_run : -INFINITY;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      uint8_t* prow = p_s + buf * BLK + r * 128;
+      const bool store = owner && r < rows_pad;
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float p0 = ex2(sc[c] + mneg);
-        const float p1 = ex2(sc[c + 1] + mneg);
-        ps[(c >> 1) & 7] += p0 + p1;
-        pk[c >> 1] = pack_f16(p0 * scl[4 * c + 1], p1 * scl[4 * c + 5]);
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 8 * ch + 2 * e;
+          const float p0 = ex2(sc[c] + mneg);
+          const float p1 = ex2(sc[c + 1] + mneg);
+          ps[(c >> 1) & 7] += p0 + p1;
+          pk[e] = pack_f16(p0 * scl[4 * c + 1], p1 * scl[4 * c + 5]);
+        }
+        if (store) *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       l_run = l_run * alpha + psum;
-      mbar_arrive(smem_u32(&sc_free[ss]));   // this thread is done with the tile's scales
       if (named_any(1, 128, need)) {
-        // rescale the TMEM accumulators once O(n-1) has landed
+        // rescale the TMEM accumulators once O(n-1) has landed (before P(n)
+        // is published, after the scores are dead: fewer live registers)
         if (owner) alpha_s[r] = alpha;
-        if (tid == 0) lead[1] = wait8(smem_u32(&o_done[(n - 1) % NBUF]), ((n - 1) / NBUF) & 1, abort_flag, a.err, ERR8_O);
+        if (tid == 0) lead[1] = wait8(smem_u32(&o_done[(n - 1) % NBP]), ((n - 1) / NBP) & 1, abort_flag, a.err, ERR8_O);
         named_sync(1, 128);
         if (!lead[1]) { ok = false; break; }
         tc_fence_after();
@@ -413,24 +493,13 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
         tmem_wait_st();
         tc_fence_before();
       }
-      if (n >= NBUF) {
-        // P buffer `buf` is free once O(n-NBUF) has completed
-        if (tid == 0) lead[2] = wait8(smem_u32(&o_done[buf]), ((n - NBUF) / NBUF) & 1, abort_flag, a.err, ERR8_O);
-        named_sync(1, 128);
-        if (!lead[2]) { ok = false; break; }
-      }
-      if (owner && r < rows_pad) {
-        uint8_t* prow = p_s + buf * BLK + r * 128;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-      }
+      mbar_arrive(smem_u32(&sc_free[ss]));   // this thread is done with the tile's scales
       fence_proxy_async_smem();
       mbar_arrive(smem_u32(&p_full[buf]));
     }
     if (ok) {
-      if (tid == 0) lead[3] = wait8(smem_u32(&o_done[(ntiles - 1) % NBUF]), ((ntiles - 1) / NBUF) & 1, abort_flag, a.err, ERR8_O);
+      if (tid == 0)
+        lead[3] = wait8(smem_u32(&o_done[(ntiles - 1) % NBP]), ((ntiles - 1) / NBP) & 1, abort_flag, a.err, ERR8_O);
       named_sync(1, 128);
       ok = lead[3] != 0;
     }
@@ -451,7 +520,7 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
           if (vv < a.r_v) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (cc + j < rows) py[(int64_t)(cc + j) * a.r_v + vv] = v[j];
+              if (cc + j < rows) py[(int64_t)(cc + j) * a.r_v + vv] = v[j] * CODE_UNIT;
           }
         }
       }
@@ -460,23 +529,26 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 6) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
-int fp8_smem(int r_k, int r_v) {
+int fp8_smem(int r_k, int r_v, int ns) {
   Layout8 L;
-  L.nkb = r_k / 64; L.nvb = r_v / 64;
+  L.nkb = r_k / 64; L.nvb = r_v / 64; L.ns = ns;
   return L.bytes() + 1024;
 }
+
+// two slots per ring where shared memory allows, else one
+int fp8_slots(int r_k, int r_v) { return fp8_smem(r_k, r_v, 2) <= SMEM_LIMIT ? 2 : 1; }
 
 }  // namespace
 
 bool absorb_fp8_supported(int r_k, int r_v, int rows) {
   if (r_k % 64 || r_v % 64 || r_k < 64 || r_v < 64 || r_k > 768) return false;
-  if (rows < 1 || rows > 64 || fp8_smem(r_k, r_v) > SMEM_LIMIT) return false;
+  if (rows < 1 || rows > 64 || fp8_smem(r_k, r_v, 1) > SMEM_LIMIT) return false;
   const int ngrp = (r_v / 64 + 1) / 2;
   return O_COL + (uint32_t)(ngrp * absorb_tc_rows_pad(rows)) <= TMEM_COLS;
 }
@@ -509,11 +581,12 @@ cudaError_t launch_absorb_split_fp8(const AbsorbArgs& a, cudaStream_t st) {
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const int smem = fp8_smem(a.r_k, a.r_v);
+  const int ns = fp8_slots(a.r_k, a.r_v);
+  const int smem = fp8_smem(a.r_k, a.r_v, ns);
   cudaError_t e = cudaFuncSetAttribute(absorb_split_fp8, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.S, a.B);
-  absorb_split_fp8<<<grid, NTHREADS, smem, st>>>(map2, map1, mapsc, a);
+  absorb_split_fp8<<<grid, NTHREADS, smem, st>>>(map2, map1, mapsc, a, ns);
   return cudaGetLastError();
 }
 

@@ -421,6 +421,161 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(const __grid_consta
   }
 }
 
+// Windows of 16 tokens and more, in chunks of at most WC_TOK tokens: one CTA
+// per (chunk, loop x group of 8 heads, sequence) lands its whole chunk with
+// one pair of TMA boxes (per-token bulk copies where the chunk wraps around
+// the ring's end), one warp per head.  Lanes hold 4 features each: a lane's
+// partial dot products for the chunk's tokens are summed across the warp by a
+// transposing butterfly (each exchange halves the values a lane holds, so the
+// whole chunk takes WC_TOK shuffles instead of 5 per token), which leaves
+// token u's score in lanes u * (32 / WC_TOK) ..; the values are then
+// accumulated with each token's weight broadcast from its lane.  One tile, so
+// the partial state is the chunk's own maximum, sum and weighted values.
+template <bool BF16>
+struct WcTraits { static constexpr int TOK = BF16 ? 16 : 8; };
+
+// v[u] (u < N) summed over the warp's 32 lanes; lane l receives the total of
+// v[l / (32 / N)].
+template <int N>
+__device__ __forceinline__ float butterfly_transpose_sum(float (&v)[N], int lane) {
+  int steps = 0;
+#pragma unroll
+  for (int half = N / 2; half >= 1; half /= 2, ++steps) {
+    const int mask = 16 >> steps;
+    const bool up = (lane & mask) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float lo = v[i], hi = v[i + half];
+      v[i] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, mask);
+    }
+  }
+  float s = v[0];
+#pragma unroll
+  for (int o = 16 / N; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(32 * WB_HEADS) window_chunk(const __grid_constant__ RingMaps maps, WindowArgs w) {
+  typedef WinTraits<BF16> Tr;
+  constexpr int TC = WcTraits<BF16>::TOK;
+  constexpr int G = 32 / TC;   // lanes holding one token's score
+  constexpr int ES = BF16 ? 2 : 4;
+  extern __shared__ __align__(128) uint8_t wsm[];
+  const int chunk = blockIdx.x, tt = blockIdx.y / w.HG, hg = blockIdx.y % w.HG, b = blockIdx.z;
+  const int t = w.t0 + tt, h0 = hg * WB_HEADS;
+  const int nh = min(WB_HEADS, w.H - h0);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t hbytes = (uint32_t)w.d_h * ES;
+  const uint32_t tok_bytes = nh * hbytes;                  // one token's head-group slice
+  const uint32_t half = (uint32_t)w.cpt * WB_HEADS * hbytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(wsm + 2 * half);
+  const int j0 = chunk * w.cpt, nt = min(w.n_win, j0 + w.cpt) - j0;
+  if (threadIdx.x == 0) {
+    const uint32_t bar = ptx::smem_u32(full);
+    ptx::mbar_init(bar, 1);
+    ptx::fence_mbar_init();
+    const uint32_t dk = ptx::smem_u32(wsm), dv = dk + half;
+    const int s0 = (w.win_start + j0) % w.Wcap;
+    if (s0 + nt <= w.Wcap) {
+      // consecutive ring slots: one box each for K and V (slots past the
+      // chunk, or past the ring's end, land too and are never read)
+      ptx::mbar_arrive_tx(bar, 2u * half);
+      ptx::tma_load_5d(dk, &maps.k, bar, 0, h0, s0, t, b);
+      ptx::tma_load_5d(dv, &maps.v, bar, 0, h0, s0, t, b);
+    } else {
+      const char* kbase = reinterpret_cast<const char*>(w.wk) + ((int64_t)b * w.wins_b) * ES;
+      const char* vbase = reinterpret_cast<const char*>(w.wv) + ((int64_t)b * w.wins_b) * ES;
+      ptx::mbar_arrive_tx(bar, 2u * nt * tok_bytes);
+      for (int u = 0; u < nt; ++u) {
+        const int slot = (w.win_start + j0 + u) % w.Wcap;
+        const int64_t off = (((int64_t)t * w.Wcap + slot) * w.H + h0) * (int64_t)hbytes;
+        ptx::bulk_load(dk + u * WB_HEADS * hbytes, kbase + off, tok_bytes, bar);
+        ptx::bulk_load(dv + u * WB_HEADS * hbytes, vbase + off, tok_bytes, bar);
+      }
+    }
+  }
+  __syncthreads();
+
+  // the rotated, scaled query while the copies are in flight
+  const int d0 = 4 * lane;
+  const bool dv = warp < nh && d0 < w.d_h;
+  const int row = w.row0 + tt * w.H + h0 + warp;
+  float qv[4] = {0.f, 0.f, 0.f, 0.f};
+  if (dv) {
+    float c0 = 1.f, s0 = 0.f, c1 = 1.f, s1 = 0.f;
+    if (w.rotate) {
+      c0 = w.rot[2 * lane].x; s0 = w.rot[2 * lane].y;
+      c1 = w.rot[2 * lane + 1].x; s1 = w.rot[2 * lane + 1].y;
+    }
+    const float* q = w.q + (int64_t)b * w.q_sb + (int64_t)row * w.q_srow + d0;
+    const float x0 = q[0], y0 = q[1], x1 = q[2], y1 = q[3];
+    qv[0] = (x0 * c0 - y0 * s0) * w.qmul;
+    qv[1] = (x0 * s0 + y0 * c0) * w.qmul;
+    qv[2] = (x1 * c1 - y1 * s1) * w.qmul;
+    qv[3] = (x1 * s1 + y1 * c1) * w.qmul;
+  }
+  const uint32_t bar = ptx::smem_u32(full);
+  bool ok = ptx::mbar_try_wait(bar, 0);
+  if (!ok) {
+    const long long t0c = clock64();
+    while (!(ok = ptx::mbar_try_wait(bar, 0)) && clock64() - t0c <= WB_WAIT) {
+    }
+  }
+  if (__syncthreads_or(!ok)) {
+    if (threadIdx.x == 0) {
+      if (w.err) atomicExch(w.err, ERR_WINDOW_TIMEOUT);
+      // leave no copy in flight: wait (bounded) once more for the chunk
+      const long long t0c = clock64();
+      while (!ptx::mbar_try_wait(bar, 0) && clock64() - t0c < WB_WAIT) {
+      }
+    }
+    return;
+  }
+  if (warp >= nh) return;
+  const uint8_t* ks = wsm + (size_t)warp * hbytes + (size_t)d0 * ES;
+  const uint8_t* vs = ks + half;
+  float part[TC];
+#pragma unroll
+  for (int u = 0; u < TC; ++u) {
+    part[u] = 0.f;
+    if (dv && u < nt) {
+      float kk[4];
+      Tr::unpack(*reinterpret_cast<const typename Tr::raw_t*>(ks + (size_t)u * WB_HEADS * hbytes), kk);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) part[u] = fmaf(qv[e], kk[e], part[u]);
+    }
+  }
+  const int tok = lane / G;
+  float sc = butterfly_transpose_sum<TC>(part, lane);
+  if (tok >= nt) sc = -INFINITY;
+  const float m = ptx::redux_max(sc);
+  const float p = tok < nt ? exp2f(sc - m) : 0.f;
+  float l = (lane % G) == 0 ? p : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int u = 0; u < TC; ++u) {
+    const float pu = __shfl_sync(0xffffffffu, p, u * G);
+    if (dv && u < nt) {
+      float vv[4];
+      Tr::unpack(*reinterpret_cast<const typename Tr::raw_t*>(vs + (size_t)u * WB_HEADS * hbytes), vv);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] = fmaf(pu, vv[e], acc[e]);
+    }
+  }
+  const int64_t o = ((int64_t)chunk * w.B + b) * w.rows_total + row;
+  if (lane == 0) {
+    w.win_ml[o * 2] = m;
+    w.win_ml[o * 2 + 1] = l;
+  }
+  if (dv) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w.win_y[o * w.d_h + d0 + e] = acc[e];
+  }
+}
+
 // ---------------------------------------------------------------- merge --
 // Combine split partials and the window partial of each (sequence, row) for
 // head-space partials (LLA reconstruct):
@@ -597,10 +752,21 @@ bool window_bulk_ok(int dtype, int d_h) {
 }
 
 int window_chunks(int B, int nt, int H, int n_win, int dtype, int d_h, int num_sms, int* cpt, int* HG) {
-  // about four CTAs per SM; chunks of a multiple of 8 tokens.  Windows of at
-  // least 16 tokens use the bulk-copy kernel (groups of 8 heads per CTA).
+  // Windows of at least 16 tokens use the bulk-copy kernels (groups of 8 heads
+  // per CTA): chunks of at most WC_TOK tokens, one tile each (window_chunk),
+  // when that takes at most kMaxWindowChunks chunks; longer windows stream
+  // chunks of a multiple of 8 tokens through window_bulk, about four CTAs per
+  // SM.  Shorter windows use the register kernel.
   const bool bulk = n_win >= 16 && window_bulk_ok(dtype, d_h);
   *HG = bulk ? (H + WB_HEADS - 1) / WB_HEADS : 0;
+  if (bulk) {
+    const int tc = dtype == LLA_BF16 ? WcTraits<true>::TOK : WcTraits<false>::TOK;
+    const int S = (n_win + tc - 1) / tc;
+    if (S <= kMaxWindowChunks) {
+      *cpt = (n_win + S - 1) / S;
+      return (n_win + *cpt - 1) / *cpt;
+    }
+  }
   const long ctas = (long)B * nt * (bulk ? *HG : 1);
   long S = ctas > 0 ? (4L * num_sms + ctas - 1) / ctas : 1;
   S = std::max(1L, std::min(S, std::min((long)kMaxWindowChunks, (long)((n_win + 7) / 8))));
@@ -624,8 +790,11 @@ cudaError_t launch_window(const WindowArgs& w_in, cudaStream_t st) {
   const int nt = w.rows / w.H;
   if (w.HG > 0) {
     const int es = w.dtype == LLA_BF16 ? 2 : 4;
-    const int ts = w.dtype == LLA_BF16 ? WbTraits<true>::TS : WbTraits<false>::TS;
-    const size_t smem = (size_t)WB_NST * 2 * ts * WB_HEADS * w.d_h * es + 8 * WB_NST + 16;
+    const int tc = w.dtype == LLA_BF16 ? WcTraits<true>::TOK : WcTraits<false>::TOK;
+    const bool one_tile = w.cpt <= tc;   // window_chunk: the whole chunk in one tile
+    const int ts = one_tile ? w.cpt : w.dtype == LLA_BF16 ? WbTraits<true>::TS : WbTraits<false>::TS;
+    const size_t smem = one_tile ? (size_t)2 * ts * WB_HEADS * w.d_h * es + 16
+                                 : (size_t)WB_NST * 2 * ts * WB_HEADS * w.d_h * es + 8 * WB_NST + 16;
     dim3 grid(w.Sw, nt * w.HG, w.B);
     RingMaps maps;
     TmapEncodeFn enc = tmap_encoder();
@@ -643,7 +812,17 @@ cudaError_t launch_window(const WindowArgs& w_in, cudaStream_t st) {
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     if (!mapped) goto register_kernel;   // no tensor-map view: same chunks on the register kernel
     cudaError_t e;
-    if (w.dtype == LLA_BF16) {
+    if (one_tile) {
+      if (w.dtype == LLA_BF16) {
+        e = cudaFuncSetAttribute(window_chunk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        window_chunk<true><<<grid, 32 * WB_HEADS, smem, st>>>(maps, w);
+      } else {
+        e = cudaFuncSetAttribute(window_chunk<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        window_chunk<false><<<grid, 32 * WB_HEADS, smem, st>>>(maps, w);
+      }
+    } else if (w.dtype == LLA_BF16) {
       e = cudaFuncSetAttribute(window_bulk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
       window_bulk<true><<<grid, 32 * WB_HEADS, smem, st>>>(maps, w);

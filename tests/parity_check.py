@@ -46,7 +46,9 @@ def assert_rows_close(got, ref, tol, what="", elem_tol=None):
     per-element bound at elem_tol (default tol); returns (pooled, worst row)
     for printing."""
     got64 = _as64(got)
-    assert np.all(np.isfinite(got64)), f"{what}: non-finite outputs"
+    fin = np.isfinite(got64)
+    assert np.all(fin), (f"{what}: {int((~fin).sum())} of {fin.size} outputs non-finite "
+                         f"(in {int((~fin).reshape(-1, fin.shape[-1]).any(axis=1).sum())} rows)")
     pooled, rows, elem = row_errors(got64, ref)
     worst = int(np.argmax(rows))
     assert pooled <= tol, f"{what}: pooled rel L2 {pooled:.3e} > {tol}"

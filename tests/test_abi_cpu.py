@@ -31,7 +31,7 @@ def test_header_declares_the_entry_points():
     names = _declared_functions()
     for n in ["lla_write_latents", "lla_decode_attn", "hla_decode_attn", "lla_status_str",
               "lla_write_workspace_bytes", "lla_decode_workspace_bytes",
-              "hla_decode_workspace_bytes", "lla_abi_version"]:
+              "hla_decode_workspace_bytes", "lla_abi_version", "lla_last_cuda_error", "lla_cuda_error_name"]:
         assert n in names
 
 
@@ -48,6 +48,8 @@ def test_status_strings(lib):
         assert L.lla_status_str(s) != "unknown status"
     assert L.lla_status_str(99) == "unknown status"
     assert L.lla_abi_version() >= 1
+    assert L.lib().lla_last_cuda_error() == 0
+    assert L.lib().lla_cuda_error_name(0).decode() == "cudaSuccess"
 
 
 def test_struct_sizes_match_c_layout(lib):

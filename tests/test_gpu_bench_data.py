@@ -36,6 +36,7 @@ def f64(t):
 
 def _run_eager(step, dev):
     s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))   # the prefill ran on the current stream
     with torch.cuda.stream(s):
         step.run()
     torch.cuda.synchronize()

@@ -126,6 +126,8 @@ FP8_READS = [
     (2, 650, 128, 16, 1, 128, 256, 256, 129, True),    # Ouro-shaped loop-1 latent, 16 rows
     (1, 1100, 0, 16, 4, 128, 576, 576, 1, False),      # LLA-2D-shaped, 64 rows, no window
     (3, 301, 16, 4, 3, 64, 128, 192, 17, True),        # ragged tail, odd value chunk count
+    (2, 300, 0, 4, 2, 64, 64, 64, 1, False),           # one score chain and one value chain, 8 rows
+    (1, 520, 0, 16, 4, 128, 768, 768, 1, False),       # widest rows: one slot per ring, 64 rows
 ]
 
 
