@@ -31,7 +31,12 @@
  * Streams.    Every call only enqueues kernels on `stream` (a cudaStream_t;
  *             NULL = legacy default stream) and returns; it never synchronises.
  *             Inputs must stay valid until that work has run.  Two calls may
- *             share a workspace only if they are ordered on the GPU.
+ *             share a workspace only if they are ordered on the GPU.  With
+ *             LLA_PDL=1 in the environment (read once per process) kernels
+ *             are launched with programmatic dependent launch: a kernel's
+ *             set-up may overlap the end of the previous kernel on the
+ *             stream, and it touches global memory only once that kernel
+ *             has completed, so stream order is kept.
  * Threads.    Calls from several host threads are safe, each with its own
  *             workspace.  The exception is hla_decode_attn_noalloc: all of its
  *             calls share one scratch array, so calls whose work may overlap

@@ -2,11 +2,23 @@
 // orchestration.  Nothing is launched unless every check passes.
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 
 #include "kernels.cuh"
 
 namespace lla {
+
+// Launch attribute switch for launch_kernel (LLA_PDL=1 turns programmatic
+// dependent launch on); read once per process.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("LLA_PDL");
+    return v && v[0] == '1';
+  }();
+  return on;
+}
+
 namespace {
 
 constexpr int kAbiVersion = 3;   // 2: LLA_FP8_E4M3 latent rows; 3: hla_decode_params.nq

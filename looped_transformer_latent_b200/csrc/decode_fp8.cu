@@ -19,11 +19,13 @@
 // are multiplied by 2^8 when written.
 //
 // Per 64-token tile, four rings carry the chunks (64 tokens x 64 codes): key
-// chunks of the first and second half of r_K (rings 0 and 1) and value chunks
-// of the first and second half of the 128-wide value groups (rings 2 and 3).
-// A ring slot holds two f16 chunk blocks (16 KB, 128-byte swizzle); the codes
-// land by TMA in its upper half and one converter warp per ring rewrites them
-// in place into the f16 blocks.  Each ring has its own MMA issuer warp, so the
+// chunks of the first and second half of r_K (rings 0 and 1, one chunk per
+// slot, up to four slots) and the 128-wide value groups of the first and
+// second half of r_V (rings 2 and 3, two chunks per slot).  The codes land by
+// TMA in the upper half of a slot and one converter warp per ring rewrites
+// them in place into f16 chunk blocks (128-byte swizzle).  A producer thread
+// polls its two rings and issues whichever copy has a free slot.  Each ring
+// has its own MMA issuer warp, so the
 // four tcgen05 chains run concurrently (one thread's chain is bound by its own
 // issue latency):
 //   * two score chains S_a, S_b = Q~ codes^T over the two halves of r_K
@@ -50,7 +52,8 @@ using namespace ptx;
 constexpr int TOK = 64;
 constexpr int BLK = 8192;             // f16 chunk block: 64 tokens x 64 elements, 128-byte rows, swizzled
 constexpr int BLK8 = 4096;            // fp8 chunk block as landed: 64 tokens x 64 codes
-constexpr int SLOT = 2 * BLK;         // ring slot: two f16 chunk blocks; codes land in the upper half
+constexpr int SLOTK = BLK;            // key ring slot: one f16 chunk block; its codes land in the upper half
+constexpr int SLOTV = 2 * BLK;        // value ring slot: two f16 chunk blocks (one 128-wide value group)
 constexpr int NRING = 4;              // key halves a/b, value halves a/b
 constexpr int NSB = 4;                // scale slots (one per tile)
 constexpr int SBYTES = TOK * 16;      // one tile's scales: 64 x (s^K, s^V, 8 pad bytes)
@@ -106,14 +109,25 @@ __device__ __forceinline__ uint2 code4_to_f16(uint32_t w) {
   return make_uint2(lo, hi);
 }
 
+// Key rings (0, 1) have nsk one-chunk slots, value rings (2, 3) nsv
+// two-chunk slots; a key copy is one chunk, a value copy one value group.
 struct Layout8 {
-  int nkb, nvb, ns;
+  int nkb, nvb, nsk, nsv;
   __host__ __device__ int q_off() const { return 0; }
   __host__ __device__ int p_off() const { return nkb * BLK; }
   __host__ __device__ int sc_off() const { return p_off() + NBP * BLK; }
-  __host__ __device__ int ring_off(int r) const { return sc_off() + NSB * SBYTES + r * ns * SLOT; }
+  __host__ __device__ int ring_off(int r) const {
+    const int k0 = sc_off() + NSB * SBYTES;
+    return r < 2 ? k0 + r * nsk * SLOTK : k0 + 2 * nsk * SLOTK + (r - 2) * nsv * SLOTV;
+  }
+  __host__ __device__ int nslots(int r) const { return r < 2 ? nsk : nsv; }
+  __host__ __device__ int slot_bytes(int r) const { return r < 2 ? SLOTK : SLOTV; }
+  __host__ __device__ int land_off(int r) const { return r < 2 ? BLK8 : BLK; }   // where the codes land in a slot
+  __host__ __device__ int step(int r) const { return r < 2 ? 1 : 2; }            // chunks per copy
+  __host__ __device__ int bar0(int r) const { return r < 2 ? r * nsk : 2 * nsk + (r - 2) * nsv; }
+  __host__ __device__ int ring_bars() const { return 2 * nsk + 2 * nsv; }
   __host__ __device__ int bar_off() const { return ring_off(NRING); }
-  __host__ __device__ int nbars() const { return 3 * NRING * ns + 2 * NSB + 1 + 3 + 2 * NBP + 4; }
+  __host__ __device__ int nbars() const { return 3 * ring_bars() + 2 * NSB + 1 + 3 + 2 * NBP + 4; }
   __host__ __device__ int misc_off() const { return bar_off() + 8 * nbars(); }
   __host__ __device__ int bytes() const { return misc_off() + MISC_BYTES; }
 };
@@ -129,11 +143,11 @@ struct Rings {
 // 14 warps: four share an SM sub-partition's 16 K registers, so at most 128 per thread
 __global__ void __launch_bounds__(NTHREADS, 1)
 absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant__ CUtensorMap map1,
-                 const __grid_constant__ CUtensorMap mapsc, const AbsorbArgs a, const int ns) {
+                 const __grid_constant__ CUtensorMap mapsc, const AbsorbArgs a, const int nsk, const int nsv) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Layout8 L;
-  L.nkb = a.r_k / 64; L.nvb = a.r_v / 64; L.ns = ns;
+  L.nkb = a.r_k / 64; L.nvb = a.r_v / 64; L.nsk = nsk; L.nsv = nsv;
   Rings R;
   R.nkb = L.nkb; R.nvb = L.nvb;
   R.ka = (L.nkb + 1) / 2;
@@ -146,9 +160,9 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
   uint8_t* sc_s = base + L.sc_off();
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L.bar_off());
   uint64_t* lfull = bars;                       // [ring][slot] codes landed (TMA)
-  uint64_t* cfull = lfull + NRING * ns;         // [ring][slot] f16 blocks written (converter)
-  uint64_t* rempty = cfull + NRING * ns;        // [ring][slot] MMAs reading the slot done
-  uint64_t* sc_full = rempty + NRING * ns;      // [NSB] a tile's scales landed
+  uint64_t* cfull = lfull + L.ring_bars();      // [ring][slot] f16 blocks written (converter)
+  uint64_t* rempty = cfull + L.ring_bars();     // [ring][slot] MMAs reading the slot done
+  uint64_t* sc_full = rempty + L.ring_bars();   // [NSB] a tile's scales landed
   uint64_t* sc_free = sc_full + NSB;            // [NSB] softmax done with them (128 arrivals)
   uint64_t* q_full = sc_free + NSB;
   uint64_t* s_full = q_full + 1;                // [2] score chains a, b
@@ -171,7 +185,7 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
   const int rows = a.rows, rows_pad = a.rows_pad;
 
   if (tid == 0) {
-    for (int i = 0; i < NRING * ns; ++i) {
+    for (int i = 0; i < L.ring_bars(); ++i) {
       mbar_init(smem_u32(&lfull[i]), 1);
       mbar_init(smem_u32(&cfull[i]), 1);
       mbar_init(smem_u32(&rempty[i]), 1);
@@ -205,6 +219,7 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();
 
   if (warp == 4 || warp == 5) {
     // ----------------------------------------------------------- producers --
@@ -240,16 +255,16 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
         }
         for (int k = 0; k < 2; ++k) {
           if (done[k]) continue;
-          const int r = r0 + k;
+          const int r = r0 + k, ns = L.nslots(r);
           const uint32_t slot = cnt[k] % ns, ph = cnt[k] / ns;
-          if (!mbar_test_wait(smem_u32(&rempty[r * ns + slot]), (ph & 1) ^ 1)) continue;
-          const int c = chunk[k], w = R.hi(r) - c >= 2 ? 2 : 1;
-          const uint32_t fb = smem_u32(&lfull[r * ns + slot]);
+          if (!mbar_test_wait(smem_u32(&rempty[L.bar0(r) + slot]), (ph & 1) ^ 1)) continue;
+          const int c = chunk[k], w = min(L.step(r), R.hi(r) - c);
+          const uint32_t fb = smem_u32(&lfull[L.bar0(r) + slot]);
           mbar_arrive_tx(fb, w * BLK8);
-          tma_load_4d(smem_u32(base + L.ring_off(r) + slot * SLOT + BLK),
+          tma_load_4d(smem_u32(base + L.ring_off(r) + slot * L.slot_bytes(r) + L.land_off(r)),
                       w == 2 ? (const void*)&map2 : (const void*)&map1, fb, 0, tok0 + tile[k] * TOK, c0 + c, b);
           ++cnt[k];
-          chunk[k] = c + 2;
+          chunk[k] = c + w;
           if (chunk[k] >= R.hi(r)) {
             chunk[k] = R.lo(r);
             if (++tile[k] == ntiles) done[k] = true;
@@ -276,9 +291,11 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
           for (int n = max(0, nsc - NSB); n < nsc; ++n)
             wait8(smem_u32(&sc_full[n % NSB]), (n / NSB) & 1, abort_flag, nullptr, 0, false);
         }
-        for (int k = 0; k < 2; ++k)
-          for (uint32_t i = (cnt[k] > (uint32_t)ns ? cnt[k] - ns : 0); i < cnt[k]; ++i)
-            wait8(smem_u32(&lfull[(r0 + k) * ns + i % ns]), (i / ns) & 1, abort_flag, nullptr, 0, false);
+        for (int k = 0; k < 2; ++k) {
+          const uint32_t ns = L.nslots(r0 + k);
+          for (uint32_t i = (cnt[k] > ns ? cnt[k] - ns : 0); i < cnt[k]; ++i)
+            wait8(smem_u32(&lfull[L.bar0(r0 + k) + i % ns]), (i / ns) & 1, abort_flag, nullptr, 0, false);
+        }
       }
     }
   } else if (warp >= 10) {
@@ -288,18 +305,18 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
     // warp reads the 4 KB block contiguously), the warp synchronises (the
     // second chunk's f16 block overlaps its own codes), then each lane stores
     // 8 x 32 bytes into the swizzled rows.
-    const int r = warp - 10;
+    const int r = warp - 10, ns = L.nslots(r), stp = L.step(r);
     uint8_t* ring = base + L.ring_off(r);
     uint32_t cnt = 0;
     bool ok = true;
     for (int n = 0; n < ntiles && ok; ++n) {
-      for (int c = R.lo(r); c < R.hi(r); c += 2, ++cnt) {
-        const int w = R.hi(r) - c >= 2 ? 2 : 1;
+      for (int c = R.lo(r); c < R.hi(r); c += stp, ++cnt) {
+        const int w = min(stp, R.hi(r) - c);
         const uint32_t slot = cnt % ns, ph = cnt / ns;
-        if (!wait8(smem_u32(&lfull[r * ns + slot]), ph & 1, abort_flag, a.err, ERR8_LFULL)) { ok = false; break; }
-        uint8_t* sl = ring + slot * SLOT;
+        if (!wait8(smem_u32(&lfull[L.bar0(r) + slot]), ph & 1, abort_flag, a.err, ERR8_LFULL)) { ok = false; break; }
+        uint8_t* sl = ring + slot * L.slot_bytes(r);
         for (int j = 0; j < w; ++j) {
-          const uint4* src = reinterpret_cast<const uint4*>(sl + BLK + j * BLK8);
+          const uint4* src = reinterpret_cast<const uint4*>(sl + L.land_off(r) + j * BLK8);
           uint4 cw[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) cw[k] = src[lane + 32 * k];
@@ -319,7 +336,7 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&cfull[r * ns + slot]));
+        if (lane == 0) mbar_arrive(smem_u32(&cfull[L.bar0(r) + slot]));
       }
     }
   } else if (warp >= 6) {
@@ -344,21 +361,18 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
           if (n >= 1 && !wait8(smem_u32(s_free), (n - 1) & 1, abort_flag, a.err, ERR8_S)) { ok = false; break; }
           tc_fence_after();
           uint32_t acc = 0;
-          for (int c = R.lo(r); c < R.hi(r) && ok; c += 2, ++cnt) {
-            const int w = R.hi(r) - c >= 2 ? 2 : 1;
-            const uint32_t slot = cnt % ns, ph = cnt / ns;
-            if (!wait8(smem_u32(&cfull[r * ns + slot]), ph & 1, abort_flag, a.err, ERR8_CFULL)) { ok = false; break; }
+          for (int c = R.lo(r); c < R.hi(r) && ok; ++c, ++cnt) {
+            const uint32_t slot = cnt % nsk, ph = cnt / nsk;
+            if (!wait8(smem_u32(&cfull[L.bar0(r) + slot]), ph & 1, abort_flag, a.err, ERR8_CFULL)) { ok = false; break; }
             tc_fence_after();
-            for (int j = 0; j < w; ++j) {
-              const uint64_t ad = q_desc + (uint64_t)(((c + j) * BLK) >> 4);
-              const uint64_t bd = k_desc + (uint64_t)((slot * SLOT + j * BLK) >> 4);
+            const uint64_t ad = q_desc + (uint64_t)((c * BLK) >> 4);
+            const uint64_t bd = k_desc + (uint64_t)((slot * SLOTK) >> 4);
 #pragma unroll
-              for (int k16 = 0; k16 < 4; ++k16) {
-                mma_bf16(d, ad + 2 * k16, bd + 2 * k16, idS, acc);
-                acc = 1;
-              }
+            for (int k16 = 0; k16 < 4; ++k16) {
+              mma_bf16(d, ad + 2 * k16, bd + 2 * k16, idS, acc);
+              acc = 1;
             }
-            mma_commit(smem_u32(&rempty[r * ns + slot]));
+            mma_commit(smem_u32(&rempty[L.bar0(r) + slot]));
           }
           if (!ok) break;
           mma_commit(smem_u32(&s_full[r]));
@@ -370,17 +384,17 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
           tc_fence_after();
           const uint64_t bd = p_desc + (uint64_t)((buf * BLK) >> 4);
           for (int c = R.lo(r); c < R.hi(r) && ok; c += 2, ++cnt) {
-            const uint32_t slot = cnt % ns, ph = cnt / ns;
-            if (!wait8(smem_u32(&cfull[r * ns + slot]), ph & 1, abort_flag, a.err, ERR8_CFULL)) { ok = false; break; }
+            const uint32_t slot = cnt % nsv, ph = cnt / nsv;
+            if (!wait8(smem_u32(&cfull[L.bar0(r) + slot]), ph & 1, abort_flag, a.err, ERR8_CFULL)) { ok = false; break; }
             tc_fence_after();
             // one M=128 MMA covers both chunks of the slot (BLK apart); for a
             // one-chunk group rows 64..127 are value indices >= r_v, never read
             const uint32_t dO = tmem + O_COL + (c >> 1) * rows_pad;
-            const uint64_t ad = v_desc + (uint64_t)((slot * SLOT) >> 4);
+            const uint64_t ad = v_desc + (uint64_t)((slot * SLOTV) >> 4);
 #pragma unroll
             for (int k16 = 0; k16 < 4; ++k16)
               mma_bf16(dO, ad + 128 * k16, bd + 2 * k16, idO, (m > 0 || k16 > 0) ? 1u : 0u);
-            mma_commit(smem_u32(&rempty[r * ns + slot]));
+            mma_commit(smem_u32(&rempty[L.bar0(r) + slot]));
           }
           if (!ok) break;
           mma_commit(smem_u32(&o_done[buf]));
@@ -533,22 +547,29 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+  griddep_launch();
 }
 
-int fp8_smem(int r_k, int r_v, int ns) {
+int fp8_smem(int r_k, int r_v, int nsk, int nsv) {
   Layout8 L;
-  L.nkb = r_k / 64; L.nvb = r_v / 64; L.ns = ns;
+  L.nkb = r_k / 64; L.nvb = r_v / 64; L.nsk = nsk; L.nsv = nsv;
   return L.bytes() + 1024;
 }
 
-// two slots per ring where shared memory allows, else one
-int fp8_slots(int r_k, int r_v) { return fp8_smem(r_k, r_v, 2) <= SMEM_LIMIT ? 2 : 1; }
+// the deepest rings shared memory allows: key rings of 4..2 chunks with two
+// value groups per value ring, else 2 and 1
+void fp8_slots(int r_k, int r_v, int* nsk, int* nsv) {
+  static const int opts[4][2] = {{4, 2}, {3, 2}, {2, 2}, {2, 1}};
+  for (const auto& o : opts)
+    if (fp8_smem(r_k, r_v, o[0], o[1]) <= SMEM_LIMIT) { *nsk = o[0]; *nsv = o[1]; return; }
+  *nsk = 2; *nsv = 1;
+}
 
 }  // namespace
 
 bool absorb_fp8_supported(int r_k, int r_v, int rows) {
   if (r_k % 64 || r_v % 64 || r_k < 64 || r_v < 64 || r_k > 768) return false;
-  if (rows < 1 || rows > 64 || fp8_smem(r_k, r_v, 1) > SMEM_LIMIT) return false;
+  if (rows < 1 || rows > 64 || fp8_smem(r_k, r_v, 2, 1) > SMEM_LIMIT) return false;
   const int ngrp = (r_v / 64 + 1) / 2;
   return O_COL + (uint32_t)(ngrp * absorb_tc_rows_pad(rows)) <= TMEM_COLS;
 }
@@ -581,13 +602,13 @@ cudaError_t launch_absorb_split_fp8(const AbsorbArgs& a, cudaStream_t st) {
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const int ns = fp8_slots(a.r_k, a.r_v);
-  const int smem = fp8_smem(a.r_k, a.r_v, ns);
+  int nsk = 2, nsv = 1;
+  fp8_slots(a.r_k, a.r_v, &nsk, &nsv);
+  const int smem = fp8_smem(a.r_k, a.r_v, nsk, nsv);
   cudaError_t e = cudaFuncSetAttribute(absorb_split_fp8, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.S, a.B);
-  absorb_split_fp8<<<grid, NTHREADS, smem, st>>>(map2, map1, mapsc, a, ns);
-  return cudaGetLastError();
+  return launch_kernel(absorb_split_fp8, grid, dim3(NTHREADS), smem, st, 1, map2, map1, mapsc, a, nsk, nsv);
 }
 
 }  // namespace lla

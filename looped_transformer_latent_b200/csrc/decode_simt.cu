@@ -21,6 +21,7 @@ namespace {
 constexpr int RB = 16, TT = 16, VC = 4;  // r_v <= 1024
 
 __global__ void __launch_bounds__(256) absorb_split_simt(AbsorbArgs a) {
+  griddep_wait();
   extern __shared__ float sm[];
   const int s = blockIdx.x, b = blockIdx.y, row0 = blockIdx.z * RB;
   const int nr = min(RB, a.rows - row0);
@@ -112,6 +113,7 @@ __global__ void __launch_bounds__(256) absorb_split_simt(AbsorbArgs a) {
       a.part_y[(((int64_t)s * a.B + b) * a.rows + row0 + r) * a.r_v + v] = acc[r][c];
     }
   }
+  griddep_launch();
 }
 
 // --------------------------------------------------------------- window --
@@ -154,6 +156,7 @@ struct WinTraits<false> {  // 4 fp32 per lane
 // few tokens (fewer registers, so more CTAs per SM).
 template <bool BF16, int WU, int MINB>
 __global__ void __launch_bounds__(256, MINB) window_part(WindowArgs w) {
+  griddep_wait();
   typedef WinTraits<BF16> Tr;
   const int chunk = blockIdx.x, tt = blockIdx.y, b = blockIdx.z;
   const int t = w.t0 + tt;
@@ -241,6 +244,7 @@ __global__ void __launch_bounds__(256, MINB) window_part(WindowArgs w) {
       for (int e = 0; e < 4; ++e) w.win_y[o * w.d_h + d0 + e] = acc[e];
     }
   }
+  griddep_launch();
 }
 
 // Large windows: the same partial states, with the ring rows staged in shared
@@ -266,6 +270,7 @@ struct RingMaps {
 
 template <bool BF16>
 __global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(const __grid_constant__ RingMaps maps, WindowArgs w) {
+  griddep_wait();
   typedef WinTraits<BF16> Tr;
   constexpr int TS = WbTraits<BF16>::TS;
   constexpr int ES = BF16 ? 2 : 4;
@@ -419,6 +424,7 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_bulk(const __grid_consta
       for (int e = 0; e < 4; ++e) w.win_y[o * w.d_h + d0 + e] = acc[e];
     }
   }
+  griddep_launch();
 }
 
 // Windows of 16 tokens and more, in chunks of at most WC_TOK tokens: one CTA
@@ -457,6 +463,7 @@ __device__ __forceinline__ float butterfly_transpose_sum(float (&v)[N], int lane
 
 template <bool BF16>
 __global__ void __launch_bounds__(32 * WB_HEADS) window_chunk(const __grid_constant__ RingMaps maps, WindowArgs w) {
+  griddep_wait();
   typedef WinTraits<BF16> Tr;
   constexpr int TC = WcTraits<BF16>::TOK;
   constexpr int G = 32 / TC;   // lanes holding one token's score
@@ -574,6 +581,7 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_chunk(const __grid_const
 #pragma unroll
     for (int e = 0; e < 4; ++e) w.win_y[o * w.d_h + d0 + e] = acc[e];
   }
+  griddep_launch();
 }
 
 // ---------------------------------------------------------------- merge --
@@ -582,6 +590,7 @@ __global__ void __launch_bounds__(32 * WB_HEADS) window_chunk(const __grid_const
 //   M = max_s m_s, w_s = 2^(m_s - M), l = sum_s w_s l_s + w_w l_w,
 //   o = (sum_s w_s y_s + w_w y_w) / l
 __global__ void __launch_bounds__(128) merge_plain(MergeArgs g) {
+  griddep_wait();
   const int row = blockIdx.x, b = blockIdx.y;
   const int64_t br = (int64_t)b * g.rows + row;
   const int64_t bstride = (int64_t)g.B * g.rows;   // between partials of consecutive splits / chunks
@@ -610,6 +619,7 @@ __global__ void __launch_bounds__(128) merge_plain(MergeArgs g) {
     }
     g.out[(int64_t)b * g.outs_b + (int64_t)row * g.d_h + d] = (g.err && *g.err) ? NAN : y * li;
   }
+  griddep_launch();
 }
 
 // ------------------------------------------- LLA reconstruct, SIMT --
@@ -621,6 +631,7 @@ constexpr int RT = 32;   // tokens per tile
 constexpr int RKD = 16;  // d_h <= 128 -> 16 values per thread
 
 __global__ void __launch_bounds__(256) recon_split_simt(ReconArgs a) {
+  griddep_wait();
   extern __shared__ float sm[];
   const int s = blockIdx.x, row = blockIdx.y, b = blockIdx.z;
   const int tt = row / a.H, h = row % a.H;
@@ -727,6 +738,7 @@ __global__ void __launch_bounds__(256) recon_split_simt(ReconArgs a) {
     for (int u = 0; u < 8; ++u) y += accs[u * dh + d];
     a.part_y[o * dh + d] = y;
   }
+  griddep_launch();
 }
 
 }  // namespace
@@ -742,8 +754,7 @@ cudaError_t launch_absorb_split_simt(const AbsorbArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(absorb_split_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.S, a.B, ceil_div(a.rows, RB));
-  absorb_split_simt<<<grid, 256, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(absorb_split_simt, grid, dim3(256), smem, st, 1, a);
 }
 
 bool window_bulk_ok(int dtype, int d_h) {
@@ -816,40 +827,37 @@ cudaError_t launch_window(const WindowArgs& w_in, cudaStream_t st) {
       if (w.dtype == LLA_BF16) {
         e = cudaFuncSetAttribute(window_chunk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        window_chunk<true><<<grid, 32 * WB_HEADS, smem, st>>>(maps, w);
+        e = launch_kernel(window_chunk<true>, grid, dim3(32 * WB_HEADS), smem, st, 1, maps, w);
       } else {
         e = cudaFuncSetAttribute(window_chunk<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        window_chunk<false><<<grid, 32 * WB_HEADS, smem, st>>>(maps, w);
+        e = launch_kernel(window_chunk<false>, grid, dim3(32 * WB_HEADS), smem, st, 1, maps, w);
       }
     } else if (w.dtype == LLA_BF16) {
       e = cudaFuncSetAttribute(window_bulk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      window_bulk<true><<<grid, 32 * WB_HEADS, smem, st>>>(maps, w);
+      e = launch_kernel(window_bulk<true>, grid, dim3(32 * WB_HEADS), smem, st, 1, maps, w);
     } else {
       e = cudaFuncSetAttribute(window_bulk<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      window_bulk<false><<<grid, 32 * WB_HEADS, smem, st>>>(maps, w);
+      e = launch_kernel(window_bulk<false>, grid, dim3(32 * WB_HEADS), smem, st, 1, maps, w);
     }
-    return cudaGetLastError();
+    return e;
   }
 register_kernel:
   dim3 grid(w.Sw, nt, w.B);
   const bool small = w.cpt <= 8;
   if (w.dtype == LLA_BF16) {
-    if (small) window_part<true, 4, 4><<<grid, 256, 0, st>>>(w);
-    else window_part<true, WinTraits<true>::WU, 1><<<grid, 256, 0, st>>>(w);
-  } else {
-    if (small) window_part<false, 4, 4><<<grid, 256, 0, st>>>(w);
-    else window_part<false, WinTraits<false>::WU, 1><<<grid, 256, 0, st>>>(w);
+    if (small) return launch_kernel(window_part<true, 4, 4>, grid, dim3(256), 0, st, 1, w);
+    return launch_kernel(window_part<true, WinTraits<true>::WU, 1>, grid, dim3(256), 0, st, 1, w);
   }
-  return cudaGetLastError();
+  if (small) return launch_kernel(window_part<false, 4, 4>, grid, dim3(256), 0, st, 1, w);
+  return launch_kernel(window_part<false, WinTraits<false>::WU, 1>, grid, dim3(256), 0, st, 1, w);
 }
 
 cudaError_t launch_merge(const MergeArgs& g, cudaStream_t st) {
   dim3 grid(g.rows, g.B);
-  merge_plain<<<grid, 128, 0, st>>>(g);
-  return cudaGetLastError();
+  return launch_kernel(merge_plain, grid, dim3(128), 0, st, 1, g);
 }
 
 cudaError_t launch_recon_split_simt(const ReconArgs& a, cudaStream_t st) {
@@ -858,8 +866,7 @@ cudaError_t launch_recon_split_simt(const ReconArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(recon_split_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.S, a.rows, a.B);
-  recon_split_simt<<<grid, 256, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(recon_split_simt, grid, dim3(256), smem, st, 1, a);
 }
 
 }  // namespace lla

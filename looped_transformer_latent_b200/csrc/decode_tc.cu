@@ -145,6 +145,7 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();
 
   // The ring is two rings: slots [0, RK) carry key chunks, read only by the
   // score issuer, and slots [RK, R) value chunks, read only by the value
@@ -402,6 +403,7 @@ absorb_split_tc(const __grid_constant__ CUtensorMap tmap2, const __grid_constant
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+  griddep_launch();
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -485,8 +487,7 @@ cudaError_t launch_absorb_split_tc(const AbsorbArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(absorb_split_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.S, a.B);
-  absorb_split_tc<<<grid, NTHREADS, smem, st>>>(tmap2, tmap1, a, Rslots);
-  return cudaGetLastError();
+  return launch_kernel(absorb_split_tc, grid, dim3(NTHREADS), smem, st, 1, tmap2, tmap1, a, Rslots);
 }
 
 }  // namespace lla

@@ -195,6 +195,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
     t.kc1 = KIND == KIND_OMAP ? (int)((int64_t)nk * (ks + 1) / a.ks) : nk;
     if (KIND == KIND_QMAP && t.g >= a.rows) {
       // rows of the bf16 query operand past the last query row are zero
+      griddep_wait();
       for (int idx = tid; idx < GM * BN; idx += NTHR) {
         const int m = t.m0 + (idx % GM), n = t.n0 + idx / GM;
         if (m < t.Mv && n < t.Nv) a.qbf[qbf_index(n, t.g, m, a.Mtot)] = __float2bfloat16_rn(0.f);
@@ -278,6 +279,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
     fence_mbar_init();
     prefetch_tmap(&maps.a[0]);
     prefetch_tmap(&maps.x[0]);
+    griddep_wait();
     for (int i = 0; i < first; ++i) issue_chunk(i);
   }
   uint32_t ncols = 32;
@@ -290,6 +292,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();
   // output map with a cluster k-split: this CTA's weighted partial tile, in
   // the stage memory (free once every MMA is done)
   float* part_s = reinterpret_cast<float*>(base);                          // [BN][GM]
@@ -598,6 +601,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
     tc_fence_after();
     tmem_dealloc(tmem, ncols);
   }
+  griddep_launch();
 }
 
 template <int KIND, int BN, int PREC>
@@ -631,24 +635,7 @@ cudaError_t launch_one(const TcMaps& maps, TcGemmArgs a, int grid_y, int nb, siz
   if (e != cudaSuccess) return e;
   const int ksplit = KIND == KIND_OMAP ? a.ks : 1;
   dim3 grid(a.mtiles * a.ntiles * ksplit, grid_y);
-  if (ksplit > 1) {
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(NTHR);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = ksplit;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, tc_gemm<KIND, BN, PREC>, maps, a);
-  }
-  tc_gemm<KIND, BN, PREC><<<grid, NTHR, smem, st>>>(maps, a);
-  return cudaGetLastError();
+  return launch_kernel(tc_gemm<KIND, BN, PREC>, grid, dim3(NTHR), smem, st, ksplit, maps, a);
 }
 
 int pick_bn(int n) { return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : 256; }

@@ -29,6 +29,7 @@ __device__ __forceinline__ int64_t qbf_index(int b, int row, int k, int r_k) {
 
 template <int MODE, int GB, int GK>
 __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
+  griddep_wait();
   constexpr int BPW = GB / (GT / 32);   // sequences per warp
   constexpr int LX = GB * GK / GT;      // activation loads per thread
   __shared__ float Xs[2][GK][GB + 1];
@@ -184,6 +185,7 @@ __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
       dst[1] = bad ? NAN : y1 * li;
     }
   }
+  griddep_launch();
 }
 
 }  // namespace
@@ -193,19 +195,16 @@ int map_max_splits() { return MAXS; }
 cudaError_t launch_query_map(const MapArgs& g, cudaStream_t st) {
   const int ntile = (g.N + GN - 1) / GN;
   dim3 grid(g.use_tc ? 64 : g.rows, ntile, (g.B + 31) / 32);
-  row_gemm<0, 32, 32><<<grid, GT, 0, st>>>(g);
-  return cudaGetLastError();
+  return launch_kernel(row_gemm<0, 32, 32>, grid, dim3(GT), 0, st, 1, g);
 }
 
 cudaError_t launch_output_map(const MapArgs& g, cudaStream_t st) {
   if (g.B <= 64) {
     dim3 grid(g.rows, (g.N + GN - 1) / GN, (g.B + 15) / 16);
-    row_gemm<1, 16, 32><<<grid, GT, 0, st>>>(g);
-  } else {
-    dim3 grid(g.rows, (g.N + GN - 1) / GN, (g.B + 31) / 32);
-    row_gemm<1, 32, 32><<<grid, GT, 0, st>>>(g);
+    return launch_kernel(row_gemm<1, 16, 32>, grid, dim3(GT), 0, st, 1, g);
   }
-  return cudaGetLastError();
+  dim3 grid(g.rows, (g.N + GN - 1) / GN, (g.B + 31) / 32);
+  return launch_kernel(row_gemm<1, 32, 32>, grid, dim3(GT), 0, st, 1, g);
 }
 
 }  // namespace lla

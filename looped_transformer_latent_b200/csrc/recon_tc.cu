@@ -181,6 +181,7 @@ recon_group_tc(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();
 
   if (warp == 8) {
     // ---------------------------------------------------------- TMA copies --
@@ -490,6 +491,7 @@ recon_group_tc(const __grid_constant__ CUtensorMap mapK, const __grid_constant__
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+  griddep_launch();
 }
 
 struct ReconPlan { int G, SB, smem; };
@@ -568,8 +570,7 @@ cudaError_t launch_recon_tc(const ReconArgs& a, int* err, cudaStream_t st, int n
   // sequence chunks fastest: the CTAs that share a group's decoders run side
   // by side, then the loop groups of a head (which share its latent stream)
   dim3 grid((a.B + p.SB - 1) / p.SB, (a.nt + p.G - 1) / p.G, a.H);
-  kern<<<grid, RCT, p.smem, st>>>(mk, mv, a, p.G, p.SB, err);
-  return cudaGetLastError();
+  return launch_kernel(kern, grid, dim3(RCT), (size_t)p.smem, st, 1, mk, mv, a, p.G, p.SB, err);
 }
 
 }  // namespace lla

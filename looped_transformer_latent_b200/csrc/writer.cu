@@ -20,6 +20,7 @@ constexpr int BK = 32, WT = 256;
 // current one is multiplied; each thread owns a 4 x 4 block of outputs.
 template <int TM, int TN>
 __global__ void __launch_bounds__(WT) writer_gemm(WriterArgs a) {
+  griddep_wait();
   constexpr int LA = TM * BK / WT, LB = TN * BK / WT;   // loads per thread
   constexpr int TX = TN / 4;                              // threads along n
   const int z = blockIdx.z / a.S, split = blockIdx.z % a.S;
@@ -103,10 +104,12 @@ __global__ void __launch_bounds__(WT) writer_gemm(WriterArgs a) {
       if (nn < s.N) P[(int64_t)mm * a.Nmax + nn] = acc[i][jj];
     }
   }
+  griddep_launch();
 }
 
 // Phase 2: ordered sum of the splits, rotation of key pairs, rounding, store.
 __global__ void writer_epilogue(WriterArgs a) {
+  griddep_wait();
   const int64_t pairs = a.Nmax / 2;
   const int64_t total = (int64_t)a.Z * a.M * pairs;
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
@@ -136,6 +139,7 @@ __global__ void writer_epilogue(WriterArgs a) {
     store_elem(s.out, o, a.dtype, x);
     store_elem(s.out, o + 1, a.dtype, y);
   }
+  griddep_launch();
 }
 
 // Phase 2 for fp8 rows (e4m3 codes with per-token, per-part scales): one warp
@@ -158,6 +162,7 @@ __device__ __forceinline__ float fp8_part_value(const WriterArgs& a, int tgt, in
 }
 
 __global__ void __launch_bounds__(FP8_WARPS * 32) writer_epilogue_fp8(WriterArgs a) {
+  griddep_wait();
   __shared__ float rowbuf[FP8_WARPS][FP8_ROW_MAX];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntgt = a.mode == LLA_WRITE_HLA ? 2 : 1;
@@ -211,6 +216,7 @@ __global__ void __launch_bounds__(FP8_WARPS * 32) writer_epilogue_fp8(WriterArgs
     }
     __syncwarp();
   }
+  griddep_launch();
 }
 
 }  // namespace
@@ -251,26 +257,23 @@ cudaError_t launch_writer(const WriterArgs& a_in, cudaStream_t st) {
   if (simt) {
     if (small_batch(a)) {
       dim3 grid(ceil_div(a.Nmax, 128), ceil_div(a.M, 32), a.Z * a.S);
-      writer_gemm<32, 128><<<grid, WT, 0, st>>>(a);
+      e0 = launch_kernel(writer_gemm<32, 128>, grid, dim3(WT), 0, st, 1, a);
     } else {
       dim3 grid(ceil_div(a.Nmax, 64), ceil_div(a.M, 64), a.Z * a.S);
-      writer_gemm<64, 64><<<grid, WT, 0, st>>>(a);
+      e0 = launch_kernel(writer_gemm<64, 64>, grid, dim3(WT), 0, st, 1, a);
     }
-    e0 = cudaGetLastError();
   }
   if (e0 != cudaSuccess) return e0;
   if (a.dtype == LLA_FP8_E4M3) {
     const int64_t rows = (int64_t)(a.mode == LLA_WRITE_HLA ? 2 : 1) * a.M;
     int blocks = (int)((rows + FP8_WARPS - 1) / FP8_WARPS);
     if (blocks > 148 * 16) blocks = 148 * 16;
-    writer_epilogue_fp8<<<blocks, FP8_WARPS * 32, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_kernel(writer_epilogue_fp8, dim3(blocks), dim3(FP8_WARPS * 32), 0, st, 1, a);
   }
   const int64_t total = (int64_t)a.Z * a.M * (a.Nmax / 2);
   int blocks = (int)((total + 255) / 256);
   if (blocks > 148 * 16) blocks = 148 * 16;
-  writer_epilogue<<<blocks, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(writer_epilogue, dim3(blocks), dim3(256), 0, st, 1, a);
 }
 
 }  // namespace lla
