@@ -107,6 +107,7 @@ class Step:
     'main' marks the read calls whose latent-read kernel is the roofline's."""
 
     kind_launches = {"hla": 3, "lla": 2, "write": 2}
+    overlap_writes = True   # False: writers in stream order (a read needs their row, or saturates HBM)
 
     def __init__(self, cfg, dev, mode):
         import looped_transformer_latent_b200 as L
@@ -119,7 +120,7 @@ class Step:
 
     def _workspace(self):
         L = self.L
-        nb = 0
+        nb, nbw = 0, 0
         for kind, kw, _ in self.calls:
             if kind == "hla":
                 nb = max(nb, L.hla_decode_workspace_bytes(**kw))
@@ -127,8 +128,16 @@ class Step:
                 nb = max(nb, L.lla_decode_workspace_bytes(**kw))
             else:
                 mode = kw["mode"]
-                nb = max(nb, L.lla_write_workspace_bytes(mode, **{k: v for k, v in kw.items() if k != "mode"}))
-        self.ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=self.dev)
+                nbw = max(nbw, L.lla_write_workspace_bytes(mode, **{k: v for k, v in kw.items() if k != "mode"}))
+        self.ws = torch.empty(max(nb, nbw, 256), dtype=torch.uint8, device=self.dev)
+        # The writer stores the new token's latent row, which no read of this
+        # step uses (the next step's reads do): it runs on its own stream with
+        # its own workspace, forked at its layer's start and joined at the end
+        # of the step, so it overlaps the reads.
+        self.wstream = torch.cuda.Stream(self.dev)
+        self.ws_w = torch.empty(max(nbw, 256), dtype=torch.uint8, device=self.dev)
+        self.wfork = [torch.cuda.Event() for _ in range(self.cfg.L)]
+        self.wjoin = torch.cuda.Event()
         # the prefill ran on the constructing stream; the step may run on any
         # other, so setup ends with everything it issued complete
         torch.cuda.synchronize(self.dev)
@@ -145,11 +154,15 @@ class Step:
         if given, runs on the current stream before a layer's first call and
         after its last one."""
         L = self.L
+        main = torch.cuda.current_stream(self.dev)
         ei = 0
         per = len(self.calls) // self.cfg.L
         for idx, (kind, kw, _) in enumerate(self.calls):
-            if hook is not None and idx % per == 0:
-                hook(idx // per, "begin")
+            layer = idx // per
+            if idx % per == 0:
+                if hook is not None:
+                    hook(layer, "begin")
+                self.wfork[layer].record(main)
             if kind in ("hla", "lla"):
                 ev = None
                 if events is not None:
@@ -157,11 +170,25 @@ class Step:
                     ei += 1
                 fn = L.hla_decode_attn if kind == "hla" else L.lla_decode_attn
                 fn(workspace=self.ws, timing_events=ev, **kw)
+            elif self.overlap_writes:
+                self.write_async(layer, kw)
             else:
-                mode = kw["mode"]
-                L.lla_write_latents(mode, workspace=self.ws, **{k: v for k, v in kw.items() if k != "mode"})
+                L.lla_write_latents(kw["mode"], workspace=self.ws, **{k: v for k, v in kw.items() if k != "mode"})
             if hook is not None and idx % per == per - 1:
-                hook(idx // per, "end")
+                hook(layer, "end")
+        if self.overlap_writes:
+            self.join_writers(main)
+
+    def write_async(self, layer, kw):
+        """The layer's writer on the writer stream, after everything issued on
+        the step's stream before the layer began."""
+        self.wstream.wait_event(self.wfork[layer])
+        self.L.lla_write_latents(kw["mode"], workspace=self.ws_w, stream=self.wstream,
+                                 **{k: v for k, v in kw.items() if k != "mode"})
+
+    def join_writers(self, main):
+        self.wjoin.record(self.wstream)
+        main.wait_event(self.wjoin)
 
     def read_tags(self):
         return [tag for kind, _, tag in self.calls if kind in ("hla", "lla")]
@@ -308,12 +335,12 @@ class HlaStep(Step):
             if hook is not None:
                 hook(layer, "begin")
             self.fork[layer].record(main)
+            self.wfork[layer].record(main)
             self.side.wait_event(self.fork[layer])
             L.hla_decode_attn(workspace=self.ws_side, stream=self.side,
                               timing_events=events[ei] if events is not None else None, **kw1)
             # the writer only touches the new token's row, which neither read uses
-            L.lla_write_latents(kww["mode"], workspace=self.ws_side, stream=self.side,
-                                **{k: v for k, v in kww.items() if k != "mode"})
+            self.write_async(layer, kww)
             self.join[layer].record(self.side)
             L.hla_decode_attn(workspace=self.ws, stream=main,
                               timing_events=events[ei + 1] if events is not None else None, **kw2)
@@ -321,6 +348,7 @@ class HlaStep(Step):
             if hook is not None:
                 hook(layer, "end")
             ei += 2
+        self.join_writers(main)
 
 
 class Lla2dStep(Step):
@@ -354,6 +382,11 @@ class Lla2dStep(Step):
             L.lla_write_latents(L.LLA_WRITE_FOLDED, x=k, xv=v, E_K=codec["E_K"], E_V=codec["E_V"],
                                 out0=lat0[b0:b0 + nb], pos0=0)
             del k, v
+        # The bf16 read streams at close to full HBM bandwidth on every SM: a
+        # writer running beside it slows it by more than the writer's own time
+        # (measured 40.1 vs 38.7 ms per step), so the writers stay in stream
+        # order there.  The fp8 read leaves bandwidth to spare.
+        self.overlap_writes = c.lat_dtype == "fp8"
         lats = [lat0] + [lat0.clone() for _ in range(self.NBUF - 1)]
         self.ins, self.outs, self.layers = [], [], []
         for layer in range(c.L):
@@ -399,9 +432,11 @@ class LlaStep(Step):
     writer.  With W = 0 the writer stores the new token's latent (read from the
     next step on).  With W > 0 (served semantics: an exact ring of the last W
     tokens and the current one) the writer is the streaming store of the token
-    leaving the window, N - 2 - W, whose latent this step's read already needs
+    leaving the window, N - 2 - W, issued before the read, which needs it
     (prefill wrote it too; the writer's rows do not depend on how many tokens a
-    call writes, so the store reproduces them bit for bit)."""
+    call writes, so the store reproduces them bit for bit).  Elsewhere the
+    writer's row is read only from the next step on, so writers run on their
+    own stream, overlapping the reads."""
 
     def __init__(self, cfg, dev, mode, seed=777):
         super().__init__(cfg, dev, mode)
@@ -443,15 +478,20 @@ class LlaStep(Step):
         self.q = torch.randn(B, T, H, d_h, generator=g, device=dev)
         self.out = torch.empty(B, T, H, d_h, device=dev)
         self.ins, self.outs = [self.q, self.k, self.v], [self.out]
-        self.calls.append(("lla", dict(cK=cK, cV=cV, UK=codec["U_K"], UV=codec["U_V"], q=self.q, win_k=ring_k,
-                                       win_v=ring_v, out=self.out, N=N, W=W, t0=0), "main"))
+        read = ("lla", dict(cK=cK, cV=cV, UK=codec["U_K"], UV=codec["U_V"], q=self.q, win_k=ring_k,
+                            win_v=ring_v, out=self.out, N=N, W=W, t0=0), "main")
         if W > 0:
+            # served: the token leaving the window is stored first, then read
+            # (it is among this step's latent tokens), in stream order
             self.ins += [self.ek, self.ev]
-            wx, wv, wpos = self.ek, self.ev, evict
+            self.overlap_writes = False
+            self.calls.append(("write", dict(mode=L.LLA_WRITE_PERHEAD, x=self.ek, xv=self.ev, E_K=codec["E_K"],
+                                             E_V=codec["E_V"], out0=cK, out1=cV, pos0=evict), None))
+            self.calls.append(read)
         else:
-            wx, wv, wpos = self.k, self.v, self.i
-        self.calls.append(("write", dict(mode=L.LLA_WRITE_PERHEAD, x=wx, xv=wv, E_K=codec["E_K"],
-                                         E_V=codec["E_V"], out0=cK, out1=cV, pos0=wpos), None))
+            self.calls.append(read)
+            self.calls.append(("write", dict(mode=L.LLA_WRITE_PERHEAD, x=self.k, xv=self.v, E_K=codec["E_K"],
+                                             E_V=codec["E_V"], out0=cK, out1=cV, pos0=self.i), None))
         self._workspace()
 
 
