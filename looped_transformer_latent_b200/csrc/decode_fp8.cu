@@ -11,16 +11,16 @@
 // so the tensor cores contract the codes and the scales are applied per token
 // on the softmax side.
 //
-// Codes become f16 operands by bit placement on the integer pipe, not by the
-// conversion unit: an e4m3 byte s.eeee.mmm moved to the f16 bits
-// s.0eeee.mmm0000000 is the f16 number code * 2^-8 exactly (normal codes: the
-// exponent biases are 15 and 7; subnormal codes m * 2^-9 become the f16
-// subnormals m * 2^-17), so the scores take s^K * 2^8 and the value partials
-// are multiplied by 2^8 when written.
+// Codes become the f16 operands code * 2^-8, half of them by bit placement on
+// the integer pipe (an e4m3 byte s.eeee.mmm moved to the f16 bits
+// s.0eeee.mmm0000000 is exactly code * 2^-8: the exponent biases are 15 and
+// 7, and subnormal codes m * 2^-9 become the f16 subnormals m * 2^-17), half
+// by the conversion unit and a multiply by 2^-8; the scores take s^K * 2^8
+// and the value partials are multiplied by 2^8 when written.
 //
-// Per 64-token tile, four rings carry the chunks (64 tokens x 64 codes): key
-// chunks of the first and second half of r_K (rings 0 and 1, one chunk per
-// slot, up to four slots) and the 128-wide value groups of the first and
+// Four rings carry the chunks (64 tokens x 64 codes): the key chunks of the
+// even and of the odd 64-token tiles (rings 0 and 1, one chunk per slot, up
+// to four slots) and each tile's 128-wide value groups of the first and
 // second half of r_V (rings 2 and 3, two chunks per slot).  The codes land by
 // TMA in the upper half of a slot and one converter warp per ring rewrites
 // them in place into f16 chunk blocks (128-byte swizzle).  A producer thread
@@ -28,9 +28,10 @@
 // has its own MMA issuer warp, so the
 // four tcgen05 chains run concurrently (one thread's chain is bound by its own
 // issue latency):
-//   * two score chains S_a, S_b = Q~ codes^T over the two halves of r_K
-//     (M = 64 rows, N = 64 tokens, f16 in, fp32 in TMEM), summed by the
-//     softmax in a fixed order;
+//   * two score chains S = Q~ codes^T (M = 64 rows, N = 64 tokens, f16 in,
+//     fp32 in TMEM), one for the even and one for the odd tiles, each into
+//     its own TMEM buffer, so a chain works on its next tile while the
+//     softmax reads the other's;
 //   * two value chains O^T += codes^V^T P'^T over their value groups
 //     (M = 128 value indices, N = rows);
 //   * four softmax warps scale the scores by s^K, run the online softmax
@@ -39,6 +40,7 @@
 // then emits NaN), drains its copies and frees TMEM.
 #include <cuda.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "kernels.cuh"
 #include "tc_ptx.cuh"
@@ -111,6 +113,19 @@ __device__ __forceinline__ uint2 code4_to_f16(uint32_t w) {
 
 // Key rings (0, 1) have nsk one-chunk slots, value rings (2, 3) nsv
 // two-chunk slots; a key copy is one chunk, a value copy one value group.
+// The same four values through the conversion unit: the exact f16 of each
+// code (cvt.f16x2.e4m3x2), times 2^-8 (exact: a power of two, subnormal f16
+// results included).  The converters alternate words between this and the
+// integer form, so the two pipes share the work.
+__device__ __forceinline__ uint2 code4_to_f16_cvt(uint32_t w) {
+  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
+  const __half2 unit = __halves2half2(__ushort_as_half((unsigned short)0x1C00u), __ushort_as_half((unsigned short)0x1C00u));
+  const __half2 l = __hmul2(*reinterpret_cast<const __half2*>(&lo), unit);
+  const __half2 h = __hmul2(*reinterpret_cast<const __half2*>(&hi), unit);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(&l), *reinterpret_cast<const uint32_t*>(&h));
+}
+
 struct Layout8 {
   int nkb, nvb, nsk, nsv;
   __host__ __device__ int q_off() const { return 0; }
@@ -127,17 +142,21 @@ struct Layout8 {
   __host__ __device__ int bar0(int r) const { return r < 2 ? r * nsk : 2 * nsk + (r - 2) * nsv; }
   __host__ __device__ int ring_bars() const { return 2 * nsk + 2 * nsv; }
   __host__ __device__ int bar_off() const { return ring_off(NRING); }
-  __host__ __device__ int nbars() const { return 3 * ring_bars() + 2 * NSB + 1 + 3 + 2 * NBP + 4; }
+  __host__ __device__ int nbars() const { return 3 * ring_bars() + 2 * NSB + 1 + 4 + 2 * NBP + 4; }
   __host__ __device__ int misc_off() const { return bar_off() + 8 * nbars(); }
   __host__ __device__ int bytes() const { return misc_off() + MISC_BYTES; }
 };
 
-// Chunk range of ring r: key chunks [0, ka) and [ka, nkb); value chunks of the
-// groups [0, ga) and [ga, ngrp) (a group is two chunks, the last possibly one).
+// What ring r carries: the key rings every key chunk of the even (ring 0)
+// and the odd (ring 1) tiles; the value rings every tile's chunks of the
+// value groups [0, ga) and [ga, ngrp) (a group is two chunks, the last
+// possibly one).
 struct Rings {
-  int nkb, nvb, ka, ngrp, ga;
-  __device__ int lo(int r) const { return r == 0 ? 0 : r == 1 ? ka : r == 2 ? 0 : 2 * ga; }
-  __device__ int hi(int r) const { return r == 0 ? ka : r == 1 ? nkb : r == 2 ? min(nvb, 2 * ga) : nvb; }
+  int nkb, nvb, ngrp, ga;
+  __device__ int lo(int r) const { return r < 2 ? 0 : r == 2 ? 0 : 2 * ga; }
+  __device__ int hi(int r) const { return r < 2 ? nkb : r == 2 ? min(nvb, 2 * ga) : nvb; }
+  __device__ int tile0(int r) const { return r < 2 ? r : 0; }
+  __device__ int tstep(int r) const { return r < 2 ? 2 : 1; }
 };
 
 // 14 warps: four share an SM sub-partition's 16 K registers, so at most 128 per thread
@@ -150,10 +169,8 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
   L.nkb = a.r_k / 64; L.nvb = a.r_v / 64; L.nsk = nsk; L.nsv = nsv;
   Rings R;
   R.nkb = L.nkb; R.nvb = L.nvb;
-  R.ka = (L.nkb + 1) / 2;
   R.ngrp = (L.nvb + 1) / 2;
   R.ga = (R.ngrp + 1) / 2;
-  const bool two_s = R.ka < L.nkb;      // a second score chain (r_K >= 128)
   const bool two_v = R.ga < R.ngrp;     // a second value chain (r_V > 128)
   uint8_t* q_s = base + L.q_off();
   uint8_t* p_s = base + L.p_off();
@@ -165,9 +182,9 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
   uint64_t* sc_full = rempty + L.ring_bars();   // [NSB] a tile's scales landed
   uint64_t* sc_free = sc_full + NSB;            // [NSB] softmax done with them (128 arrivals)
   uint64_t* q_full = sc_free + NSB;
-  uint64_t* s_full = q_full + 1;                // [2] score chains a, b
-  uint64_t* s_free = s_full + 2;                // softmax has read S_a and S_b (128 arrivals)
-  uint64_t* p_full = s_free + 1;                // [NBP]
+  uint64_t* s_full = q_full + 1;                // [2] scores of the even / odd tiles in TMEM
+  uint64_t* s_free = s_full + 2;                // [2] softmax has read them (128 arrivals)
+  uint64_t* p_full = s_free + 2;                // [NBP]
   uint64_t* o_done = p_full + NBP;              // [NBP] the value chains are done with a tile
   uint64_t* fin = o_done + NBP;                 // [4] one per MMA issuer (abort path)
   uint8_t* misc = base + L.misc_off();
@@ -195,9 +212,10 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
       mbar_init(smem_u32(&sc_free[i]), 128);
     }
     mbar_init(smem_u32(q_full), 1);
-    mbar_init(smem_u32(&s_full[0]), 1);
-    mbar_init(smem_u32(&s_full[1]), 1);
-    mbar_init(smem_u32(s_free), 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&s_free[i]), 128);
+    }
     for (int i = 0; i < NBP; ++i) {
       mbar_init(smem_u32(&p_full[i]), 128);
       mbar_init(smem_u32(&o_done[i]), two_v ? 2 : 1);
@@ -237,8 +255,8 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
         bulk_load(smem_u32(q_s), a.qbf + (size_t)b * nkb * (BLK / 2), nkb * BLK, qb);
       }
       uint32_t cnt[2] = {0, 0};
-      int tile[2] = {0, 0}, chunk[2] = {R.lo(r0), R.lo(r0 + 1)};
-      bool done[2] = {R.lo(r0) >= R.hi(r0), R.lo(r0 + 1) >= R.hi(r0 + 1)};
+      int tile[2] = {R.tile0(r0), R.tile0(r0 + 1)}, chunk[2] = {R.lo(r0), R.lo(r0 + 1)};
+      bool done[2] = {R.lo(r0) >= R.hi(r0) || tile[0] >= ntiles, R.lo(r0 + 1) >= R.hi(r0 + 1) || tile[1] >= ntiles};
       int nsc = kside ? 0 : ntiles;
       bool ok = true;
       long long t_last = clock64();
@@ -267,7 +285,8 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
           chunk[k] = c + w;
           if (chunk[k] >= R.hi(r)) {
             chunk[k] = R.lo(r);
-            if (++tile[k] == ntiles) done[k] = true;
+            tile[k] += R.tstep(r);
+            if (tile[k] >= ntiles) done[k] = true;
           }
           progress = true;
         }
@@ -309,7 +328,7 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
     uint8_t* ring = base + L.ring_off(r);
     uint32_t cnt = 0;
     bool ok = true;
-    for (int n = 0; n < ntiles && ok; ++n) {
+    for (int n = R.tile0(r); n < ntiles && ok; n += R.tstep(r)) {
       for (int c = R.lo(r); c < R.hi(r); c += stp, ++cnt) {
         const int w = min(stp, R.hi(r) - c);
         const uint32_t slot = cnt % ns, ph = cnt / ns;
@@ -326,8 +345,8 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
           uint8_t* dst = sl + j * BLK + (lane >> 2) * 128;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const uint2 h0 = code4_to_f16(cw[k].x), h1 = code4_to_f16(cw[k].y);
-            const uint2 h2 = code4_to_f16(cw[k].z), h3 = code4_to_f16(cw[k].w);
+            const uint2 h0 = code4_to_f16(cw[k].x), h1 = code4_to_f16_cvt(cw[k].y);
+            const uint2 h2 = code4_to_f16(cw[k].z), h3 = code4_to_f16_cvt(cw[k].w);
             uint8_t* drow = dst + k * 8 * 128;
             *reinterpret_cast<uint4*>(drow + (((2 * p) ^ sw) << 4)) = make_uint4(h0.x, h0.y, h1.x, h1.y);
             *reinterpret_cast<uint4*>(drow + (((2 * p + 1) ^ sw) << 4)) = make_uint4(h2.x, h2.y, h3.x, h3.y);
@@ -341,11 +360,11 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
     }
   } else if (warp >= 6) {
     // --------------------------------------------------------- MMA issuers --
-    // Warps 6/7: score chains a/b over rings 0/1; warps 8/9: value chains a/b
-    // over rings 2/3.
+    // Warps 6/7: the score chains of the even / odd tiles over rings 0/1, into
+    // TMEM score buffers 0/1; warps 8/9: value chains a/b over rings 2/3.
     const int r = warp - 6;
     const bool scores = r < 2;
-    const bool has_chain = scores ? (r == 0 || two_s) : (r == 2 || two_v);
+    const bool has_chain = scores ? r < ntiles : (r == 2 || two_v);
     if (lane == 0 && has_chain) {
       const uint32_t idS = idesc_f16(64, 64, false, false);
       const uint32_t idO = idesc_f16(128, rows_pad, true, false);
@@ -357,8 +376,9 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
       uint32_t cnt = 0;
       if (scores) {
         const uint32_t d = tmem + r * 64;
-        for (int n = 0; n < ntiles && ok; ++n) {
-          if (n >= 1 && !wait8(smem_u32(s_free), (n - 1) & 1, abort_flag, a.err, ERR8_S)) { ok = false; break; }
+        for (int n = r; n < ntiles && ok; n += 2) {
+          // buffer r is free once the softmax has read tile n - 2's scores
+          if (n >= 2 && !wait8(smem_u32(&s_free[r]), ((n - 2) >> 1) & 1, abort_flag, a.err, ERR8_S)) { ok = false; break; }
           tc_fence_after();
           uint32_t acc = 0;
           for (int c = R.lo(r); c < R.hi(r) && ok; ++c, ++cnt) {
@@ -418,28 +438,19 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
     bool ok = true;
     for (int n = 0; n < ntiles; ++n) {
       const int buf = n % NBP, ss = n % NSB;
+      const int sb = n & 1;   // score buffer (and chain) of tile n
       if (tid == 0)
-        lead[0] = wait8(smem_u32(&s_full[0]), n & 1, abort_flag, a.err, ERR8_S) &&
-                  (!two_s || wait8(smem_u32(&s_full[1]), n & 1, abort_flag, a.err, ERR8_S)) &&
+        lead[0] = wait8(smem_u32(&s_full[sb]), (n >> 1) & 1, abort_flag, a.err, ERR8_S) &&
                   wait8(smem_u32(&sc_full[ss]), (n / NSB) & 1, abort_flag, a.err, ERR8_SC);
       named_sync(1, 128);
       if (!lead[0]) { ok = false; break; }
       tc_fence_after();
       float sc[64];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        tmem_ld16(tmem + q * 16 + lane_off, sc + q * 16);
-        if (two_s) {
-          float t[16];
-          tmem_ld16(tmem + 64 + q * 16 + lane_off, t);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) sc[q * 16 + j] += t[j];
-        }
-      }
+      for (int q = 0; q < 4; ++q) tmem_ld16(tmem + sb * 64 + q * 16 + lane_off, sc + q * 16);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(smem_u32(s_free));
+      mbar_arrive(smem_u32(&s_free[sb]));
       const float* scl = reinterpret_cast<const float*>(sc_s + ss * SBYTES);   // [64][4]: s^K, s^V, pad
       const int nvalid = min(TOK, min(tok1, rlim) - (tok0 + n * TOK));
 #pragma unroll
