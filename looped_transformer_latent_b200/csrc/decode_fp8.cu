@@ -11,31 +11,37 @@
 // so the tensor cores contract the codes and the scales are applied per token
 // on the softmax side.
 //
-// Codes become the f16 operands code * 2^-8, half of them by bit placement on
-// the integer pipe (an e4m3 byte s.eeee.mmm moved to the f16 bits
-// s.0eeee.mmm0000000 is exactly code * 2^-8: the exponent biases are 15 and
-// 7, and subnormal codes m * 2^-9 become the f16 subnormals m * 2^-17), half
-// by the conversion unit and a multiply by 2^-8; the scores take s^K * 2^8
-// and the value partials are multiplied by 2^8 when written.
+// Keys: the tensor cores take the codes as they land (tcgen05.mma of
+// kind::f8f6f4, e4m3 x e4m3, fp32 accumulate).  The query side is made 8-bit
+// once per CTA: each row of Q~ is scaled by a power of two 2^e_row that brings
+// its largest magnitude into (224, 448] and written as two e4m3 terms,
+// hi = e4m3(x 2^e) and lo = e4m3(x 2^e - hi), whose sum carries about 8
+// significant bits; S = 2^-e_row s^K (hi + lo) . codes^K.
+//
+// Values: the codes become the f16 operands code * 2^-8, half of them by bit
+// placement on the integer pipe (an e4m3 byte s.eeee.mmm moved to the f16
+// bits s.0eeee.mmm0000000 is exactly code * 2^-8: the exponent biases are 15
+// and 7, and subnormal codes m * 2^-9 become the f16 subnormals m * 2^-17),
+// half by the conversion unit and a multiply by 2^-8; the value partials are
+// multiplied by 2^8 when written.
 //
 // Four rings carry the chunks (64 tokens x 64 codes): the key chunks of the
-// even and of the odd 64-token tiles (rings 0 and 1, one chunk per slot, up
-// to four slots) and each tile's 128-wide value groups of the first and
-// second half of r_V (rings 2 and 3, two chunks per slot).  The codes land by
-// TMA in the upper half of a slot and one converter warp per ring rewrites
-// them in place into f16 chunk blocks (128-byte swizzle).  A producer thread
+// even and of the odd 64-token tiles (rings 0 and 1, one chunk per slot,
+// landed in the 64-byte swizzle the MMA reads) and each tile's 128-wide
+// value groups of the first and second half of r_V (rings 2 and 3, one group
+// per slot: the codes land token-major in the slot's upper half and two
+// converter warps per ring, one per half of the tokens, rewrite them in place
+// into two f16 chunk blocks in the 128-byte swizzle).  A producer thread
 // polls its two rings and issues whichever copy has a free slot.  Each ring
-// has its own MMA issuer warp, so the
-// four tcgen05 chains run concurrently (one thread's chain is bound by its own
-// issue latency):
-//   * two score chains S = Q~ codes^T (M = 64 rows, N = 64 tokens, f16 in,
-//     fp32 in TMEM), one for the even and one for the odd tiles, each into
-//     its own TMEM buffer, so a chain works on its next tile while the
-//     softmax reads the other's;
+// has its own MMA issuer warp, so the four tcgen05 chains run concurrently
+// (one thread's chain is bound by its own issue latency):
+//   * two score chains S (M = 64 rows, N = 64 tokens), one for the even and
+//     one for the odd tiles, each into its own TMEM buffer, so a chain works
+//     on its next tile while the softmax reads the other's;
 //   * two value chains O^T += codes^V^T P'^T over their value groups
-//     (M = 128 value indices, N = rows);
-//   * four softmax warps scale the scores by s^K, run the online softmax
-//     (base 2, lazy rescale) and write P' = p * s^V in f16.
+//     (M = 128 value indices, N = rows, f16 in);
+//   * four softmax warps scale the scores, run the online softmax (base 2,
+//     lazy rescale) and write P' = p * s^V in f16.
 // Every wait is bounded; on a timeout the CTA records an error code (the merge
 // then emits NaN), drains its copies and frees TMEM.
 #include <cuda.h>
@@ -54,19 +60,20 @@ using namespace ptx;
 constexpr int TOK = 64;
 constexpr int BLK = 8192;             // f16 chunk block: 64 tokens x 64 elements, 128-byte rows, swizzled
 constexpr int BLK8 = 4096;            // fp8 chunk block as landed: 64 tokens x 64 codes
-constexpr int SLOTK = BLK;            // key ring slot: one f16 chunk block; its codes land in the upper half
+constexpr int QBLK = 4096;            // 8-bit chunk block: 64 rows x 64 codes, 64-byte rows, 64-byte swizzle
+constexpr int SLOTK = QBLK;           // key ring slot: one landed code chunk, the MMA's operand as it is
 constexpr int SLOTV = 2 * BLK;        // value ring slot: two f16 chunk blocks (one 128-wide value group)
 constexpr int NRING = 4;              // key halves a/b, value halves a/b
 constexpr int NSB = 4;                // scale slots (one per tile)
 constexpr int SBYTES = TOK * 16;      // one tile's scales: 64 x (s^K, s^V, 8 pad bytes)
 constexpr int NBP = 2;                // P buffers (smem)
-constexpr int NTHREADS = 448;         // 0-3 softmax, 4/5 producers, 6/7 score MMA, 8/9 value MMA, 10-13 converters
+constexpr int NTHREADS = 448;         // 0-3 softmax, 4/5 producers, 6/7 score MMA, 8/9 value MMA, 10-13 value converters
 constexpr int SMEM_LIMIT = 232448;
-constexpr int MISC_BYTES = 512;
+constexpr int MISC_BYTES = 1024;
 constexpr long long WAIT_CYCLES = 1ll << 32;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t O_COL = 128;       // S_a at column 0, S_b at 64, the value groups from 128
-constexpr float CODE_UNIT = 256.f;    // f16 operand = code * 2^-8
+constexpr float CODE_UNIT = 256.f;    // f16 value operand = code * 2^-8
 
 enum : int { ERR8_EMPTY = 51, ERR8_LFULL = 52, ERR8_CFULL = 54, ERR8_Q = 55, ERR8_S = 56, ERR8_P = 57,
              ERR8_O = 58, ERR8_SC = 59 };
@@ -128,8 +135,9 @@ __device__ __forceinline__ uint2 code4_to_f16_cvt(uint32_t w) {
 
 struct Layout8 {
   int nkb, nvb, nsk, nsv;
-  __host__ __device__ int q_off() const { return 0; }
-  __host__ __device__ int p_off() const { return nkb * BLK; }
+  __host__ __device__ int qh_off() const { return 0; }
+  __host__ __device__ int ql_off() const { return nkb * QBLK; }
+  __host__ __device__ int p_off() const { return 2 * nkb * QBLK; }
   __host__ __device__ int sc_off() const { return p_off() + NBP * BLK; }
   __host__ __device__ int ring_off(int r) const {
     const int k0 = sc_off() + NSB * SBYTES;
@@ -137,7 +145,11 @@ struct Layout8 {
   }
   __host__ __device__ int nslots(int r) const { return r < 2 ? nsk : nsv; }
   __host__ __device__ int slot_bytes(int r) const { return r < 2 ? SLOTK : SLOTV; }
-  __host__ __device__ int land_off(int r) const { return r < 2 ? BLK8 : BLK; }   // where the codes land in a slot
+  __host__ __device__ int land_off(int r) const { return r < 2 ? 0 : BLK; }      // where the codes land in a slot
+  // Q~ in f16 (the query map's output) is staged in the ring memory, which is
+  // free until the rings start
+  __host__ __device__ int stage_off() const { return ring_off(0); }
+  __host__ __device__ int ring_bytes() const { return ring_off(NRING) - ring_off(0); }
   __host__ __device__ int step(int r) const { return r < 2 ? 1 : 2; }            // chunks per copy
   __host__ __device__ int bar0(int r) const { return r < 2 ? r * nsk : 2 * nsk + (r - 2) * nsv; }
   __host__ __device__ int ring_bars() const { return 2 * nsk + 2 * nsv; }
@@ -146,6 +158,15 @@ struct Layout8 {
   __host__ __device__ int misc_off() const { return bar_off() + 8 * nbars(); }
   __host__ __device__ int bytes() const { return misc_off() + MISC_BYTES; }
 };
+
+// Q~[t][k], Q~[t][k + 1] (k even) from the f16 staging copy: r_K/64 blocks of
+// 64 rows x 64 values, 128-byte rows in the 128-byte swizzle.
+__device__ __forceinline__ float2 q_pair(const uint8_t* stage, int t, int k) {
+  const uint8_t* blk = stage + (k >> 6) * BLK + t * 128;
+  const int kk = k & 63;
+  const __half2 v = *reinterpret_cast<const __half2*>(blk + (((kk >> 3) ^ (t & 7)) << 4) + (kk & 7) * 2);
+  return __half22float2(v);
+}
 
 // What ring r carries: the key rings every key chunk of the even (ring 0)
 // and the odd (ring 1) tiles; the value rings every tile's chunks of the
@@ -161,8 +182,9 @@ struct Rings {
 
 // 14 warps: four share an SM sub-partition's 16 K registers, so at most 128 per thread
 __global__ void __launch_bounds__(NTHREADS, 1)
-absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant__ CUtensorMap map1,
-                 const __grid_constant__ CUtensorMap mapsc, const AbsorbArgs a, const int nsk, const int nsv) {
+absorb_split_fp8(const __grid_constant__ CUtensorMap mapk, const __grid_constant__ CUtensorMap map64,
+                 const __grid_constant__ CUtensorMap map128, const __grid_constant__ CUtensorMap mapsc,
+                 const AbsorbArgs a, const int nsk, const int nsv) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Layout8 L;
@@ -172,7 +194,8 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
   R.ngrp = (L.nvb + 1) / 2;
   R.ga = (R.ngrp + 1) / 2;
   const bool two_v = R.ga < R.ngrp;     // a second value chain (r_V > 128)
-  uint8_t* q_s = base + L.q_off();
+  uint8_t* qh_s = base + L.qh_off();
+  uint8_t* ql_s = base + L.ql_off();
   uint8_t* p_s = base + L.p_off();
   uint8_t* sc_s = base + L.sc_off();
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L.bar_off());
@@ -192,6 +215,7 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   volatile int* lead = reinterpret_cast<volatile int*>(misc + 16);   // [4]
   float* alpha_s = reinterpret_cast<float*>(misc + 64);               // [64]
+  float* qinv_s = reinterpret_cast<float*>(misc + 320);               // [64] 2^-e of each Q~ row
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int s = blockIdx.x, b = blockIdx.y;
@@ -204,7 +228,7 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
   if (tid == 0) {
     for (int i = 0; i < L.ring_bars(); ++i) {
       mbar_init(smem_u32(&lfull[i]), 1);
-      mbar_init(smem_u32(&cfull[i]), 1);
+      mbar_init(smem_u32(&cfull[i]), 2);   // value groups: the two converter warps (unused on key rings)
       mbar_init(smem_u32(&rempty[i]), 1);
     }
     for (int i = 0; i < NSB; ++i) {
@@ -229,8 +253,9 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
     tmem_relinquish();
   }
   if (warp == 4 && lane == 0) {
-    prefetch_tmap(&map2);
-    prefetch_tmap(&map1);
+    prefetch_tmap(&mapk);
+    prefetch_tmap(&map64);
+    prefetch_tmap(&map128);
     prefetch_tmap(&mapsc);
   }
   tc_fence_before();
@@ -239,7 +264,62 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
   const uint32_t tmem = *tmem_slot;
   griddep_wait();
 
-  if (warp == 4 || warp == 5) {
+  // ---- Q~ to e4m3 hi/lo (once per CTA) --------------------------------------
+  // Q~ (f16, [r_k/64][64 rows x 64], 128-byte swizzle) lands in the ring
+  // memory; warp w takes rows w, w + 14, ...: the row's largest magnitude
+  // gives the power of two, then each pair of values becomes hi and lo codes,
+  // stored K-major in the 64-byte swizzle (16-byte piece q of row t at
+  // (t / 8) * 512 + (t % 8) * 64 + 16 (q ^ ((t / 2) % 4))).
+  bool q_ok = true;
+  {
+    uint8_t* stage = base + L.stage_off();
+    const uint32_t qb = smem_u32(q_full);
+    if (warp == 4 && lane == 0) {
+      mbar_arrive_tx(qb, nkb * BLK);
+      bulk_load(smem_u32(stage), a.qbf + (size_t)b * nkb * (BLK / 2), nkb * BLK, qb);
+    }
+    q_ok = wait8(qb, 0, abort_flag, a.err, ERR8_Q);
+    if (q_ok) {
+      for (int t = warp; t < 64; t += NTHREADS / 32) {
+        float amax = 0.f;
+        for (int k = 2 * lane; k < a.r_k; k += 64) {
+          const float2 v = q_pair(stage, t, k);
+          amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
+        }
+        amax = redux_max(amax);
+        // 2^e with amax * 2^e in (224, 448] (amax = m 2^x, m in [0.5, 1):
+        // e = 9 - x if m <= 0.875, else 8 - x); zero rows keep e = 0
+        float sc = 1.f;
+        if (amax > 0.f) {
+          int x;
+          const float m = frexpf(amax, &x);
+          sc = ldexpf(1.f, max(-126, min(127, (m <= 0.875f ? 9 : 8) - x)));
+        }
+        if (lane == 0) qinv_s[t] = 1.f / sc;
+        for (int k = 2 * lane; k < a.r_k; k += 64) {
+          const float2 v = q_pair(stage, t, k);
+          const float2 x = make_float2(v.x * sc, v.y * sc);
+          const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
+          const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(hi, __NV_E4M3);
+          const float2 hv = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+          const __nv_fp8x2_storage_t lo =
+              __nv_cvt_float2_to_fp8x2(make_float2(x.x - hv.x, x.y - hv.y), __NV_SATFINITE, __NV_E4M3);
+          const int kk = k & 63;
+          const uint32_t off = (uint32_t)((k >> 6) * QBLK + (t >> 3) * 512 + (t & 7) * 64 +
+                                          (((kk >> 4) ^ ((t >> 1) & 3)) << 4) + (kk & 15));
+          *reinterpret_cast<__nv_fp8x2_storage_t*>(qh_s + off) = hi;
+          *reinterpret_cast<__nv_fp8x2_storage_t*>(ql_s + off) = lo;
+        }
+      }
+    }
+    fence_proxy_async_smem();   // the codes are read by the MMAs; the staging area is reused by TMA
+    if (__syncthreads_or(!q_ok)) q_ok = false;
+  }
+
+  if (!q_ok) {
+    // Q~ never landed: nothing was issued but that copy; let it land (bounded)
+    if (warp == 4 && lane == 0) wait8(smem_u32(q_full), 0, abort_flag, nullptr, 0, false);
+  } else if (warp == 4 || warp == 5) {
     // ----------------------------------------------------------- producers --
     // Warp 4: Q~ (one bulk copy), the tiles' scales and the key copies of
     // rings 0 and 1; warp 5: the value copies of rings 2 and 3.  A copy is two
@@ -249,11 +329,6 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
     if (lane == 0) {
       const bool kside = warp == 4;
       const int r0 = kside ? 0 : 2, c0 = kside ? 0 : nkb;
-      const uint32_t qb = smem_u32(q_full);
-      if (kside) {
-        mbar_arrive_tx(qb, nkb * BLK);
-        bulk_load(smem_u32(q_s), a.qbf + (size_t)b * nkb * (BLK / 2), nkb * BLK, qb);
-      }
       uint32_t cnt[2] = {0, 0};
       int tile[2] = {R.tile0(r0), R.tile0(r0 + 1)}, chunk[2] = {R.lo(r0), R.lo(r0 + 1)};
       bool done[2] = {R.lo(r0) >= R.hi(r0) || tile[0] >= ntiles, R.lo(r0 + 1) >= R.hi(r0 + 1) || tile[1] >= ntiles};
@@ -279,8 +354,11 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
           const int c = chunk[k], w = min(L.step(r), R.hi(r) - c);
           const uint32_t fb = smem_u32(&lfull[L.bar0(r) + slot]);
           mbar_arrive_tx(fb, w * BLK8);
-          tma_load_4d(smem_u32(base + L.ring_off(r) + slot * L.slot_bytes(r) + L.land_off(r)),
-                      w == 2 ? (const void*)&map2 : (const void*)&map1, fb, 0, tok0 + tile[k] * TOK, c0 + c, b);
+          // keys: one chunk in the 64-byte swizzle (the MMA's operand as it
+          // lands); values: a group token-major (64 rows of 64 w codes)
+          tma_load_3d(smem_u32(base + L.ring_off(r) + slot * L.slot_bytes(r) + L.land_off(r)),
+                      r < 2 ? (const void*)&mapk : w == 2 ? (const void*)&map128 : (const void*)&map64, fb,
+                      (c0 + c) * 64, tok0 + tile[k] * TOK, b);
           ++cnt[k];
           chunk[k] = c + w;
           if (chunk[k] >= R.hi(r)) {
@@ -306,7 +384,6 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
       if (!ok) {
         // drain: every copy this producer issued must land before the CTA exits
         if (kside) {
-          wait8(qb, 0, abort_flag, nullptr, 0, false);
           for (int n = max(0, nsc - NSB); n < nsc; ++n)
             wait8(smem_u32(&sc_full[n % NSB]), (n / NSB) & 1, abort_flag, nullptr, 0, false);
         }
@@ -318,40 +395,43 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
       }
     }
   } else if (warp >= 10) {
-    // ----------------------------------------------------------- converters --
-    // Warp 10 + r rewrites ring r's landed codes into f16 blocks, copy by copy
-    // in the producer's order.  Per chunk each lane loads 8 x 16 codes (the
-    // warp reads the 4 KB block contiguously), the warp synchronises (the
-    // second chunk's f16 block overlaps its own codes), then each lane stores
-    // 8 x 32 bytes into the swizzled rows.
-    const int r = warp - 10, ns = L.nslots(r), stp = L.step(r);
+    // ----------------------------------------------------- value converters --
+    // Warp 10 + 2 (r - 2) + h rewrites tokens 32h .. 32h + 31 of value ring
+    // r's groups into f16 chunk blocks, copy by copy in the producer's order.
+    // The codes landed token-major (a token's 64 w codes in one row) in the
+    // slot's upper half, so the warp's f16 rows of both chunks cover its own
+    // codes and no other warp's: it loads its 2 or 4 KB, synchronises, and
+    // stores into the swizzled rows.
+    const int r = 2 + (warp - 10) / 2, h = (warp - 10) & 1;
+    const int ns = L.nslots(r);
     uint8_t* ring = base + L.ring_off(r);
     uint32_t cnt = 0;
     bool ok = true;
-    for (int n = R.tile0(r); n < ntiles && ok; n += R.tstep(r)) {
-      for (int c = R.lo(r); c < R.hi(r); c += stp, ++cnt) {
-        const int w = min(stp, R.hi(r) - c);
+    for (int n = 0; n < ntiles && ok; ++n) {
+      for (int c = R.lo(r); c < R.hi(r); c += 2, ++cnt) {
+        const int w = min(2, R.hi(r) - c);
         const uint32_t slot = cnt % ns, ph = cnt / ns;
         if (!wait8(smem_u32(&lfull[L.bar0(r) + slot]), ph & 1, abort_flag, a.err, ERR8_LFULL)) { ok = false; break; }
-        uint8_t* sl = ring + slot * L.slot_bytes(r);
-        for (int j = 0; j < w; ++j) {
-          const uint4* src = reinterpret_cast<const uint4*>(sl + L.land_off(r) + j * BLK8);
-          uint4 cw[8];
+        uint8_t* sl = ring + slot * SLOTV;
+        // 16-byte piece u of this warp's rows holds codes 16 (u % (4w)) .. of token 32h + u / (4w)
+        const uint4* src = reinterpret_cast<const uint4*>(sl + BLK + 32 * h * 64 * w);
+        const int npieces = 4 * w;   // per lane
+        uint4 cw[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) cw[k] = src[lane + 32 * k];
-          __syncwarp();
-          // 16-byte piece lane + 32k holds codes 16p..16p+15 of token row lane/4 + 8k
-          const int p = lane & 3, sw = (lane >> 2) & 7;
-          uint8_t* dst = sl + j * BLK + (lane >> 2) * 128;
+        for (int k = 0; k < 8; ++k)
+          if (k < npieces) cw[k] = src[lane + 32 * k];
+        __syncwarp();
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint2 h0 = code4_to_f16(cw[k].x), h1 = code4_to_f16_cvt(cw[k].y);
-            const uint2 h2 = code4_to_f16(cw[k].z), h3 = code4_to_f16_cvt(cw[k].w);
-            uint8_t* drow = dst + k * 8 * 128;
-            *reinterpret_cast<uint4*>(drow + (((2 * p) ^ sw) << 4)) = make_uint4(h0.x, h0.y, h1.x, h1.y);
-            *reinterpret_cast<uint4*>(drow + (((2 * p + 1) ^ sw) << 4)) = make_uint4(h2.x, h2.y, h3.x, h3.y);
-          }
-          __syncwarp();
+        for (int k = 0; k < 8; ++k) {
+          if (k >= npieces) break;
+          const int u = lane + 32 * k, per = 4 * w;
+          const int t = 32 * h + u / per, j = (u % per) >> 2, p = u & 3;
+          uint8_t* drow = sl + j * BLK + t * 128;
+          const int sw = t & 7;
+          const uint2 h0 = code4_to_f16(cw[k].x), h1 = code4_to_f16_cvt(cw[k].y);
+          const uint2 h2 = code4_to_f16(cw[k].z), h3 = code4_to_f16_cvt(cw[k].w);
+          *reinterpret_cast<uint4*>(drow + (((2 * p) ^ sw) << 4)) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+          *reinterpret_cast<uint4*>(drow + (((2 * p + 1) ^ sw) << 4)) = make_uint4(h2.x, h2.y, h3.x, h3.y);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -366,13 +446,14 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
     const bool scores = r < 2;
     const bool has_chain = scores ? r < ntiles : (r == 2 || two_v);
     if (lane == 0 && has_chain) {
-      const uint32_t idS = idesc_f16(64, 64, false, false);
+      const uint32_t idS = idesc_e4m3(64, 64);
       const uint32_t idO = idesc_f16(128, rows_pad, true, false);
-      const uint64_t q_desc = smem_desc_sw128(smem_u32(q_s), 16, 1024);
-      const uint64_t k_desc = smem_desc_sw128(smem_u32(base + L.ring_off(r)), 16, 1024);
+      const uint64_t qh_desc = smem_desc_sw64(smem_u32(qh_s));
+      const uint64_t ql_desc = smem_desc_sw64(smem_u32(ql_s));
+      const uint64_t k_desc = smem_desc_sw64(smem_u32(base + L.ring_off(r)));
       const uint64_t v_desc = smem_desc_sw128(smem_u32(base + L.ring_off(r)), BLK, 1024);
       const uint64_t p_desc = smem_desc_sw128(smem_u32(p_s), 16, 1024);
-      bool ok = !scores || wait8(smem_u32(q_full), 0, abort_flag, a.err, ERR8_Q);
+      bool ok = true;
       uint32_t cnt = 0;
       if (scores) {
         const uint32_t d = tmem + r * 64;
@@ -382,16 +463,21 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
           tc_fence_after();
           uint32_t acc = 0;
           for (int c = R.lo(r); c < R.hi(r) && ok; ++c, ++cnt) {
+            // the landed key chunk is the operand: wait for the copy itself
             const uint32_t slot = cnt % nsk, ph = cnt / nsk;
-            if (!wait8(smem_u32(&cfull[L.bar0(r) + slot]), ph & 1, abort_flag, a.err, ERR8_CFULL)) { ok = false; break; }
+            if (!wait8(smem_u32(&lfull[L.bar0(r) + slot]), ph & 1, abort_flag, a.err, ERR8_LFULL)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t ad = q_desc + (uint64_t)((c * BLK) >> 4);
+            const uint64_t ah = qh_desc + (uint64_t)((c * QBLK) >> 4);
+            const uint64_t al = ql_desc + (uint64_t)((c * QBLK) >> 4);
             const uint64_t bd = k_desc + (uint64_t)((slot * SLOTK) >> 4);
+            // K = 32 codes (32 bytes) per MMA: two steps per chunk, hi then lo
 #pragma unroll
-            for (int k16 = 0; k16 < 4; ++k16) {
-              mma_bf16(d, ad + 2 * k16, bd + 2 * k16, idS, acc);
+            for (int k32 = 0; k32 < 2; ++k32) {
+              mma_f8f6f4(d, ah + 2 * k32, bd + 2 * k32, idS, acc);
               acc = 1;
             }
+#pragma unroll
+            for (int k32 = 0; k32 < 2; ++k32) mma_f8f6f4(d, al + 2 * k32, bd + 2 * k32, idS, 1u);
             mma_commit(smem_u32(&rempty[L.bar0(r) + slot]));
           }
           if (!ok) break;
@@ -434,6 +520,7 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
     // last latent token (exclusive) of this row's query position
     const int rlim = a.nq > 1 ? a.n_lat - (a.nq - 1 - r / a.rows_per_q) : a.n_lat;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const float qinv = qinv_s[r];   // 2^-e of this row's 8-bit query terms
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int n = 0; n < ntiles; ++n) {
@@ -454,7 +541,7 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap map2, const __grid_constant
       const float* scl = reinterpret_cast<const float*>(sc_s + ss * SBYTES);   // [64][4]: s^K, s^V, pad
       const int nvalid = min(TOK, min(tok1, rlim) - (tok0 + n * TOK));
 #pragma unroll
-      for (int c = 0; c < 64; ++c) sc[c] = c < nvalid ? sc[c] * (scl[4 * c] * CODE_UNIT) : -INFINITY;
+      for (int c = 0; c < 64; ++c) sc[c] = c < nvalid ? sc[c] * (scl[4 * c] * qinv) : -INFINITY;
       float mx[4] = {sc[0], sc[1], sc[2], sc[3]};
 #pragma unroll
       for (int c = 4; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], sc[c]);
@@ -567,20 +654,29 @@ int fp8_smem(int r_k, int r_v, int nsk, int nsv) {
   return L.bytes() + 1024;
 }
 
-// the deepest rings shared memory allows: key rings of 4..2 chunks with two
-// value groups per value ring, else 2 and 1
-void fp8_slots(int r_k, int r_v, int* nsk, int* nsv) {
-  static const int opts[4][2] = {{4, 2}, {3, 2}, {2, 2}, {2, 1}};
+// ring memory must also hold the f16 staging copy of Q~ (r_K/64 blocks of 8 KB)
+bool fp8_fits(int r_k, int r_v, int nsk, int nsv) {
+  Layout8 L;
+  L.nkb = r_k / 64; L.nvb = r_v / 64; L.nsk = nsk; L.nsv = nsv;
+  return fp8_smem(r_k, r_v, nsk, nsv) <= SMEM_LIMIT && L.ring_bytes() >= L.nkb * BLK;
+}
+
+// ring depths, first that fits: value rings of three groups (a tile's worth
+// for r_V up to 768, measured the better split) with key rings of four
+// chunks, then shallower
+bool fp8_slots(int r_k, int r_v, int* nsk, int* nsv) {
+  static const int opts[7][2] = {{4, 3}, {8, 2}, {6, 2}, {4, 2}, {3, 2}, {2, 2}, {2, 1}};
   for (const auto& o : opts)
-    if (fp8_smem(r_k, r_v, o[0], o[1]) <= SMEM_LIMIT) { *nsk = o[0]; *nsv = o[1]; return; }
-  *nsk = 2; *nsv = 1;
+    if (fp8_fits(r_k, r_v, o[0], o[1])) { *nsk = o[0]; *nsv = o[1]; return true; }
+  return false;
 }
 
 }  // namespace
 
 bool absorb_fp8_supported(int r_k, int r_v, int rows) {
   if (r_k % 64 || r_v % 64 || r_k < 64 || r_v < 64 || r_k > 768) return false;
-  if (rows < 1 || rows > 64 || fp8_smem(r_k, r_v, 2, 1) > SMEM_LIMIT) return false;
+  int nsk, nsv;
+  if (rows < 1 || rows > 64 || !fp8_slots(r_k, r_v, &nsk, &nsv)) return false;
   const int ngrp = (r_v / 64 + 1) / 2;
   return O_COL + (uint32_t)(ngrp * absorb_tc_rows_pad(rows)) <= TMEM_COLS;
 }
@@ -588,20 +684,22 @@ bool absorb_fp8_supported(int r_k, int r_v, int rows) {
 cudaError_t launch_absorb_split_fp8(const AbsorbArgs& a, cudaStream_t st) {
   TmapEncodeFn enc = tmap_encoder();
   if (!enc) return cudaErrorNotSupported;
-  // codes: 4-D byte view (64 codes, token, 64-code chunk, sequence); boxes of
-  // one or two chunks x 64 tokens land as dense 4 KB chunk blocks
+  // codes: 3-D byte view (code byte of the row, token, sequence).  Keys: boxes
+  // of 64 codes x 64 tokens in the 64-byte swizzle (the MMA's K-major
+  // operand); values: boxes of 128 or 64 codes x 64 tokens, token-major
   const cuuint64_t row_bytes = (cuuint64_t)a.ls_n;
   cuuint64_t batch_bytes = (cuuint64_t)a.ls_b;
   if (a.B == 1 && batch_bytes < row_bytes * (cuuint64_t)a.n_lat) batch_bytes = row_bytes * (cuuint64_t)a.n_lat;
-  const cuuint64_t dims[4] = {64, (cuuint64_t)a.n_lat, (cuuint64_t)((a.r_k + a.r_v) / 64), (cuuint64_t)a.B};
-  const cuuint64_t strides[3] = {row_bytes, 64, batch_bytes};
-  cuuint32_t es[4] = {1, 1, 1, 1};
-  CUtensorMap map2, map1, mapsc;
-  for (int w = 1; w <= 2; ++w) {
-    const cuuint32_t box[4] = {64, TOK, (cuuint32_t)w, 1};
-    if (enc(w == 2 ? &map2 : &map1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(a.lat), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+  const cuuint64_t dims[3] = {(cuuint64_t)(a.r_k + a.r_v), (cuuint64_t)a.n_lat, (cuuint64_t)a.B};
+  const cuuint64_t strides[2] = {row_bytes, batch_bytes};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUtensorMap mapk, map64, map128, mapsc;
+  for (int m = 0; m < 3; ++m) {
+    const cuuint32_t box[3] = {m == 2 ? 128u : 64u, TOK, 1};
+    CUtensorMap* dst = m == 0 ? &mapk : m == 1 ? &map64 : &map128;
+    if (enc(dst, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(a.lat), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, m == 0 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
   // scales: 3-D byte view (16 bytes at offset r_k + r_v of each row, token, sequence)
@@ -614,12 +712,13 @@ cudaError_t launch_absorb_split_fp8(const AbsorbArgs& a, cudaStream_t st) {
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   int nsk = 2, nsv = 1;
-  fp8_slots(a.r_k, a.r_v, &nsk, &nsv);
+  if (!fp8_slots(a.r_k, a.r_v, &nsk, &nsv)) return cudaErrorNotSupported;
   const int smem = fp8_smem(a.r_k, a.r_v, nsk, nsv);
   cudaError_t e = cudaFuncSetAttribute(absorb_split_fp8, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.S, a.B);
-  return launch_kernel(absorb_split_fp8, grid, dim3(NTHREADS), smem, st, 1, map2, map1, mapsc, a, nsk, nsv);
+  return launch_kernel(absorb_split_fp8, grid, dim3(NTHREADS), smem, st, 1, mapk, map64, map128, mapsc, a, nsk,
+                       nsv);
 }
 
 }  // namespace lla
