@@ -16,7 +16,8 @@
 // once per CTA: each row of Q~ is scaled by a power of two 2^e_row that brings
 // its largest magnitude into (224, 448] and written as two e4m3 terms,
 // hi = e4m3(x 2^e) and lo = e4m3(x 2^e - hi), whose sum carries about 8
-// significant bits; S = 2^-e_row s^K (hi + lo) . codes^K.
+// significant bits, on lines 2 row and 2 row + 1 of the operand;
+// S = 2^-e_row s^K (hi + lo) . codes^K.
 //
 // Values: the codes become the f16 operands code * 2^-8, half of them by bit
 // placement on the integer pipe (an e4m3 byte s.eeee.mmm moved to the f16
@@ -35,9 +36,13 @@
 // polls its two rings and issues whichever copy has a free slot.  Each ring
 // has its own MMA issuer warp, so the four tcgen05 chains run concurrently
 // (one thread's chain is bound by its own issue latency):
-//   * two score chains S (M = 64 rows, N = 64 tokens), one for the even and
-//     one for the odd tiles, each into its own TMEM buffer, so a chain works
-//     on its next tile while the softmax reads the other's;
+//   * two score chains (M = 128: the hi and lo terms of the 64 query rows on
+//     interleaved lines, N = 64 tokens, K = 32), one for the even and one for
+//     the odd tiles, each into its own TMEM buffer, so a chain works on its
+//     next tile while the softmax reads the other's; the hi and lo partial
+//     scores of a row sit in adjacent TMEM lanes, and the two softmax lanes
+//     that hold them add them with one shuffle per column pair, each keeping
+//     half of the row's columns;
 //   * two value chains O^T += codes^V^T P'^T over their value groups
 //     (M = 128 value indices, N = rows, f16 in);
 //   * four softmax warps scale the scores, run the online softmax (base 2,
@@ -60,8 +65,8 @@ using namespace ptx;
 constexpr int TOK = 64;
 constexpr int BLK = 8192;             // f16 chunk block: 64 tokens x 64 elements, 128-byte rows, swizzled
 constexpr int BLK8 = 4096;            // fp8 chunk block as landed: 64 tokens x 64 codes
-constexpr int QBLK = 4096;            // 8-bit chunk block: 64 rows x 64 codes, 64-byte rows, 64-byte swizzle
-constexpr int SLOTK = QBLK;           // key ring slot: one landed code chunk, the MMA's operand as it is
+constexpr int QBLK = 8192;            // query chunk block: 128 lines (hi, lo of 64 rows) x 64 codes, 64-byte swizzle
+constexpr int SLOTK = 4096;           // key ring slot: one landed code chunk (64 x 64), the MMA's operand as it is
 constexpr int SLOTV = 2 * BLK;        // value ring slot: two f16 chunk blocks (one 128-wide value group)
 constexpr int NRING = 4;              // key halves a/b, value halves a/b
 constexpr int NSB = 4;                // scale slots (one per tile)
@@ -135,9 +140,8 @@ __device__ __forceinline__ uint2 code4_to_f16_cvt(uint32_t w) {
 
 struct Layout8 {
   int nkb, nvb, nsk, nsv;
-  __host__ __device__ int qh_off() const { return 0; }
-  __host__ __device__ int ql_off() const { return nkb * QBLK; }
-  __host__ __device__ int p_off() const { return 2 * nkb * QBLK; }
+  __host__ __device__ int q8_off() const { return 0; }
+  __host__ __device__ int p_off() const { return nkb * QBLK; }
   __host__ __device__ int sc_off() const { return p_off() + NBP * BLK; }
   __host__ __device__ int ring_off(int r) const {
     const int k0 = sc_off() + NSB * SBYTES;
@@ -194,8 +198,7 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap mapk, const __grid_constant
   R.ngrp = (L.nvb + 1) / 2;
   R.ga = (R.ngrp + 1) / 2;
   const bool two_v = R.ga < R.ngrp;     // a second value chain (r_V > 128)
-  uint8_t* qh_s = base + L.qh_off();
-  uint8_t* ql_s = base + L.ql_off();
+  uint8_t* q8_s = base + L.q8_off();
   uint8_t* p_s = base + L.p_off();
   uint8_t* sc_s = base + L.sc_off();
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L.bar_off());
@@ -268,8 +271,9 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap mapk, const __grid_constant
   // Q~ (f16, [r_k/64][64 rows x 64], 128-byte swizzle) lands in the ring
   // memory; warp w takes rows w, w + 14, ...: the row's largest magnitude
   // gives the power of two, then each pair of values becomes hi and lo codes,
-  // stored K-major in the 64-byte swizzle (16-byte piece q of row t at
-  // (t / 8) * 512 + (t % 8) * 64 + 16 (q ^ ((t / 2) % 4))).
+  // stored K-major in the 64-byte swizzle (16-byte piece q of line L at
+  // (L / 8) * 512 + (L % 8) * 64 + 16 (q ^ ((L / 2) % 4)); hi on line 2t, lo
+  // on line 2t + 1 of row t).
   bool q_ok = true;
   {
     uint8_t* stage = base + L.stage_off();
@@ -305,10 +309,13 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap mapk, const __grid_constant
           const __nv_fp8x2_storage_t lo =
               __nv_cvt_float2_to_fp8x2(make_float2(x.x - hv.x, x.y - hv.y), __NV_SATFINITE, __NV_E4M3);
           const int kk = k & 63;
-          const uint32_t off = (uint32_t)((k >> 6) * QBLK + (t >> 3) * 512 + (t & 7) * 64 +
-                                          (((kk >> 4) ^ ((t >> 1) & 3)) << 4) + (kk & 15));
-          *reinterpret_cast<__nv_fp8x2_storage_t*>(qh_s + off) = hi;
-          *reinterpret_cast<__nv_fp8x2_storage_t*>(ql_s + off) = lo;
+          // hi on line 2t, lo on line 2t + 1 of the chunk's 128 lines
+          const int lh = 2 * t, ll = 2 * t + 1;
+          const uint32_t blk = (uint32_t)((k >> 6) * QBLK + (kk & 15));
+          const uint32_t oh = blk + (lh >> 3) * 512 + (lh & 7) * 64 + ((((kk >> 4) ^ ((lh >> 1) & 3))) << 4);
+          const uint32_t ol = blk + (ll >> 3) * 512 + (ll & 7) * 64 + ((((kk >> 4) ^ ((ll >> 1) & 3))) << 4);
+          *reinterpret_cast<__nv_fp8x2_storage_t*>(q8_s + oh) = hi;
+          *reinterpret_cast<__nv_fp8x2_storage_t*>(q8_s + ol) = lo;
         }
       }
     }
@@ -446,10 +453,9 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap mapk, const __grid_constant
     const bool scores = r < 2;
     const bool has_chain = scores ? r < ntiles : (r == 2 || two_v);
     if (lane == 0 && has_chain) {
-      const uint32_t idS = idesc_e4m3(64, 64);
+      const uint32_t idS = idesc_e4m3(128, 64);
       const uint32_t idO = idesc_f16(128, rows_pad, true, false);
-      const uint64_t qh_desc = smem_desc_sw64(smem_u32(qh_s));
-      const uint64_t ql_desc = smem_desc_sw64(smem_u32(ql_s));
+      const uint64_t q8_desc = smem_desc_sw64(smem_u32(q8_s));
       const uint64_t k_desc = smem_desc_sw64(smem_u32(base + L.ring_off(r)));
       const uint64_t v_desc = smem_desc_sw128(smem_u32(base + L.ring_off(r)), BLK, 1024);
       const uint64_t p_desc = smem_desc_sw128(smem_u32(p_s), 16, 1024);
@@ -467,17 +473,15 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap mapk, const __grid_constant
             const uint32_t slot = cnt % nsk, ph = cnt / nsk;
             if (!wait8(smem_u32(&lfull[L.bar0(r) + slot]), ph & 1, abort_flag, a.err, ERR8_LFULL)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t ah = qh_desc + (uint64_t)((c * QBLK) >> 4);
-            const uint64_t al = ql_desc + (uint64_t)((c * QBLK) >> 4);
+            const uint64_t ad = q8_desc + (uint64_t)((c * QBLK) >> 4);
             const uint64_t bd = k_desc + (uint64_t)((slot * SLOTK) >> 4);
-            // K = 32 codes (32 bytes) per MMA: two steps per chunk, hi then lo
+            // M = 128 lines (hi and lo of each row, interleaved), K = 32 codes
+            // (32 bytes) per MMA: two steps per chunk
 #pragma unroll
             for (int k32 = 0; k32 < 2; ++k32) {
-              mma_f8f6f4(d, ah + 2 * k32, bd + 2 * k32, idS, acc);
+              mma_f8f6f4(d, ad + 2 * k32, bd + 2 * k32, idS, acc);
               acc = 1;
             }
-#pragma unroll
-            for (int k32 = 0; k32 < 2; ++k32) mma_f8f6f4(d, al + 2 * k32, bd + 2 * k32, idS, 1u);
             mma_commit(smem_u32(&rempty[L.bar0(r) + slot]));
           }
           if (!ok) break;
@@ -514,9 +518,12 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap mapk, const __grid_constant
     }
   } else {
     // -------------------------------------------------------- softmax warps --
-    const int r = 16 * warp + (lane & 15);
-    const bool owner = lane < 16;
-    const bool active = owner && r < rows;
+    // TMEM lane 32w + l holds the hi (l even) or lo (l odd) part of query row
+    // 16w + l/2; the pair swaps halves so that the even lane owns columns
+    // 0..31 of the row's scores and the odd lane columns 32..63.
+    const int r = 16 * warp + (lane >> 1), part = lane & 1;
+    const bool owner = part == 0;
+    const bool active = r < rows;
     // last latent token (exclusive) of this row's query position
     const int rlim = a.nq > 1 ? a.n_lat - (a.nq - 1 - r / a.rows_per_q) : a.n_lat;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
@@ -532,20 +539,31 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap mapk, const __grid_constant
       named_sync(1, 128);
       if (!lead[0]) { ok = false; break; }
       tc_fence_after();
-      float sc[64];
+      float sc[32];
+      {
+        float raw[64];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld16(tmem + sb * 64 + q * 16 + lane_off, sc + q * 16);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&s_free[sb]));
-      const float* scl = reinterpret_cast<const float*>(sc_s + ss * SBYTES);   // [64][4]: s^K, s^V, pad
-      const int nvalid = min(TOK, min(tok1, rlim) - (tok0 + n * TOK));
+        for (int q = 0; q < 4; ++q) tmem_ld16(tmem + sb * 64 + q * 16 + lane_off, raw + q * 16);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&s_free[sb]));
+        // keep this lane's half, add the partner's part of it
 #pragma unroll
-      for (int c = 0; c < 64; ++c) sc[c] = c < nvalid ? sc[c] * (scl[4 * c] * qinv) : -INFINITY;
+        for (int j = 0; j < 32; ++j) {
+          const float keep = part ? raw[32 + j] : raw[j];
+          const float give = part ? raw[j] : raw[32 + j];
+          sc[j] = keep + __shfl_xor_sync(0xffffffffu, give, 1);
+        }
+      }
+      const float* scl = reinterpret_cast<const float*>(sc_s + ss * SBYTES) + 4 * 32 * part;   // [32][4]: s^K, s^V, pad
+      const int nvalid = min(TOK, min(tok1, rlim) - (tok0 + n * TOK)) - 32 * part;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) sc[c] = c < nvalid ? sc[c] * (scl[4 * c] * qinv) : -INFINITY;
       float mx[4] = {sc[0], sc[1], sc[2], sc[3]};
 #pragma unroll
-      for (int c = 4; c < 64; ++c) mx[c & 3] = fmaxf(mx[c & 3], sc[c]);
-      const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      for (int c = 4; c < 32; ++c) mx[c & 3] = fmaxf(mx[c & 3], sc[c]);
+      float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
       bool need = false;
       float alpha = 1.f;
       if (active) {
@@ -567,9 +585,9 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap mapk, const __grid_constant
       const float mneg = (active && m_run != -INFINITY) ? -m_run : -INFINITY;
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       uint8_t* prow = p_s + buf * BLK + r * 128;
-      const bool store = owner && r < rows_pad;
+      const bool store = r < rows_pad;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
+      for (int ch = 0; ch < 4; ++ch) {
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -579,10 +597,11 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap mapk, const __grid_constant
           ps[(c >> 1) & 7] += p0 + p1;
           pk[e] = pack_f16(p0 * scl[4 * c + 1], p1 * scl[4 * c + 5]);
         }
-        if (store) *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        const int unit = 4 * part + ch;   // 16-byte unit of the row: columns 8 unit ..
+        if (store) *reinterpret_cast<uint4*>(prow + ((unit ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      l_run = l_run * alpha + psum;
+      l_run = l_run * alpha + psum;   // this lane's half of the row
       if (named_any(1, 128, need)) {
         // rescale the TMEM accumulators once O(n-1) has landed (before P(n)
         // is published, after the scores are dead: fewer live registers)
@@ -617,10 +636,11 @@ absorb_split_fp8(const __grid_constant__ CUtensorMap mapk, const __grid_constant
     }
     if (ok) {
       tc_fence_after();
-      if (active) {
+      const float l_row = l_run + __shfl_xor_sync(0xffffffffu, l_run, 1);
+      if (active && owner) {
         float* ml = a.part_ml + (((int64_t)s * a.B + b) * rows + r) * 2;
         ml[0] = m_run;
-        ml[1] = l_run;
+        ml[1] = l_row;
       }
       float* py = a.part_y + ((int64_t)s * a.B + b) * rows * (int64_t)a.r_v;
       for (int g = 0; g < ngrp; ++g) {
