@@ -56,7 +56,8 @@
  *             (its status was already returned when it was enqueued).
  * Precision.  Accumulation is fp32 throughout.  bf16 latents are read on the
  *             tensor cores (query operand rounded to bf16 for the score MMA,
- *             probabilities to bf16 for the accumulate MMA, tf32 maps); bf16
+ *             probabilities to bf16 for the accumulate MMA, tf32 maps; fp8
+ *             rows: query as two e4m3 terms, probabilities in f16); bf16
  *             writer rows use 3xTF32 products (fp32-accurate) before one
  *             round-to-nearest-even; the LLA reconstruction rounds each fp32
  *             decoder to bf16 for its tensor-core product (about 2^-9
@@ -110,7 +111,9 @@ typedef enum {
  * "Conclusion / Future directions": combining the latents with quantisation;
  * per-token, per-part scales are this library's reading).  Written by
  * lla_write_latents (HLA and FOLDED modes) and read by hla_decode_attn on the
- * tensor cores (codes widened exactly to f16). */
+ * tensor cores: key codes are contracted as e4m3 against the absorbed query
+ * written as two e4m3 terms (hi + lo, about 8 significant bits, under a
+ * per-row power of two), value codes are widened exactly to f16. */
 typedef enum { LLA_F32 = 0, LLA_BF16 = 1, LLA_FP8_E4M3 = 2 } lla_dtype;
 
 /* Version of this ABI; bumped whenever a struct below changes. */
