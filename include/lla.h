@@ -291,6 +291,18 @@ typedef struct {
    * (Wcap >= min(N, W + nq)), and every latent tile is shared by all
    * nq * nt * H rows on the tensor cores (at most 64 rows; bf16 or fp8 rows). */
   int32_t nq;
+  /* Optional concurrency for the exact window (HLA summary eq. 4, second
+   * sum), which needs neither the query map nor the latent read: NULL, or a
+   * stream of the caller's on which the call runs its window kernels while
+   * the query map and the latent read run on `stream`.  win_events is then
+   * the address of two cudaEvent_t values of the caller's (fork, join): the
+   * call records fork on `stream` after zeroing its error word, makes
+   * win_stream wait on it, records join on win_stream after the window, and
+   * makes `stream` wait on join before the output map; under stream capture
+   * this is the usual fork and join.  Results are bit-identical to the
+   * single-stream call.  win_stream without win_events: LLA_ERR_NULL. */
+  lla_stream win_stream;
+  void *win_events;
 } hla_decode_params;
 
 size_t hla_decode_workspace_bytes(const hla_decode_params *p);

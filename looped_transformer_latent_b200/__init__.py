@@ -245,8 +245,26 @@ def _events(p, timing_events):
     p.timing_events = ctypes.cast(arr, ctypes.c_void_p)
 
 
+def _win_side(p, win_stream, win_events):
+    """Attach the optional window stream and its (fork, join) torch.cuda.Event pair."""
+    if win_stream is None:
+        p.win_stream = None
+        p.win_events = None
+        return
+    if win_events is None:
+        raise ValueError("win_stream needs win_events: a (fork, join) pair of torch.cuda.Event")
+    ev0, ev1 = win_events
+    for ev in (ev0, ev1):
+        if ev.cuda_event == 0:
+            raise ValueError("record each window event once before passing it (creates the handle)")
+    arr = (ctypes.c_void_p * 2)(ev0.cuda_event, ev1.cuda_event)
+    p._keep_win = arr
+    p.win_stream = ctypes.c_void_p(win_stream.cuda_stream)
+    p.win_events = ctypes.cast(arr, ctypes.c_void_p)
+
+
 def _hla_params(lat, A, Bm, q, win_k, win_v, out, N, W, t0, r_k, rotate_query, rope_base, scale,
-                timing_events=None):
+                timing_events=None, win_stream=None, win_events=None):
     p = _abi.HlaDecodeParams()
     if q.dim() == 5:                       # [B, nq, nt, H, d_h]: the last nq positions at once
         B, nq, nt, H, d_h = q.shape
@@ -284,6 +302,7 @@ def _hla_params(lat, A, Bm, q, win_k, win_v, out, N, W, t0, r_k, rotate_query, r
     p.out_stride_b = out.stride(0)
     p.scale = float(scale)
     _events(p, timing_events)
+    _win_side(p, win_stream, win_events)
     return p
 
 
@@ -294,7 +313,8 @@ def hla_decode_workspace_bytes(**kw):
 
 def _hla_kw(kw):
     d = dict(lat=None, A=None, Bm=None, q=None, win_k=None, win_v=None, out=None, N=None, W=None,
-             t0=0, r_k=None, rotate_query=True, rope_base=10000.0, scale=0.0, timing_events=None)
+             t0=0, r_k=None, rotate_query=True, rope_base=10000.0, scale=0.0, timing_events=None,
+             win_stream=None, win_events=None)
     unknown = set(kw) - set(d) - {"workspace", "stream"}
     if unknown:
         raise TypeError(f"unknown arguments {sorted(unknown)}")
@@ -309,7 +329,10 @@ def hla_decode_attn(*, workspace=None, stream=None, **kw):
     uint8 fp8 rows of r_k+r_v+16 bytes), A [nt,H,d_h,r_k], Bm [nt,H,r_v,d_h],
     q [B,nt,H,d_h] (or [B,nq,nt,H,d_h]: the last nq positions of the context
     at once), ring win_k/win_v [B,T,Wcap,H,d_h], out shaped like q, float32;
-    N = context length, W = exact window, t0 = first loop served.
+    N = context length, W = exact window, t0 = first loop served.  Optional
+    win_stream (torch.cuda.Stream) with win_events (a (fork, join) pair of
+    torch.cuda.Event, each recorded once beforehand): the window runs on
+    win_stream beside the query map and the latent read.
     """
     args = _hla_kw(kw)
     dev = _cuda(args["lat"], args["A"], args["Bm"], args["q"], args["win_k"], args["win_v"], args["out"])

@@ -93,6 +93,8 @@ class HlaDecodeParams(ctypes.Structure):
         ("scale", c_f32),
         ("timing_events", c_vp),
         ("nq", c_i32),
+        ("win_stream", c_vp),
+        ("win_events", c_vp),
     ]
 
 

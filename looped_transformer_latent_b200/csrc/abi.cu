@@ -21,7 +21,7 @@ bool pdl_enabled() {
 
 namespace {
 
-constexpr int kAbiVersion = 3;   // 2: LLA_FP8_E4M3 latent rows; 3: hla_decode_params.nq
+constexpr int kAbiVersion = 4;   // 2: LLA_FP8_E4M3 latent rows; 3: hla_decode_params.nq; 4: win_stream
 constexpr int kDefaultSms = 148;        // B200; used only when no device can be queried
 constexpr int kMaxDevices = 64;
 constexpr size_t kAlign = 256;
@@ -146,6 +146,7 @@ WriterArgs writer_args(const lla_write_params& p) {
 
 // ------------------------------------------------------- decode checks --
 int check_hla(const hla_decode_params& p) {
+  if (p.win_stream && !p.win_events) return LLA_ERR_NULL;
   if (p.B < 0 || p.nt < 0 || p.nq < 0) return LLA_ERR_SHAPE;
   const int nq = p.nq > 1 ? p.nq : 1;
   if (!lat_dtype_ok(p.lat_dtype) || !dtype_ok(p.win_dtype)) return LLA_ERR_DTYPE;
@@ -426,6 +427,13 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
   qm.qlat = a.qlat; qm.qbf = a.qbf;
   cudaError_t e = cudaSuccess;
   e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
+  // optional: the window on the caller's second stream, beside the map and the read
+  const cudaStream_t sw = p->win_stream ? static_cast<cudaStream_t>(p->win_stream) : s;
+  cudaEvent_t* wev = reinterpret_cast<cudaEvent_t*>(p->win_events);
+  if (e == cudaSuccess && sw != s) {
+    e = cudaEventRecord(wev[0], s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sw, wev[0], 0);
+  }
   if (e == cudaSuccess) {
     // tensor-core map when the shapes allow a tensor-map view, else the SIMT map
     e = query_map_tc_ok(qm) ? launch_query_map_tc(qm, a.err, s) : cudaErrorNotSupported;
@@ -449,7 +457,11 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
     wa.rotate = a.rotate; wa.pos = ip; wa.base = a.base;
     wa.win_ml = a.win_ml; wa.win_y = a.win_y; wa.err = a.err;
     wa.rows_total = a.rows; wa.row0 = qp * rows_q;
-    e = launch_window(wa, s);
+    e = launch_window(wa, sw);
+  }
+  if (e == cudaSuccess && sw != s) {
+    e = cudaEventRecord(wev[1], sw);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, wev[1], 0);
   }
   if (e == cudaSuccess) {
     MapArgs om;

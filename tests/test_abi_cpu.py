@@ -80,6 +80,7 @@ def _call_hla(lib, p, ws=0x100000, nbytes=1 << 30):
     (dict(lat=0), _abi.LLA_ERR_NULL),
     (dict(A=0), _abi.LLA_ERR_NULL),
     (dict(out=0), _abi.LLA_ERR_NULL),
+    (dict(win_stream=0x1234), _abi.LLA_ERR_NULL),  # a window stream needs its fork/join events
     (dict(lat_dtype=7), _abi.LLA_ERR_DTYPE),
     (dict(win_dtype=-1), _abi.LLA_ERR_DTYPE),
     (dict(t0=2), _abi.LLA_ERR_SHAPE),            # t0 + nt > T

@@ -483,3 +483,44 @@ def test_several_query_positions(cuda_device, case):
                                          N, W, r_k, r_v, d_h, BASE, rotate_query=rotate) for b in range(B)])
     err = assert_rows_close(out, ref, TOL_BF16, f"multi-query {case}")
     print(f"multi-query {case}: rel L2 (pooled, worst row) {err}")
+
+
+# ------------------------------------------ window on a second stream --
+@pytest.mark.parametrize("W,N", [(128, 700), (16, 300), (0, 200)])
+def test_window_stream_bit_identical(cuda_device, W, N):
+    """The exact window on the caller's second stream (fork and join events)
+    gives the bits of the single-stream call, eagerly and replayed from a
+    captured graph."""
+    g = _gen(90 + W)
+    B, H, nt, t0, d_h, r_k, r_v = 3, 16, 3, 1, 128, 512, 512
+    T = t0 + nt
+    dev = cuda_device
+    lat = (torch.randn(B, N, r_k + r_v, generator=g) * math.sqrt(d_h / r_k)).to(torch.bfloat16).to(dev)
+    A = (torch.randn(nt, H, d_h, r_k, generator=g) / math.sqrt(d_h)).to(dev)
+    Bm = (torch.randn(nt, H, r_v, d_h, generator=g) / math.sqrt(r_v)).to(dev)
+    q = torch.randn(B, nt, H, d_h, generator=g).to(dev)
+    wk = torch.randn(B, T, W + 1, H, d_h, generator=g).to(torch.bfloat16).to(dev)
+    wv = torch.randn(B, T, W + 1, H, d_h, generator=g).to(torch.bfloat16).to(dev)
+    kw = dict(lat=lat, A=A, Bm=Bm, q=q, win_k=wk, win_v=wv, N=N, W=W, t0=t0, rotate_query=True, rope_base=BASE)
+    ref = torch.full((B, nt, H, d_h), float("nan"), device=dev)
+    L.hla_decode_attn(out=ref, **kw)
+    side = torch.cuda.Stream(dev)
+    evs = (torch.cuda.Event(), torch.cuda.Event())
+    for ev in evs:
+        ev.record()
+    out = torch.full_like(ref, float("nan"))
+    L.hla_decode_attn(out=out, win_stream=side, win_events=evs, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    # the same call captured and replayed (fork and join become graph edges)
+    s = torch.cuda.Stream(dev)
+    ws = torch.empty(L.hla_decode_workspace_bytes(out=out, **kw), dtype=torch.uint8, device=dev)
+    out2 = torch.full_like(ref, float("nan"))
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        L.hla_decode_attn(out=out2, workspace=ws, stream=s, win_stream=side, win_events=evs, **kw)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out2, ref)
+    del graph
