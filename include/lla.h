@@ -36,7 +36,10 @@
  *             are launched with programmatic dependent launch: a kernel's
  *             set-up may overlap the end of the previous kernel on the
  *             stream, and it touches global memory only once that kernel
- *             has completed, so stream order is kept.
+ *             has completed, so stream order is kept.  LLA_READ_SPLITS=S
+ *             (read at each plan) fixes the number of context splits of the
+ *             tensor-core latent read instead of the planner's choice; it
+ *             changes the workspace size, so set it before any size query.
  * Threads.    Calls from several host threads are safe, each with its own
  *             workspace.  The exception is hla_decode_attn_noalloc: all of its
  *             calls share one scratch array, so calls whose work may overlap

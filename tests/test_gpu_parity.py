@@ -129,6 +129,21 @@ def test_absorbed_read_bf16(cuda_device, case, rotate):
     print(f"absorbed {case} rotate={rotate}: rel L2 (pooled, worst row) {err}")
 
 
+@pytest.mark.parametrize("splits", [1, 2, 5, 16])
+def test_absorbed_read_split_count(cuda_device, monkeypatch, splits):
+    """The tensor-core read with the planner's split count forced: one split
+    (no merge of partials), a few, and more than the context has tiles (the
+    count is capped at one tile per split)."""
+    monkeypatch.setenv("LLA_READ_SPLITS", str(splits))
+    for case in (ABSORBED_CASES[0], ABSORBED_CASES[4]):
+        B, N, W, H, nt, d_h, r_k, r_v, Wcap = case
+        cs = _absorbed_case(1000 + N + H, B, N, W, H, nt, d_h, r_k, r_v, Wcap)
+        ref = _absorbed_oracle(cs, N, W, r_k, r_v, d_h, True)
+        got = _absorbed_gpu(cs, cuda_device, N, W, True)
+        err = assert_rows_close(got, ref, TOL_BF16, f"absorbed {case}, {splits} splits")
+        print(f"absorbed {case}, {splits} splits: rel L2 (pooled, worst row) {err}")
+
+
 def test_absorbed_read_fp32_latents(cuda_device):
     B, N, W, H, nt, d_h, r_k, r_v, Wcap = 2, 333, 16, 4, 2, 64, 128, 64, 20
     cs = _absorbed_case(77, B, N, W, H, nt, d_h, r_k, r_v, Wcap, lat_dtype=torch.float32)
