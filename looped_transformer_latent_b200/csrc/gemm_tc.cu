@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
   const int ne = KIND == KIND_OMAP ? a.NB + a.Sw : 0;            // partials per sequence
   const int cols_per = KIND == KIND_OMAP ? (BN + a.ks - 1) / a.ks : BN;
   const int col_lo = min(BN, ks * cols_per), col_hi = min(BN, col_lo + cols_per);
-  const bool yw_smem = KIND == KIND_OMAP && cols_per * GM * 4 <= YW_SMEM_MAX;
+  const bool yw_smem = KIND == KIND_OMAP && a.Sw > 0 && cols_per * GM * 4 <= YW_SMEM_MAX;
   float* wts = reinterpret_cast<float*>(misc + 16);                                       // [BN][ne + 1]
   float2* mls = reinterpret_cast<float2*>(misc + 16 + align8(BN * (ne + 1) * 4));         // [BN][ne]
   float* ywin_d = reinterpret_cast<float*>(misc + 16 + align8(BN * (ne + 1) * 4) + align16(BN * ne * 8));
@@ -343,41 +343,48 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
       }
       named_sync(1, NPROD);
       if (yw_smem) {
-        // float4 groups of 4 columns; per pass each thread keeps 4 groups and
-        // loops over the window chunks outermost, so its loads of a chunk are
-        // independent and in flight together
+        // float4 groups of 4 columns; each thread takes two groups at a time
+        // and issues the loads of up to eight window chunks of both before
+        // using any, so a pass costs one round trip to L2, not one per chunk
+        constexpr int WCB = 8;
         const int g4_hi = (col_hi - col_lo) * (GM / 4);
-        for (int base4 = 0; base4 < g4_hi; base4 += 4 * NPROD) {
-          float4 acc4[4];
-          int64_t off4[4];
-          bool live[4];
+        for (int base4 = 0; base4 < g4_hi; base4 += 2 * NPROD) {
+          float4 acc4[2];
+          int64_t off4[2];
+          bool live[2];
+          int bcol[2];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < 2; ++u) {
             const int idx4 = base4 + u * NPROD + tid;
             const int bb = col_lo + idx4 / (GM / 4), mm = 4 * (idx4 % (GM / 4));
             const int n = t.n0 + bb, m = t.m0 + mm;
             live[u] = idx4 < g4_hi && n < t.Nv && m < t.Mv;
             off4[u] = live[u] ? ((int64_t)n * a.rows + t.g) * a.Mtot + m : 0;
+            bcol[u] = idx4 < g4_hi ? bb : col_lo;
             acc4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
           }
-          for (int cw = 0; cw < a.Sw; ++cw) {
-            float4 v4[4];
+          for (int c0 = 0; c0 < a.Sw; c0 += WCB) {
+            float4 v4[2][WCB];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-              v4[u] = live[u] ? *reinterpret_cast<const float4*>(a.win_y + cw * bstride * a.Mtot + off4[u])
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < WCB; ++j)
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int idx4 = base4 + u * NPROD + tid;
-              const float w = live[u] ? wts[(col_lo + idx4 / (GM / 4)) * ld + a.NB + cw] : 0.f;
-              acc4[u].x = fmaf(w, v4[u].x, acc4[u].x);
-              acc4[u].y = fmaf(w, v4[u].y, acc4[u].y);
-              acc4[u].z = fmaf(w, v4[u].z, acc4[u].z);
-              acc4[u].w = fmaf(w, v4[u].w, acc4[u].w);
-            }
+              for (int u = 0; u < 2; ++u)
+                v4[u][j] = live[u] && c0 + j < a.Sw
+                               ? *reinterpret_cast<const float4*>(a.win_y + (c0 + j) * bstride * a.Mtot + off4[u])
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < WCB; ++j)
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const float w = live[u] && c0 + j < a.Sw ? wts[bcol[u] * ld + a.NB + c0 + j] : 0.f;
+                acc4[u].x = fmaf(w, v4[u][j].x, acc4[u].x);
+                acc4[u].y = fmaf(w, v4[u][j].y, acc4[u].y);
+                acc4[u].z = fmaf(w, v4[u][j].z, acc4[u].z);
+                acc4[u].w = fmaf(w, v4[u][j].w, acc4[u].w);
+              }
           }
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < 2; ++u) {
             const int idx4 = base4 + u * NPROD + tid;
             if (idx4 < g4_hi) reinterpret_cast<float4*>(ywin_d)[idx4] = acc4[u];
           }
@@ -584,13 +591,32 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
       const int ld = ne + 1;
       const bool bad = *abort_flag || (a.err && *a.err);
       const uint32_t ps_addr = smem_u32(part_s);
-      for (int idx = col_lo * GM + tid; idx < col_hi * GM; idx += NPROD) {
-        const int bb = idx / GM, mm = idx % GM;
-        const int n = t.n0 + bb, m = t.m0 + mm;
-        float y = ywin_d[idx - col_lo * GM];
-        for (int rk = 0; rk < a.ks; ++rk) y += ld_shared_cluster(mapa_shared(ps_addr + 4u * idx, (uint32_t)rk));
-        if (m < t.Mv && n < t.Nv)
-          a.out[(int64_t)n * a.outs_b + (int64_t)t.g * a.Mtot + m] = bad ? NAN : y * wts[bb * ld + ne];
+      // four elements per thread at a time, all their remote loads issued
+      // before any is summed (in rank order, as before)
+      constexpr int EU = 4;
+      for (int idx0 = col_lo * GM + tid; idx0 < col_hi * GM; idx0 += EU * NPROD) {
+        float r[EU][4];
+#pragma unroll
+        for (int u = 0; u < EU; ++u) {
+          const int idx = idx0 + u * NPROD;
+#pragma unroll
+          for (int rk = 0; rk < 4; ++rk)
+            r[u][rk] = idx < col_hi * GM && rk < a.ks ? ld_shared_cluster(mapa_shared(ps_addr + 4u * idx, (uint32_t)rk))
+                                                      : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < EU; ++u) {
+          const int idx = idx0 + u * NPROD;
+          if (idx >= col_hi * GM) break;
+          const int bb = idx / GM, mm = idx % GM;
+          const int n = t.n0 + bb, m = t.m0 + mm;
+          float y = yw_smem ? ywin_d[idx - col_lo * GM] : 0.f;
+#pragma unroll
+          for (int rk = 0; rk < 4; ++rk)
+            if (rk < a.ks) y += r[u][rk];
+          if (m < t.Mv && n < t.Nv)
+            a.out[(int64_t)n * a.outs_b + (int64_t)t.g * a.Mtot + m] = bad ? NAN : y * wts[bb * ld + ne];
+        }
       }
     }
     // no CTA leaves while a neighbour may still read its partial tile
@@ -611,17 +637,39 @@ cudaError_t launch_one(const TcMaps& maps, TcGemmArgs a, int grid_y, int nb, siz
   int misc = 0;
   if (KIND == KIND_OMAP) {
     const int ne = nb + a.Sw, cols_per = (BN + a.ks - 1) / a.ks;
-    misc = align8(BN * (ne + 1) * 4) + align16(BN * ne * 8) + (cols_per * GM * 4 <= YW_SMEM_MAX ? cols_per * GM * 4 : 0);
+    misc = align8(BN * (ne + 1) * 4) + align16(BN * ne * 8) +
+           (a.Sw > 0 && cols_per * GM * 4 <= YW_SMEM_MAX ? cols_per * GM * 4 : 0);
   }
-  // stages: 2 to 6, as many as the budget allows (16 bytes for aligning the misc region)
+  // stages: 2 to 6, as many as the budget allows (16 bytes for aligning the
+  // misc region), and no more than a CTA's k-chunks of the maps: a stage that
+  // is never filled only keeps other CTAs off the SM
   const size_t fixed = 1024 + 16 + 16 + misc + 8;
-  int nst = 2;
-  while (nst < 6 && fixed + (size_t)(nst + 1) * (stage + 24) <= smem_budget) ++nst;
+  const int nk = (a.K + KCH - 1) / KCH;
+  const int cta_chunks = KIND == KIND_QMAP ? nk : KIND == KIND_OMAP ? (nk + a.ks - 1) / a.ks : 6;
+  auto plan = [&](size_t budget) {
+    auto fits = [&](int n) { return fixed + (size_t)n * (stage + 24) <= budget; };
+    int n = 2;
+    while (n < 6 && n < cta_chunks && fits(n + 1)) ++n;
+    // a cluster k-split keeps its partial tile in the stage memory
+    while (KIND == KIND_OMAP && a.ks > 1 && (size_t)BN * GM * 4 > (size_t)n * stage && n < 6 && fits(n + 1)) ++n;
+    return n;
+  };
+  int nst = plan(smem_budget);
+  // the output map runs beside the window and the other group's kernels:
+  // two CTAs per SM when that still leaves three stages (or all its chunks)
+  const size_t half = (size_t)SMEM_MAX / 2 - 1024;
+  if (KIND == KIND_OMAP && smem_budget > half) {
+    const int n2 = plan(half);
+    if (n2 >= std::min(3, cta_chunks) && fixed + (size_t)n2 * stage + 8 * (3 * n2 + 1) <= half &&
+        !(a.ks > 1 && (size_t)BN * GM * 4 > (size_t)n2 * stage))
+      nst = n2;
+  }
   a.nst = nst;
   // with a cluster k-split, the partial tile reuses the stages
   if (KIND == KIND_OMAP && a.ks > 1 && (size_t)BN * GM * 4 > (size_t)nst * stage) return cudaErrorNotSupported;
   // a cluster k-split needs the window term of its slice in shared memory
-  if (KIND == KIND_OMAP && a.ks > 1 && ((BN + a.ks - 1) / a.ks) * GM * 4 > YW_SMEM_MAX) return cudaErrorNotSupported;
+  if (KIND == KIND_OMAP && a.ks > 1 && a.Sw > 0 && ((BN + a.ks - 1) / a.ks) * GM * 4 > YW_SMEM_MAX)
+    return cudaErrorNotSupported;
   size_t smem = fixed + (size_t)nst * stage + 8 * (3 * nst + 1);
   // keep the CTAs an SM can hold (228 KB of shared memory, 1 KB reserved per
   // CTA) within its 512 TMEM columns, so that no allocation ever waits
