@@ -426,9 +426,12 @@ int hla_decode_attn(const hla_decode_params* p, void* ws, size_t ws_bytes, lla_s
   qm.q_f16 = a.lat_dtype == LLA_FP8_E4M3 && a.use_tc;   // no latent token: the operand is unused
   qm.qlat = a.qlat; qm.qbf = a.qbf;
   cudaError_t e = cudaSuccess;
-  e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
   // optional: the window on the caller's second stream, beside the map and the read
   const cudaStream_t sw = p->win_stream ? static_cast<cudaStream_t>(p->win_stream) : s;
+  // the error word is cleared by the query map, the call's first kernel, unless
+  // the window runs on its own stream beside it: then by a memset before both
+  if (sw != s) e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
+  else qm.clear_err = a.err;
   cudaEvent_t* wev = reinterpret_cast<cudaEvent_t*>(p->win_events);
   if (e == cudaSuccess && sw != s) {
     e = cudaEventRecord(wev[0], s);

@@ -163,6 +163,12 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the query map opens the call: it clears the call's error word, which the
+  // kernels after it write (its own timeouts also turn its output into NaN)
+  if (KIND == KIND_QMAP && a.clear_err && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) {
+    griddep_wait();
+    *a.clear_err = 0;
+  }
 
   // ---- tile ------------------------------------------------------------
   Tile t;
@@ -298,6 +304,16 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
   float* part_s = reinterpret_cast<float*>(base);                          // [BN][GM]
 
   if (warp < NPROD / 32) {
+    // query map: the rotation of this thread's codec row (TMEM lane) for the
+    // epilogue, computed while the first stage is in flight
+    float cq = 1.f, sq = 0.f;
+    if (KIND == KIND_QMAP && a.rotate) {
+      const int mr = t.m0 + 32 * (warp & 3) + lane;
+      if (mr < t.Mv) {
+        const int pos = a.pos + (a.rows_per_q > 0 ? t.g / a.rows_per_q : 0);   // this row's query position
+        rope_cs(mr >> 1, a.Mtot, a.d_h, a.base, (double)pos, &cq, &sq);
+      }
+    }
     // ---- converters: round each landed stage to tf32 in place ---------------
     // (the hi and lo tiles share one layout, so pieces are plain 16-byte slots)
     auto convert = [&](uint32_t addr, uint32_t lo_addr) {
@@ -430,11 +446,6 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
         for (int i = 0; i < 16; ++i) v[i] += w[i];
       }
     };
-    float cq = 1.f, sq = 0.f;
-    if (KIND == KIND_QMAP && a.rotate && m < t.Mv) {
-      const int pos = a.pos + (a.rows_per_q > 0 ? t.g / a.rows_per_q : 0);   // this row's query position
-      rope_cs(m >> 1, a.Mtot, a.d_h, a.base, (double)pos, &cq, &sq);
-    }
     const bool bad = !ok || (KIND == KIND_OMAP && a.err && *a.err);
 #pragma unroll 1
     for (int c = half * (BN / 32); c < (half + 1) * (BN / 32); ++c) {
@@ -781,6 +792,7 @@ cudaError_t launch_query_map_tc(const MapArgs& g, int* err, cudaStream_t st) {
   a.Aw = g.W; a.X = g.X; a.xs_b = g.xs_b;
   a.rotate = g.rotate; a.pos = g.pos; a.d_h = g.d_h; a.base = g.base; a.qmul = g.qmul; a.qbf = g.qbf;
   a.qf16 = g.q_f16;
+  a.clear_err = g.clear_err;
   a.ncodec = g.ncodec > 0 ? g.ncodec : g.rows;
   a.rows_per_q = g.rows_per_q;
   a.err = err; a.NB = 1; a.S = 1; a.ks = 1;

@@ -150,6 +150,7 @@ struct MapArgs {
   float* out;
   int64_t outs_b;
   const int* err;
+  int* clear_err;          // query map: set to 0 before any later kernel of the call reads it (null: no)
 };
 int map_max_splits();
 cudaError_t launch_query_map(const MapArgs& g, cudaStream_t st);
@@ -173,6 +174,7 @@ struct TcGemmArgs {
   float* out;
   int64_t outs_b;
   int* err;
+  int* clear_err;          // query map: the call's error word, cleared by one thread (null: no)
   WriterArgs w;            // writer slices
 };
 bool query_map_tc_ok(const MapArgs& g);

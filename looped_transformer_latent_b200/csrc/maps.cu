@@ -30,6 +30,10 @@ __device__ __forceinline__ int64_t qbf_index(int b, int row, int k, int r_k) {
 template <int MODE, int GB, int GK>
 __global__ void __launch_bounds__(GT) row_gemm(MapArgs g) {
   griddep_wait();
+  // the query map opens the call: it clears the call's error word, which only
+  // the kernels after it write
+  if (MODE == 0 && g.clear_err && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0)
+    *g.clear_err = 0;
   constexpr int BPW = GB / (GT / 32);   // sequences per warp
   constexpr int LX = GB * GK / GT;      // activation loads per thread
   __shared__ float Xs[2][GK][GB + 1];
