@@ -236,7 +236,13 @@ HlaPlan plan_hla(const hla_decode_params& p) {
   pl.rows_pad = pl.use_tc ? absorb_tc_rows_pad(pl.rows) : pl.rows;
   if (pl.use_tc) {
     // tensor-core read: one CTA per (split, sequence), 64-token tiles
-    const int S = absorb_tc_splits(p.B, pl.n_lat, sms);
+    // LLA_READ_SPLITS overrides the planner's split count (tuning and tests;
+    // it sizes the workspace too, so set it before the first size query)
+    int S = absorb_tc_splits(p.B, pl.n_lat, sms);
+    if (const char* env = std::getenv("LLA_READ_SPLITS")) {
+      const int v = std::atoi(env);
+      if (v >= 1) S = std::min(v, std::min((pl.n_lat + 63) / 64, 16));
+    }
     pl.tps = (int)(((pl.n_lat + S - 1) / S + 63) / 64 * 64);
     pl.S = (pl.n_lat + pl.tps - 1) / pl.tps;
   } else if (pl.n_lat > 0) {

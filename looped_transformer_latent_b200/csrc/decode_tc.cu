@@ -26,7 +26,6 @@
 // mbarrier wait is bounded; on timeout the CTA records an error code in the
 // workspace (the merge then emits NaN), drains its copies and frees TMEM.
 #include <cuda.h>
-#include <cstdlib>
 
 #include "kernels.cuh"
 #include "tc_ptx.cuh"
@@ -446,14 +445,8 @@ bool absorb_tc_supported(int lat_dtype, int r_k, int r_v, int rows) {
 
 int absorb_tc_splits(int B, int n_lat, int num_sms) {
   // pick the split count with the smallest modelled time: waves of one CTA per
-  // SM, each CTA streaming ceil(tiles / S) tiles plus a fixed start-up cost.
-  // LLA_READ_SPLITS overrides it (tuning and tests; it sizes the workspace
-  // too, so set it before the first call of the process)
+  // SM, each CTA streaming ceil(tiles / S) tiles plus a fixed start-up cost
   const int tiles = (n_lat + TOK - 1) / TOK;
-  if (const char* env = std::getenv("LLA_READ_SPLITS")) {
-    const int v = std::atoi(env);
-    if (v >= 1) return std::max(1, std::min(v, std::min(tiles, 16)));
-  }
   int best = 1;
   double best_t = 1e300;
   for (int S = 1; S <= 16 && S <= tiles; ++S) {
