@@ -666,8 +666,9 @@ cudaError_t launch_one(const TcMaps& maps, TcGemmArgs a, int grid_y, int nb, siz
     return n;
   };
   int nst = plan(smem_budget);
-  // the output map runs beside the window and the other group's kernels:
-  // two CTAs per SM when that still leaves three stages (or all its chunks)
+  // the output map runs beside the window and the other group's kernels: at
+  // most half an SM's shared memory when that still leaves three stages (or
+  // all its chunks); measured faster than the full budget on batch-32 calls
   const size_t half = (size_t)SMEM_MAX / 2 - 1024;
   if (KIND == KIND_OMAP && smem_budget > half) {
     const int n2 = plan(half);
