@@ -108,6 +108,23 @@ def test_hla_workspace_checks(lib):
     assert lib.hla_decode_workspace_bytes(ctypes.byref(_hla(N=0))) == 0
 
 
+def test_read_split_override_sizes_the_workspace(lib, monkeypatch):
+    # LLA_READ_SPLITS fixes the latent read's context splits: each split keeps
+    # (max, sum) and an r_V-wide partial per (sequence, row) in fp32, and the
+    # count is capped at one 64-token tile per split (here 83 latent tokens: 2)
+    p = _hla()
+    rows = p.nt * p.H
+    per_split = p.B * rows * p.r_v * 4      # the r_V-wide partials (the (max, sum) pairs share an aligned block)
+    need = {}
+    for v in ("1", "2", "50"):
+        monkeypatch.setenv("LLA_READ_SPLITS", v)
+        need[v] = lib.hla_decode_workspace_bytes(ctypes.byref(p))
+    monkeypatch.delenv("LLA_READ_SPLITS")
+    assert need["2"] - need["1"] >= per_split
+    assert need["50"] == need["2"]
+    assert lib.hla_decode_workspace_bytes(ctypes.byref(p)) > 0
+
+
 def test_empty_batch_is_a_no_op(lib):
     # B = 0 or nt = 0: nothing to do, null pointers allowed, no workspace
     p = _hla(B=0, lat=0, A=0, Bm=0, q=0, win_k=0, win_v=0, out=0)
