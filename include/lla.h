@@ -40,6 +40,9 @@
  *             (read at each plan) fixes the number of context splits of the
  *             tensor-core latent read instead of the planner's choice; it
  *             changes the workspace size, so set it before any size query.
+ *             LLA_RECON_SEQ_PER_CTA=n fixes how many sequences one CTA of
+ *             the tensor-core reconstruct walks (lla_decode_attn).  Both are
+ *             for tuning and tests; unset, the planners choose.
  * Threads.    Calls from several host threads are safe, each with its own
  *             workspace.  The exception is hla_decode_attn_noalloc: all of its
  *             calls share one scratch array, so calls whose work may overlap
