@@ -102,7 +102,7 @@ typedef enum {
   LLA_ERR_DTYPE = 3,       /* unknown dtype code                             */
   LLA_ERR_ALIGN = 4,       /* a pointer or stride breaks 16-byte alignment   */
   LLA_ERR_WORKSPACE = 5,   /* ws is NULL, misaligned or smaller than needed  */
-  LLA_ERR_UNSUPPORTED = 6, /* valid, but a combination this build rejects    */
+  LLA_ERR_UNSUPPORTED = 6, /* valid, but a combination the library rejects  */
   LLA_ERR_CUDA = 7         /* a CUDA runtime call or launch failed           */
 } lla_status;
 

@@ -356,7 +356,7 @@ const char* lla_status_str(int s) {
     case LLA_ERR_DTYPE: return "unknown dtype code";
     case LLA_ERR_ALIGN: return "pointer or stride breaks the 16-byte alignment rule";
     case LLA_ERR_WORKSPACE: return "workspace is NULL, misaligned or too small";
-    case LLA_ERR_UNSUPPORTED: return "valid arguments outside what this build supports";
+    case LLA_ERR_UNSUPPORTED: return "valid arguments outside what the library supports";
     case LLA_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
     default: return "unknown status";
   }
