@@ -603,7 +603,7 @@ __global__ void __launch_bounds__(NTHR, 1) tc_gemm(const __grid_constant__ TcMap
       const bool bad = *abort_flag || (a.err && *a.err);
       const uint32_t ps_addr = smem_u32(part_s);
       // four elements per thread at a time, all their remote loads issued
-      // before any is summed (in rank order, as before)
+      // before any is summed, in rank order (the launcher keeps ks <= 4)
       constexpr int EU = 4;
       for (int idx0 = col_lo * GM + tid; idx0 < col_hi * GM; idx0 += EU * NPROD) {
         float r[EU][4];
